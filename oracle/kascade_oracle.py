@@ -1,0 +1,287 @@
+"""Kascade oracle: a plain, slow fp64 CPU statement of head-aware, cross-layer
+reused Top-k sparse attention.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports this module:
+only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` use it.  It shares no code with the CUDA library.
+
+Sources (page "A Practical Sparse Attention Method for Long-Context LLM
+Inference", the Kascade README):
+
+* Abstract: post-softmax attention is sparse; exact Top-k indices are computed
+  in a few *anchor* layers and reused by the *reuse* layers in between;
+  selection and reuse are head-aware; operations are tile-level in prefill and
+  decode.
+* "Running Evaluations and Performance Benchmarks": the selection strategy is
+  ``post_softmax_pooled_prefill_topk`` and the efficient kernels use
+  ``tile_size 32``; the figure caption under the Abstract and the ``--topk 10``
+  / ``k=10`` arguments ("Kernel Benchmarks", "Python API") give the budget as a
+  percentage of the context.
+
+Readings of what the page leaves open (each one is listed in the design doc):
+
+* scores are q.k / sqrt(d) with no bias (standard scaled dot product);
+* query head qh belongs to kv head qh // G (contiguous GQA groups);
+* "pooled" = the mean of post-softmax probabilities over the G query heads of
+  a kv head and, in prefill, over the rows of one query tile; masked
+  (future) entries count as 0 and the mean is over all G*rows entries;
+* k = ceil(frac * e) computed in integers, frac = num/den; e = the number of
+  candidate keys (decode: N; prefill tile t: min(tile*(t+1), N));
+* the k largest pooled values win; equal values go to the lower key index;
+  index lists are reported in ascending order;
+* decode: the single query sees all N cached keys;
+* prefill: the candidates of tile t are keys [0, e_t); row i attends only to
+  selected keys j <= i; a row that sees no selected key outputs 0 with
+  log-sum-exp -inf;
+* a reuse kv head h reads the index set of anchor head head_map[h].
+
+Everything is computed in float64 from the exact values of the (bf16) inputs.
+Array layout: q [B, Hq, L, d], k/v [B, Hkv, N, d] (L = 1 in decode).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+F64 = np.float64
+
+__all__ = [
+    "topk_count", "tile_ends", "tile_topk_counts", "index_offsets",
+    "scores", "masked_softmax", "pooled_decode", "pooled_prefill_tile",
+    "select_topk", "anchor_select_decode", "anchor_select_prefill_tile",
+    "sparse_attend", "sparse_decode", "sparse_prefill_tile", "dense_attention",
+    "check_index_set",
+]
+
+
+# ---------------------------------------------------------------------------
+# budgets and tiles
+
+
+def topk_count(e: int, frac_num: int, frac_den: int) -> int:
+    """k = ceil(frac * e) with frac = frac_num / frac_den, in exact integers.
+
+    The README gives the budget as a percentage ("Top-k set to 10%", Abstract
+    figure caption; ``--topk 10``, Kernel Benchmarks)."""
+    if e <= 0:
+        return 0
+    return -((-frac_num * e) // frac_den)
+
+
+def tile_ends(n_ctx: int, tile: int) -> list[int]:
+    """e_t = min(tile*(t+1), N) for t = 0..ceil(N/tile)-1: the keys that the
+    last row of query tile t can see (tile-level prefill, README Abstract)."""
+    n_tiles = -(-n_ctx // tile)
+    return [min(tile * (t + 1), n_ctx) for t in range(n_tiles)]
+
+
+def tile_topk_counts(n_ctx: int, tile: int, frac_num: int, frac_den: int) -> list[int]:
+    """k_t for every prefill tile."""
+    return [topk_count(e, frac_num, frac_den) for e in tile_ends(n_ctx, tile)]
+
+
+def index_offsets(n_ctx: int, tile: int, frac_num: int, frac_den: int) -> np.ndarray:
+    """Start of each tile's index list in a ragged [sum_t k_t] row (plus the
+    total at the end)."""
+    ks = tile_topk_counts(n_ctx, tile, frac_num, frac_den)
+    out = np.zeros(len(ks) + 1, dtype=np.int64)
+    out[1:] = np.cumsum(ks)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# scores, softmax, pooling
+
+
+def scores(q_rows: np.ndarray, k_rows: np.ndarray) -> np.ndarray:
+    """s[r, j] = q_r . k_j / sqrt(d) in float64."""
+    q64 = np.asarray(q_rows, dtype=F64)
+    k64 = np.asarray(k_rows, dtype=F64)
+    return (q64 @ k64.T) / math.sqrt(q64.shape[-1])
+
+
+def masked_softmax(s: np.ndarray, visible: np.ndarray) -> np.ndarray:
+    """Row softmax over the visible entries; invisible entries are 0.  A row
+    with nothing visible is all zeros."""
+    s = np.where(visible, s, -np.inf)
+    m = np.max(s, axis=-1, keepdims=True)
+    m = np.where(np.isfinite(m), m, 0.0)
+    p = np.where(visible, np.exp(s - m), 0.0)
+    den = p.sum(axis=-1, keepdims=True)
+    return np.divide(p, den, out=np.zeros_like(p), where=den > 0)
+
+
+def pooled_decode(q: np.ndarray, k: np.ndarray, b: int, h: int) -> np.ndarray:
+    """Pooled post-softmax scores of kv head h for one decode query.
+
+    P[j] = (1/G) sum_g softmax_j(q_{hG+g} . k_j / sqrt(d)), j < N."""
+    hq, hkv = q.shape[1], k.shape[1]
+    g_size = hq // hkv
+    q_rows = q[b, h * g_size:(h + 1) * g_size, 0, :]
+    s = scores(q_rows, k[b, h])
+    p = masked_softmax(s, np.ones_like(s, dtype=bool))
+    return p.mean(axis=0)
+
+
+def pooled_prefill_tile(q: np.ndarray, k: np.ndarray, b: int, h: int, t: int,
+                        tile: int) -> np.ndarray:
+    """Pooled post-softmax scores of kv head h over query tile t.
+
+    Rows are the G heads x the tile's query positions i; candidates are keys
+    j < e_t; row i sees j <= i.  P[j] = sum over rows of p[r, j] divided by
+    G * rows_t (rows_t = the tile's real rows)."""
+    hq, hkv, n_ctx = q.shape[1], k.shape[1], k.shape[2]
+    g_size = hq // hkv
+    i0 = t * tile
+    i1 = min(i0 + tile, n_ctx)
+    e_t = i1
+    pos = np.arange(i0, i1)
+    total = np.zeros(e_t, dtype=F64)
+    for g in range(g_size):
+        s = scores(q[b, h * g_size + g, i0:i1, :], k[b, h, :e_t, :])
+        visible = np.arange(e_t)[None, :] <= pos[:, None]
+        total += masked_softmax(s, visible).sum(axis=0)
+    return total / (g_size * (i1 - i0))
+
+
+# ---------------------------------------------------------------------------
+# Top-k
+
+
+def select_topk(pooled: np.ndarray, k: int) -> np.ndarray:
+    """The k largest pooled values, equal values going to the lower index,
+    returned as ascending indices."""
+    n = pooled.shape[0]
+    order = np.lexsort((np.arange(n), -np.asarray(pooled, dtype=F64)))
+    return np.sort(order[:k]).astype(np.int64)
+
+
+def anchor_select_decode(q: np.ndarray, k: np.ndarray, frac_num: int, frac_den: int):
+    """Anchor decode layer: idx [B, Hkv, kk] (ascending) and pooled [B, Hkv, N]."""
+    bsz, hkv, n_ctx = k.shape[0], k.shape[1], k.shape[2]
+    kk = topk_count(n_ctx, frac_num, frac_den)
+    idx = np.zeros((bsz, hkv, kk), dtype=np.int64)
+    pooled = np.zeros((bsz, hkv, n_ctx), dtype=F64)
+    for b in range(bsz):
+        for h in range(hkv):
+            pooled[b, h] = pooled_decode(q, k, b, h)
+            idx[b, h] = select_topk(pooled[b, h], kk)
+    return idx, pooled
+
+
+def anchor_select_prefill_tile(q, k, b, h, t, tile, frac_num, frac_den):
+    """Anchor prefill, one (b, h, t) problem: (ascending idx of k_t keys, pooled)."""
+    pooled = pooled_prefill_tile(q, k, b, h, t, tile)
+    return select_topk(pooled, topk_count(pooled.shape[0], frac_num, frac_den)), pooled
+
+
+# ---------------------------------------------------------------------------
+# sparse attention over a selected set
+
+
+def sparse_attend(q_rows: np.ndarray, k_rows: np.ndarray, v_rows: np.ndarray,
+                  visible: np.ndarray):
+    """o_r = sum_j softmax_j(q_r . k_j / sqrt(d)) v_j over the visible j, with
+    log-sum-exp lse_r of the scaled scores.  Rows with nothing visible give
+    o = 0 and lse = -inf."""
+    s = scores(q_rows, k_rows)
+    p = masked_softmax(s, visible)
+    o = p @ np.asarray(v_rows, dtype=F64)
+    s_vis = np.where(visible, s, -np.inf)
+    m = np.max(s_vis, axis=-1)
+    has = np.isfinite(m)
+    m0 = np.where(has, m, 0.0)
+    with np.errstate(divide="ignore"):
+        lse = np.where(has, m0 + np.log(np.where(visible, np.exp(s_vis - m0[:, None]), 0.0).sum(-1)),
+                       -np.inf)
+    return o, lse
+
+
+def sparse_decode(q, k, v, idx, head_map=None):
+    """Reuse (or anchor) decode layer.  kv head h attends over the set
+    idx[b, head_map[h]]; head_map None means identity.
+
+    Returns o [B, Hq, d] and lse [B, Hq] (natural log of the softmax
+    denominator of the scaled scores)."""
+    bsz, hq, _, d = q.shape
+    hkv = k.shape[1]
+    g_size = hq // hkv
+    hm = np.arange(hkv) if head_map is None else np.asarray(head_map)
+    o = np.zeros((bsz, hq, d), dtype=F64)
+    lse = np.zeros((bsz, hq), dtype=F64)
+    for b in range(bsz):
+        for h in range(hkv):
+            sel = np.asarray(idx[b, hm[h]], dtype=np.int64)
+            rows = q[b, h * g_size:(h + 1) * g_size, 0, :]
+            vis = np.ones((g_size, sel.shape[0]), dtype=bool)
+            ob, lb = sparse_attend(rows, k[b, h, sel], v[b, h, sel], vis)
+            o[b, h * g_size:(h + 1) * g_size] = ob
+            lse[b, h * g_size:(h + 1) * g_size] = lb
+    return o, lse
+
+
+def sparse_prefill_tile(q, k, v, sel, b, h, t, tile):
+    """Reuse (or anchor) prefill, one (b, h, t) problem over the selected set
+    ``sel`` (the anchor head's list for tile t).  Row i of the tile sees the
+    selected keys j <= i.  Returns o [G, rows_t, d] and lse [G, rows_t]."""
+    hq, hkv, n_ctx = q.shape[1], k.shape[1], k.shape[2]
+    g_size = hq // hkv
+    i0 = t * tile
+    i1 = min(i0 + tile, n_ctx)
+    sel = np.asarray(sel, dtype=np.int64)
+    pos = np.arange(i0, i1)
+    vis = sel[None, :] <= pos[:, None]
+    o = np.zeros((g_size, i1 - i0, q.shape[-1]), dtype=F64)
+    lse = np.zeros((g_size, i1 - i0), dtype=F64)
+    for g in range(g_size):
+        o[g], lse[g] = sparse_attend(q[b, h * g_size + g, i0:i1, :], k[b, h, sel], v[b, h, sel], vis)
+    return o, lse
+
+
+def dense_attention(q_rows, k_rows, v_rows, row_pos=None):
+    """Dense attention of q_rows over all keys (row_pos None) or causally
+    (key j visible to the row at position row_pos[r] iff j <= row_pos[r])."""
+    n = k_rows.shape[0]
+    if row_pos is None:
+        vis = np.ones((q_rows.shape[0], n), dtype=bool)
+    else:
+        vis = np.arange(n)[None, :] <= np.asarray(row_pos)[:, None]
+    return sparse_attend(q_rows, k_rows, v_rows, vis)
+
+
+# ---------------------------------------------------------------------------
+# acceptance rule for a selected set
+
+
+def check_index_set(pooled: np.ndarray, k: int, got, rel: float = 1e-6) -> str:
+    """Judge an index set against the oracle's pooled values.
+
+    Let tau_k, tau_k1 be the k-th and (k+1)-th largest pooled values.  If
+    tau_k - tau_k1 > rel * tau_k the set must equal the oracle's exactly
+    ("exact").  Otherwise (a near tie) it passes ("near_tie") when it holds
+    every j with P_j > tau_k (1 + rel) and all of its other members lie
+    within rel * tau_k of tau_k.  Anything else is "fail".  The set must also
+    be strictly ascending with k members in range."""
+    pooled = np.asarray(pooled, dtype=F64)
+    got = np.asarray(got, dtype=np.int64)
+    n = pooled.shape[0]
+    if got.shape[0] != k or (k > 0 and (got.min() < 0 or got.max() >= n)):
+        return "fail"
+    if k > 1 and not np.all(np.diff(got) > 0):
+        return "fail"
+    want = select_topk(pooled, k)
+    if np.array_equal(want, got):
+        return "exact"
+    srt = np.sort(pooled)[::-1]
+    tau_k = srt[k - 1]
+    tau_k1 = srt[k] if k < n else -np.inf
+    if tau_k - tau_k1 > rel * tau_k:
+        return "fail"
+    must = np.nonzero(pooled > tau_k * (1.0 + rel))[0]
+    if not np.all(np.isin(must, got)):
+        return "fail"
+    others = np.setdiff1d(got, must)
+    if np.all(np.abs(pooled[others] - tau_k) <= rel * tau_k):
+        return "near_tie"
+    return "fail"
