@@ -1,0 +1,167 @@
+/*
+ * kascade.h -- C ABI of the Kascade head-aware, cross-layer-reused Top-k
+ * sparse attention library for NVIDIA B200 (sm_100a).
+ *
+ * The method (page "A Practical Sparse Attention Method for Long-Context LLM
+ * Inference", the Kascade README, Abstract): a few *anchor* layers compute
+ * exact post-softmax attention, pool it per kv head and pick exact Top-k key
+ * indices; the *reuse* layers in between attend only over the index set of an
+ * anchor head chosen by a per-layer head map.  Selection is tile-level in
+ * prefill (tile_size 32, README "Running Evaluations and Performance
+ * Benchmarks") and the budget is a fraction of the context ("Top-k set to
+ * 10%", Abstract figure caption).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Tensors are dense, row-major, bf16 unless stated:
+ *   q   [B, Hq,  L, d]   L = q_len (1 in decode, N in prefill)
+ *   k,v [B, Hkv, N, d]   one contiguous [N, d] slab per (batch, kv head)
+ *   o   [B, Hq,  L, d]   bf16 output
+ *   lse [B, Hq,  L]      fp32 natural-log softmax denominator of the scaled
+ *                        scores (may be NULL); -inf for a row that sees no key
+ * Query head qh belongs to kv head qh / G, G = Hq / Hkv.  Scores are
+ * q.k / sqrt(d).
+ *
+ * Index sets (int32, ascending within each list):
+ *   decode  idx [B, Hkv, K]          K = ceil(frac * N)
+ *   prefill idx [B, Hkv, S]          S = sum_t k_t, k_t = ceil(frac * e_t),
+ *                                    e_t = min(32 (t+1), N); the list of tile t
+ *                                    starts at offsets[t] (kascade_index_offsets)
+ *
+ * Ownership: the caller owns every buffer (device memory for tensors, index
+ * lists and the workspace; host memory for kascade_shape and offsets).  The
+ * library never allocates or frees memory and keeps no state between calls.
+ * All device work is enqueued on `stream` (a cudaStream_t; NULL = legacy
+ * default stream) and is asynchronous: results are ready when the stream is.
+ *
+ * Workspace: each call takes `ws`/`ws_bytes` of device scratch of at least
+ * kascade_workspace_bytes() bytes, 256-byte aligned.  Its first bytes hold
+ * per-(batch, kv head) ticket counters that the split-K kernels use to find
+ * the last CTA; they must be zero before the first call (zero-fill the whole
+ * workspace once with kascade_workspace_init) and every call leaves them zero
+ * again, so one workspace sized for the largest op can serve every call of a
+ * shape.  Calls that may run concurrently must not share a workspace.
+ *
+ * Errors: every call returns KASCADE_OK (0) or a status below; argument
+ * errors are detected on the host before anything is launched.  No kernel
+ * traps or waits on another kernel.
+ */
+#ifndef KASCADE_H_
+#define KASCADE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KASCADE_API __attribute__((visibility("default")))
+#else
+#define KASCADE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KASCADE_OK 0
+#define KASCADE_ERR_INVALID_ARG 1  /* null pointer, bad dims, Hq % Hkv != 0, frac outside (0,1] */
+#define KASCADE_ERR_UNSUPPORTED 2  /* d not 64/128, tile != 32, G > 8, q_len not 1 or N, misaligned pointer */
+#define KASCADE_ERR_WORKSPACE 3    /* ws NULL, misaligned or smaller than kascade_workspace_bytes() */
+#define KASCADE_ERR_CUDA 4         /* a CUDA launch or device query failed */
+
+/* Operations for kascade_workspace_bytes(). */
+#define KASCADE_OP_SELECT 0
+#define KASCADE_OP_SPARSE_DECODE 1
+#define KASCADE_OP_SPARSE_PREFILL 2
+#define KASCADE_OP_DENSE 3
+
+typedef struct kascade_shape {
+  int32_t batch;        /* B  >= 1 */
+  int32_t num_q_heads;  /* Hq >= 1, multiple of Hkv */
+  int32_t num_kv_heads; /* Hkv >= 1 */
+  int32_t head_dim;     /* d: 64 or 128 */
+  int32_t q_len;        /* 1 = decode; == kv_len = causal prefill */
+  int32_t kv_len;       /* N >= 1 (N <= 2^20) */
+  int32_t tile;         /* prefill query tile; must be 32 (ignored in decode) */
+  int32_t topk_num;     /* frac = topk_num / topk_den, 0 < frac <= 1, */
+  int32_t topk_den;     /*   e.g. 10/100 for the README's Top-k of 10 % */
+} kascade_shape;
+
+/* Bytes of workspace that `op` needs for `shape` (0 on an invalid shape). */
+KASCADE_API size_t kascade_workspace_bytes(const kascade_shape* shape, int op);
+
+/* Number of int32 entries of the index buffer: B * Hkv * K (decode) or
+ * B * Hkv * sum_t k_t (prefill).  Returns -1 on an invalid shape. */
+KASCADE_API int64_t kascade_index_count(const kascade_shape* shape);
+
+/* Host-side: writes T+1 int64 tile offsets (T = ceil(N/32)) of one
+ * (batch, kv head) index row to `offsets` (host memory, caller-owned);
+ * offsets[T] is the row length.  Decode shapes write {0, K}. */
+KASCADE_API int kascade_index_offsets(const kascade_shape* shape, int64_t* offsets);
+
+/* Zero-fills `ws_bytes` bytes of device workspace on `stream`. */
+KASCADE_API int kascade_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Anchor-layer selection (README Abstract: "exact Top-k indices ... in a
+ * small set of anchor layers"; strategy post_softmax_pooled_prefill_topk).
+ *
+ * For every (b, kv head h) in decode, or (b, h, query tile t) in prefill:
+ * softmax over the visible keys of every query row of h's G query heads,
+ * mean of those probabilities over the rows (masked entries count as 0),
+ * then the k (= ceil(frac * e)) keys with the largest pooled value among the
+ * candidates [0, e), equal values going to the lower index, written in
+ * ascending order to `idx` (layout above).  Selection is exact: near the
+ * k-th value the pooled scores are recomputed in fp64.
+ *   q, k  device, bf16, layouts above
+ *   idx   device, int32, kascade_index_count(shape) entries, written
+ */
+KASCADE_API int kascade_select(const kascade_shape* shape, const void* q, const void* k,
+                   int32_t* idx, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Sparse decode attention of an anchor or reuse layer (README Abstract:
+ * reuse layers attend over the anchor's indices; selection and reuse are
+ * head-aware).  kv head h attends over the list idx[b, head_map[h]] (the
+ * anchor layer's decode index buffer) and for each of its G query heads
+ * writes o = softmax(q . k_S / sqrt(d)) v_S.
+ *   head_map  device int32 [Hkv], entries in [0, Hkv); NULL = identity
+ *             (an anchor layer attending over its own sets).  The host
+ *             cannot read it, so the kernel guards it: a kv head whose entry
+ *             is out of range attends over an empty list (o = 0, lse = -inf).
+ *   idx       device int32 [B, Hkv, K] as written by kascade_select
+ *   o, lse    device outputs (lse may be NULL)
+ * Requires q_len == 1.  Index values must lie in [0, N) (not checked on the
+ * device; kascade_select only writes such values).
+ */
+KASCADE_API int kascade_sparse_decode(const kascade_shape* shape, const void* q, const void* k,
+                          const void* v, const int32_t* idx, const int32_t* head_map,
+                          void* o, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Sparse causal prefill attention of an anchor or reuse layer (README
+ * Abstract, tile-level operations in prefill).  For query tile t of kv head
+ * h, the rows of h's G query heads attend over the keys j of list
+ * (b, head_map[h], t) with j <= the row's position.  A row with no such key
+ * writes o = 0 and lse = -inf.  Requires q_len == kv_len.
+ */
+KASCADE_API int kascade_sparse_prefill(const kascade_shape* shape, const void* q, const void* k,
+                           const void* v, const int32_t* idx, const int32_t* head_map,
+                           void* o, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Dense reference attention (the role FlashAttention-3 plays as the README's
+ * speed-up baseline, Abstract): every query attends over all keys (decode,
+ * q_len == 1) or causally over keys j <= i (prefill, q_len == N, causal != 0).
+ */
+KASCADE_API int kascade_dense_ref(const kascade_shape* shape, const void* q, const void* k,
+                      const void* v, int causal, void* o, float* lse,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/* Static string for a status code. */
+KASCADE_API const char* kascade_status_str(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KASCADE_H_ */

@@ -1,0 +1,372 @@
+// C ABI of the Kascade library: argument checks, workspace layout and kernel
+// launches.  Declarations and the calling contract are in include/kascade.h.
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/kascade.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace kascade {
+namespace {
+
+// Grids and workspace sizes are planned for the 148 SMs of a B200; other
+// parts run the same grids in more or fewer waves.
+constexpr int kPlanSMs = 148;
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+int check_shape(const kascade_shape* s) {
+  if (!s) return KASCADE_ERR_INVALID_ARG;
+  if (s->batch < 1 || s->num_q_heads < 1 || s->num_kv_heads < 1 || s->kv_len < 1 || s->q_len < 1)
+    return KASCADE_ERR_INVALID_ARG;
+  if (s->num_q_heads % s->num_kv_heads != 0) return KASCADE_ERR_INVALID_ARG;
+  if (s->topk_num < 1 || s->topk_den < 1 || s->topk_num > s->topk_den) return KASCADE_ERR_INVALID_ARG;
+  if (s->head_dim != 64 && s->head_dim != 128) return KASCADE_ERR_UNSUPPORTED;
+  if (s->num_q_heads / s->num_kv_heads > 8) return KASCADE_ERR_UNSUPPORTED;
+  if (s->kv_len > (1 << 20)) return KASCADE_ERR_UNSUPPORTED;
+  if (s->topk_den > (1 << 20)) return KASCADE_ERR_UNSUPPORTED;
+  if (s->q_len != 1 && s->q_len != s->kv_len) return KASCADE_ERR_UNSUPPORTED;
+  if (s->q_len != 1 && s->tile != 32) return KASCADE_ERR_UNSUPPORTED;
+  return KASCADE_OK;
+}
+
+bool is_decode(const kascade_shape* s) { return s->q_len == 1; }
+int n_tiles(const kascade_shape* s) { return (s->kv_len + 31) / 32; }
+
+int64_t prefill_row_len(const kascade_shape* s) {
+  const int T = n_tiles(s);
+  return tile_list_offset(T - 1, 32, s->topk_num, s->topk_den) + topk_count(s->kv_len, s->topk_num, s->topk_den);
+}
+
+int64_t pooled_row_len(const kascade_shape* s) { return tile_pooled_offset(n_tiles(s) - 1, 32) + s->kv_len; }
+
+// ----------------------------------------------------------------- workspace plans
+
+struct Carver {
+  char* base;
+  size_t off = 0;
+  template <class T>
+  T* take(size_t count) {
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off = align_up(off + count * sizeof(T));
+    return p;
+  }
+};
+
+struct SelectPlan {
+  float* s2;
+  float* m_part;
+  double* l_part;
+  int splits;
+  float* row_m2;
+  double* row_l;
+  float* pooled;
+  float* v_scratch;
+  int32_t* band_idx;
+  double* band_val;
+  uint8_t* state;
+  int grid;
+  size_t bytes;
+};
+
+// Every plan starts with the same counter block, so that one workspace can
+// serve all calls of a shape while the ticket counters stay zero between them.
+int* take_counters(Carver& cv, const kascade_shape* s) {
+  return cv.take<int>((size_t)s->batch * s->num_kv_heads);
+}
+
+SelectPlan plan_select(const kascade_shape* s, void* ws) {
+  SelectPlan p{};
+  Carver cv{static_cast<char*>(ws)};
+  take_counters(cv, s);
+  const size_t B = s->batch, Hq = s->num_q_heads, Hkv = s->num_kv_heads, N = s->kv_len;
+  const int n_max = s->kv_len;
+  if (is_decode(s)) {
+    p.splits = (s->kv_len + decode_score_keys_per_split() - 1) / decode_score_keys_per_split();
+    p.s2 = cv.take<float>(B * Hq * N);
+    p.m_part = cv.take<float>(B * Hq * p.splits);
+    p.l_part = cv.take<double>(B * Hq * p.splits);
+    p.grid = select_grid(false, (int)(B * Hkv), kPlanSMs);
+    p.v_scratch = cv.take<float>((size_t)p.grid * n_max);
+  } else {
+    p.row_m2 = cv.take<float>(B * Hq * N);
+    p.row_l = cv.take<double>(B * Hq * N);
+    p.pooled = cv.take<float>(B * Hkv * (size_t)pooled_row_len(s));
+    const int64_t problems = (int64_t)B * Hkv * n_tiles(s);
+    p.grid = select_grid(true, (int)(problems < (1 << 30) ? problems : (1 << 30)), kPlanSMs);
+    p.v_scratch = nullptr;
+  }
+  p.band_idx = cv.take<int32_t>((size_t)p.grid * n_max);
+  p.band_val = cv.take<double>((size_t)p.grid * n_max);
+  p.state = cv.take<uint8_t>((size_t)p.grid * n_max);
+  p.bytes = cv.off;
+  return p;
+}
+
+struct AttnPlan {
+  float* part_o;
+  float* part_ml;
+  int* counters;
+  int splits, keys_per_split;
+  size_t bytes;
+};
+
+AttnPlan plan_decode_attn(const kascade_shape* s, int list_len, void* ws) {
+  AttnPlan p{};
+  Carver cv{static_cast<char*>(ws)};
+  const size_t BH = (size_t)s->batch * s->num_kv_heads;
+  const int G = s->num_q_heads / s->num_kv_heads;
+  decode_attn_plan(s->batch, s->num_kv_heads, list_len, kPlanSMs, &p.splits, &p.keys_per_split);
+  p.counters = take_counters(cv, s);      // zero-filled once, kept zero by the kernels
+  p.part_o = cv.take<float>(BH * p.splits * G * s->head_dim);
+  p.part_ml = cv.take<float>(BH * p.splits * G * 2);
+  p.bytes = cv.off;
+  return p;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? KASCADE_OK : KASCADE_ERR_CUDA; }
+
+int check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (need == 0) return KASCADE_OK;
+  if (!ws || !aligned(ws, kAlign) || ws_bytes < need) return KASCADE_ERR_WORKSPACE;
+  return KASCADE_OK;
+}
+
+int check_tensors(const void* q, const void* k, const void* v, const void* o) {
+  if (!q || !k || !o) return KASCADE_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(o, 16) || (v && !aligned(v, 16)))
+    return KASCADE_ERR_UNSUPPORTED;
+  return KASCADE_OK;
+}
+
+AttnArgs attn_args(const kascade_shape* s, const void* q, const void* k, const void* v,
+                   const int32_t* idx, const int32_t* head_map, void* o, float* lse) {
+  AttnArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.v = static_cast<const __nv_bfloat16*>(v);
+  a.idx = idx;
+  a.head_map = head_map;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.B = s->batch;
+  a.Hq = s->num_q_heads;
+  a.Hkv = s->num_kv_heads;
+  a.G = a.Hq / a.Hkv;
+  a.D = s->head_dim;
+  a.N = s->kv_len;
+  a.tile = 32;
+  a.num = s->topk_num;
+  a.den = s->topk_den;
+  return a;
+}
+
+int run_decode_attn(const kascade_shape* s, AttnArgs a, int list_len, void* ws, size_t ws_bytes,
+                    cudaStream_t st) {
+  AttnPlan pl = plan_decode_attn(s, list_len, nullptr);
+  int rc = check_ws(ws, ws_bytes, pl.bytes);
+  if (rc) return rc;
+  pl = plan_decode_attn(s, list_len, ws);
+  a.part_o = pl.part_o;
+  a.part_ml = pl.part_ml;
+  a.counters = pl.counters;
+  a.splits = pl.splits;
+  a.keys_per_split = pl.keys_per_split;
+  return cuda_status(launch_decode_attn(a, st));
+}
+
+}  // namespace
+}  // namespace kascade
+
+using namespace kascade;
+
+extern "C" {
+
+size_t kascade_workspace_bytes(const kascade_shape* s, int op) {
+  if (check_shape(s)) return 0;
+  switch (op) {
+    case KASCADE_OP_SELECT:
+      return plan_select(s, nullptr).bytes;
+    case KASCADE_OP_SPARSE_DECODE:
+      return is_decode(s) ? plan_decode_attn(s, topk_count(s->kv_len, s->topk_num, s->topk_den), nullptr).bytes : 0;
+    case KASCADE_OP_SPARSE_PREFILL:
+      return 0;
+    case KASCADE_OP_DENSE:
+      return is_decode(s) ? plan_decode_attn(s, s->kv_len, nullptr).bytes : 0;
+    default:
+      return 0;
+  }
+}
+
+int64_t kascade_index_count(const kascade_shape* s) {
+  if (check_shape(s)) return -1;
+  const int64_t BH = (int64_t)s->batch * s->num_kv_heads;
+  if (is_decode(s)) return BH * topk_count(s->kv_len, s->topk_num, s->topk_den);
+  return BH * prefill_row_len(s);
+}
+
+int kascade_index_offsets(const kascade_shape* s, int64_t* offsets) {
+  int rc = check_shape(s);
+  if (rc) return rc;
+  if (!offsets) return KASCADE_ERR_INVALID_ARG;
+  if (is_decode(s)) {
+    offsets[0] = 0;
+    offsets[1] = topk_count(s->kv_len, s->topk_num, s->topk_den);
+    return KASCADE_OK;
+  }
+  const int T = n_tiles(s);
+  for (int t = 0; t < T; ++t) offsets[t] = tile_list_offset(t, 32, s->topk_num, s->topk_den);
+  offsets[T] = prefill_row_len(s);
+  return KASCADE_OK;
+}
+
+int kascade_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws && ws_bytes) return KASCADE_ERR_WORKSPACE;
+  if (!ws_bytes) return KASCADE_OK;
+  return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream)));
+}
+
+int kascade_select(const kascade_shape* s, const void* q, const void* k, int32_t* idx, void* ws,
+                   size_t ws_bytes, void* stream) {
+  int rc = check_shape(s);
+  if (rc) return rc;
+  if (!q || !k || !idx) return KASCADE_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(idx, 4)) return KASCADE_ERR_UNSUPPORTED;
+  SelectPlan pl = plan_select(s, nullptr);
+  rc = check_ws(ws, ws_bytes, pl.bytes);
+  if (rc) return rc;
+  pl = plan_select(s, ws);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SelArgs a{};
+  a.prefill = !is_decode(s);
+  a.B = s->batch;
+  a.Hq = s->num_q_heads;
+  a.Hkv = s->num_kv_heads;
+  a.G = a.Hq / a.Hkv;
+  a.D = s->head_dim;
+  a.N = s->kv_len;
+  a.tile = 32;
+  a.num = s->topk_num;
+  a.den = s->topk_den;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.v_scratch = pl.v_scratch;
+  a.band_idx = pl.band_idx;
+  a.band_val = pl.band_val;
+  a.state = pl.state;
+  a.n_max = s->kv_len;
+  a.grid = pl.grid;
+  a.idx = idx;
+  if (is_decode(s)) {
+    DecodeScoreArgs d{};
+    d.q = a.q;
+    d.k = a.k;
+    d.s2 = pl.s2;
+    d.m_part = pl.m_part;
+    d.l_part = pl.l_part;
+    d.B = a.B;
+    d.Hq = a.Hq;
+    d.Hkv = a.Hkv;
+    d.G = a.G;
+    d.D = a.D;
+    d.N = a.N;
+    rc = cuda_status(launch_decode_score(d, st));
+    if (rc) return rc;
+    a.s2 = pl.s2;
+    a.m_part = pl.m_part;
+    a.l_part = pl.l_part;
+    a.splits = pl.splits;
+  } else {
+    ScorePoolArgs sp{};
+    sp.q = a.q;
+    sp.k = a.k;
+    sp.row_m2 = pl.row_m2;
+    sp.row_l = pl.row_l;
+    sp.pooled = pl.pooled;
+    sp.B = a.B;
+    sp.Hq = a.Hq;
+    sp.Hkv = a.Hkv;
+    sp.G = a.G;
+    sp.D = a.D;
+    sp.N = a.N;
+    sp.tile = 32;
+    rc = cuda_status(launch_score_pool(sp, st));
+    if (rc) return rc;
+    a.pooled = pl.pooled;
+    a.row_m2 = pl.row_m2;
+    a.row_l = pl.row_l;
+  }
+  return cuda_status(launch_select(a, st));
+}
+
+int kascade_sparse_decode(const kascade_shape* s, const void* q, const void* k, const void* v,
+                          const int32_t* idx, const int32_t* head_map, void* o, float* lse, void* ws,
+                          size_t ws_bytes, void* stream) {
+  int rc = check_shape(s);
+  if (rc) return rc;
+  if (!is_decode(s)) return KASCADE_ERR_UNSUPPORTED;
+  if (!v || !idx) return KASCADE_ERR_INVALID_ARG;
+  rc = check_tensors(q, k, v, o);
+  if (rc) return rc;
+  if (!aligned(idx, 4) || (head_map && !aligned(head_map, 4)) || (lse && !aligned(lse, 4)))
+    return KASCADE_ERR_UNSUPPORTED;
+  AttnArgs a = attn_args(s, q, k, v, idx, head_map, o, lse);
+  return run_decode_attn(s, a, topk_count(s->kv_len, s->topk_num, s->topk_den), ws, ws_bytes,
+                         static_cast<cudaStream_t>(stream));
+}
+
+int kascade_sparse_prefill(const kascade_shape* s, const void* q, const void* k, const void* v,
+                           const int32_t* idx, const int32_t* head_map, void* o, float* lse, void* ws,
+                           size_t ws_bytes, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  int rc = check_shape(s);
+  if (rc) return rc;
+  // N = 1 is both a decode and a prefill shape; both index layouts coincide there
+  if (s->q_len != s->kv_len) return KASCADE_ERR_UNSUPPORTED;
+  if (!v || !idx) return KASCADE_ERR_INVALID_ARG;
+  rc = check_tensors(q, k, v, o);
+  if (rc) return rc;
+  if (!aligned(idx, 4) || (head_map && !aligned(head_map, 4)) || (lse && !aligned(lse, 4)))
+    return KASCADE_ERR_UNSUPPORTED;
+  AttnArgs a = attn_args(s, q, k, v, idx, head_map, o, lse);
+  return cuda_status(launch_prefill_attn(a, static_cast<cudaStream_t>(stream)));
+}
+
+int kascade_dense_ref(const kascade_shape* s, const void* q, const void* k, const void* v, int causal,
+                      void* o, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_shape(s);
+  if (rc) return rc;
+  if (!v) return KASCADE_ERR_INVALID_ARG;
+  rc = check_tensors(q, k, v, o);
+  if (rc) return rc;
+  if (lse && !aligned(lse, 4)) return KASCADE_ERR_UNSUPPORTED;
+  AttnArgs a = attn_args(s, q, k, v, nullptr, nullptr, o, lse);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (is_decode(s)) return run_decode_attn(s, a, s->kv_len, ws, ws_bytes, st);
+  a.causal = causal != 0;
+  return cuda_status(launch_prefill_attn(a, st));
+}
+
+const char* kascade_status_str(int status) {
+  switch (status) {
+    case KASCADE_OK:
+      return "ok";
+    case KASCADE_ERR_INVALID_ARG:
+      return "invalid argument";
+    case KASCADE_ERR_UNSUPPORTED:
+      return "unsupported shape, alignment or option";
+    case KASCADE_ERR_WORKSPACE:
+      return "workspace missing, misaligned or too small";
+    case KASCADE_ERR_CUDA:
+      return "CUDA launch or device error";
+    default:
+      return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,148 @@
+// Shared device helpers of the Kascade CUDA library (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kascade {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr double kLn2 = 0.6931471805599453;
+
+// ---------------------------------------------------------------------------
+// tile arithmetic (prefill): e_t = min(32 (t+1), N), k_t = ceil(num e_t / den)
+
+__host__ __device__ inline int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+__host__ __device__ inline int topk_count(int64_t e, int num, int den) {
+  return e <= 0 ? 0 : (int)ceil_div64((int64_t)num * e, den);
+}
+
+// sum_{i=0}^{n-1} floor((a i + b) / m) for a, b >= 0, m > 0, n >= 0.
+// Reduces a and b modulo m, then counts lattice points under the line by
+// exchanging the roles of the axes (Euclid-like recursion); O(log) steps.
+__host__ __device__ inline int64_t floor_sum(int64_t n, int64_t m, int64_t a, int64_t b) {
+  int64_t total = 0;
+  while (n > 0) {
+    if (a >= m) {
+      total += (n * (n - 1) / 2) * (a / m);
+      a %= m;
+    }
+    if (b >= m) {
+      total += n * (b / m);
+      b %= m;
+    }
+    const int64_t y = a * n + b;   // the line a x + b at x = n
+    if (y < m) break;
+    // points (x, j) with 1 <= j <= floor(y/m) - ... : swap axes
+    n = y / m;
+    b = y % m;
+    const int64_t t = m;
+    m = a;
+    a = t;
+  }
+  return total;
+}
+
+// Start of tile t's list inside one (batch, kv head) index row: sum over
+// the full tiles t' < t of ceil(num * tile (t'+1) / den).
+__host__ __device__ inline int64_t tile_list_offset(int64_t t, int tile, int num, int den) {
+  // ceil(A (i+1) / Q) = floor((A i + A + Q - 1) / Q), A = num * tile, Q = den
+  const int64_t A = (int64_t)num * tile;
+  return floor_sum(t, den, A, A + den - 1);
+}
+
+// Start of tile t's pooled-score row: sum_{t' < t} e_t' = tile * t (t+1) / 2.
+__host__ __device__ inline int64_t tile_pooled_offset(int64_t t, int tile) {
+  return (int64_t)tile * t * (t + 1) / 2;
+}
+
+// ---------------------------------------------------------------------------
+// bf16 helpers
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
+
+// ---------------------------------------------------------------------------
+// warp-level tensor-core MMA (m16n8k16, bf16 in, fp32 accumulate)
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t smem_addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_addr));
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t smem_addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_addr));
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// 16-byte global -> shared async copy; src_bytes = 0 zero-fills the line.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
+}
+
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// ---------------------------------------------------------------------------
+// block-wide inclusive scan of one int per thread (NT threads, NT % 32 == 0)
+
+template <int NT>
+__device__ __forceinline__ int block_inclusive_scan(int x, int* warp_buf /* >= NT/32 + 1 ints */,
+                                                    int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_buf[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < NT / 32 ? warp_buf[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < NT / 32) warp_buf[lane] = w;
+  }
+  __syncthreads();
+  if (warp > 0) x += warp_buf[warp - 1];
+  if (total) *total = warp_buf[NT / 32 - 1];
+  __syncthreads();
+  return x;
+}
+
+}  // namespace kascade

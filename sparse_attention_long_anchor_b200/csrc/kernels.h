@@ -1,0 +1,81 @@
+// Internal launch interface between the C ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kascade {
+
+struct DecodeScoreArgs {
+  const __nv_bfloat16* q;  // [B, Hq, 1, D]
+  const __nv_bfloat16* k;  // [B, Hkv, N, D]
+  float* s2;               // [B, Hq, N]      scores * log2(e)/sqrt(D)
+  float* m_part;           // [B, Hq, splits]
+  double* l_part;          // [B, Hq, splits]
+  int B, Hq, Hkv, G, D, N;
+};
+int decode_score_keys_per_split();
+cudaError_t launch_decode_score(const DecodeScoreArgs& a, cudaStream_t stream);
+
+// Top-k selection over pooled post-softmax scores (decode or prefill).
+struct SelArgs {
+  bool prefill;
+  int B, Hq, Hkv, G, D, N, tile, num, den;
+  const __nv_bfloat16* q;  // [B, Hq, Lq, D]
+  const __nv_bfloat16* k;  // [B, Hkv, N, D]
+  // decode inputs
+  const float* s2;         // [B, Hq, N]
+  const float* m_part;     // [B, Hq, splits]
+  const double* l_part;    // [B, Hq, splits]
+  int splits;
+  // prefill inputs
+  const float* pooled;     // [B, Hkv, sum_t e_t] fp32 pooled scores
+  const float* row_m2;     // [B, Hq, N]  row max of s2
+  const double* row_l;     // [B, Hq, N]  row sum of exp2(s2 - m2)
+  // per-CTA scratch (grid CTAs, n_max entries each)
+  float* v_scratch;        // decode only
+  int32_t* band_idx;
+  double* band_val;
+  uint8_t* state;
+  int n_max;
+  int grid;
+  int32_t* idx;            // output
+};
+size_t select_scratch_bytes_per_cta(int n_max);
+int select_grid(bool prefill, int problems, int num_sms);
+cudaError_t launch_select(const SelArgs& a, cudaStream_t stream);
+
+// Anchor prefill scoring and pooling (row statistics, then pooled scores).
+struct ScorePoolArgs {
+  const __nv_bfloat16* q;  // [B, Hq, N, D]
+  const __nv_bfloat16* k;  // [B, Hkv, N, D]
+  float* row_m2;           // [B, Hq, N]
+  double* row_l;           // [B, Hq, N]
+  float* pooled;           // [B, Hkv, sum_t e_t]
+  int B, Hq, Hkv, G, D, N, tile;
+};
+cudaError_t launch_score_pool(const ScorePoolArgs& a, cudaStream_t stream);
+
+// Sparse / dense attention over an index list (decode: split-K + combine).
+struct AttnArgs {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  const int32_t* idx;        // NULL: dense
+  const int32_t* head_map;   // NULL: identity
+  __nv_bfloat16* o;
+  float* lse;                // may be NULL
+  int B, Hq, Hkv, G, D, N, tile, num, den;
+  bool causal;               // prefill dense only
+  // decode split-K workspace
+  float* part_o;             // [B*Hkv, splits, G, D]
+  float* part_ml;            // [B*Hkv, splits, G, 2]
+  int* counters;             // [B*Hkv], zero between calls
+  int splits, keys_per_split;
+};
+void decode_attn_plan(int B, int Hkv, int list_len, int num_sms, int* splits, int* keys_per_split);
+cudaError_t launch_decode_attn(const AttnArgs& a, cudaStream_t stream);
+cudaError_t launch_prefill_attn(const AttnArgs& a, cudaStream_t stream);
+
+}  // namespace kascade

@@ -1,0 +1,420 @@
+// Exact Top-k selection over pooled post-softmax scores (Kascade README,
+// Abstract: "exact Top-k indices" in the anchor layers; strategy
+// post_softmax_pooled_prefill_topk).
+//
+// One problem = one (batch, kv head) in decode or one (batch, kv head, query
+// tile) in prefill: n candidate keys with pooled scores P_j >= 0, pick the k
+// largest, equal scores going to the lower index, write them ascending.
+//
+// 1. fp32 pooled values v_j (decode: from the raw scores and softmax stats;
+//    prefill: read from the score-and-pool kernel's output).
+// 2. Radix select on the fp32 bit patterns (non-negative floats order like
+//    their uint32 patterns): three histogram passes of 11/11/10 bits in shared
+//    memory give the exact k-th largest fp32 value tau.
+// 3. Keys with v in [tau (1 - delta), tau (1 + delta)] form the band; v is
+//    accurate to far better than delta/3 relative, so keys above the band are
+//    certainly in the true Top-k and keys below it certainly out.  Band
+//    members get their pooled score recomputed in fp64 from the bf16 inputs
+//    (exact products, fp64 sums, fp64 exp2) and the remaining slots go to the
+//    largest of those, lower index first on equal values.
+// 4. One ascending pass over the keys writes the selected indices with a
+//    block-wide prefix sum.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace kascade {
+
+namespace {
+
+constexpr int kSelThreads = 1024;
+constexpr int kBins = 2048;
+constexpr float kBandDelta = 1.0f / 8192.0f;
+constexpr float kBandFloor = 0x1p-96f;   // below this fp32 exp2 underflow may hide mass
+constexpr int kMaxRows = 256;             // G * tile rows of one prefill problem
+constexpr int kMaxD = 128;
+
+struct SelShared {
+  unsigned hist[kBins];
+  int scan_buf[kSelThreads / 32 + 1];
+  int bin, above;
+  int nb, chi;
+  int need_eq_ticket;
+  float m2[8];
+  double l[8];
+  float inv_l[8];
+  int b_idx[kSelThreads];
+  double b_val[kSelThreads];
+};
+
+// dynamic shared memory after SelShared (rounded up to 128 bytes so that the
+// 16-byte vector stores into the q tile are aligned): decode q rows as float
+// [8][D]; prefill q tile as bf16 [kMaxRows][D]; per-warp key row as double [32][D]
+constexpr size_t kSelHead = (sizeof(SelShared) + 127) / 128 * 128;
+__host__ __device__ constexpr size_t sel_dyn_bytes() {
+  return kSelHead + (size_t)kMaxRows * kMaxD * 2 + (size_t)(kSelThreads / 32) * kMaxD * 8;
+}
+
+template <int NT>
+__device__ void find_bin(const unsigned* hist, int need, SelShared& sh) {
+  constexpr int BPT = kBins / NT;
+  const int tid = threadIdx.x;
+  int local = 0;
+#pragma unroll
+  for (int i = 0; i < BPT; ++i) local += (int)hist[kBins - 1 - tid * BPT - i];
+  const int incl = block_inclusive_scan<NT>(local, sh.scan_buf, nullptr);
+  const int excl = incl - local;
+  if (excl < need && need <= incl) {
+    int cum = excl;
+#pragma unroll
+    for (int i = 0; i < BPT; ++i) {
+      const int bin = kBins - 1 - tid * BPT - i;
+      const int hc = (int)hist[bin];
+      if (cum + hc >= need) {
+        sh.bin = bin;
+        sh.above = cum;
+        break;
+      }
+      cum += hc;
+    }
+  }
+  __syncthreads();
+}
+
+__device__ __forceinline__ void clear_hist(SelShared& sh) {
+  for (int i = threadIdx.x; i < kBins; i += blockDim.x) sh.hist[i] = 0;
+  __syncthreads();
+}
+
+// Problem description handed to the per-problem routine.
+struct Problem {
+  int b, h, t;
+  int n, k;
+  int i0, rows;            // prefill tile rows [i0, i0 + rows)
+  const float* v;          // pooled values (prefill) / scratch (decode)
+  int32_t* out;
+};
+
+// fp64 pooled score of key j, computed by one warp (all lanes return it).
+__device__ double refine_decode(const SelArgs& a, const Problem& p, int j, const float* qf,
+                                const SelShared& sh, double c2) {
+  const int lane = threadIdx.x & 31;
+  const __nv_bfloat16* krow = a.k + ((size_t)(p.b * a.Hkv + p.h) * a.N + j) * a.D;
+  double total = 0.0;
+  for (int g = 0; g < a.G; ++g) {
+    double dot = 0.0;
+    for (int e = lane; e < a.D; e += 32)
+      dot += (double)qf[g * a.D + e] * (double)__bfloat162float(krow[e]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    total += exp2(dot * c2 - (double)sh.m2[g]) / sh.l[g];
+  }
+  return total / (double)a.G;
+}
+
+__device__ double refine_prefill(const SelArgs& a, const Problem& p, int j,
+                                 const __nv_bfloat16* qtile, double* kbuf, double c2) {
+  const int lane = threadIdx.x & 31;
+  const __nv_bfloat16* krow = a.k + ((size_t)(p.b * a.Hkv + p.h) * a.N + j) * a.D;
+  for (int e = lane; e < a.D; e += 32) kbuf[e] = (double)__bfloat162float(krow[e]);
+  __syncwarp();
+  double total = 0.0;
+  const int nrows = a.G * a.tile;
+  for (int r = lane; r < nrows; r += 32) {
+    const int g = r / a.tile, il = r - g * a.tile;
+    const int i = p.i0 + il;
+    if (il >= p.rows || j > i) continue;
+    const __nv_bfloat16* qr = qtile + (size_t)r * a.D;
+    double dot = 0.0;
+    for (int e = 0; e < a.D; e += 2) {
+      const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162*>(qr + e);
+      dot += (double)__low2float(q2) * kbuf[e] + (double)__high2float(q2) * kbuf[e + 1];
+    }
+    const size_t srow = (size_t)(p.b * a.Hq + p.h * a.G + g) * a.N + i;
+    total += exp2(dot * c2 - (double)a.row_m2[srow]) / a.row_l[srow];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
+  __syncwarp();
+  return total / (double)(a.G * p.rows);
+}
+
+template <int NT>
+__device__ void run_problem(const SelArgs& a, Problem& p, SelShared& sh, float* vscr,
+                            int32_t* band_idx, double* band_val, uint8_t* state, char* dyn) {
+  const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  const double c2 = 1.4426950408889634 / sqrt((double)a.D);
+
+  // fast path: everything is selected
+  if (p.k >= p.n) {
+    for (int j = tid; j < p.n; j += NT) p.out[j] = j;
+    return;
+  }
+
+  float* qf = reinterpret_cast<float*>(dyn);                      // decode
+  __nv_bfloat16* qtile = reinterpret_cast<__nv_bfloat16*>(dyn);   // prefill
+  double* kbuf = reinterpret_cast<double*>(dyn + (size_t)kMaxRows * kMaxD * 2) + warp * kMaxD;
+
+  const float* v = p.v;
+  clear_hist(sh);
+  if (!a.prefill) {
+    // combine split statistics of the G query heads (fp64)
+    if (warp < a.G) {
+      const size_t row = (size_t)(p.b * a.Hq + p.h * a.G + warp) * a.splits;
+      float m = -INFINITY;
+      for (int s = lane; s < a.splits; s += 32) m = fmaxf(m, a.m_part[row + s]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      double l = 0.0;
+      for (int s = lane; s < a.splits; s += 32)
+        l += a.l_part[row + s] * exp2((double)a.m_part[row + s] - (double)m);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+      if (lane == 0) {
+        sh.m2[warp] = m;
+        sh.l[warp] = l;
+        sh.inv_l[warp] = (float)(1.0 / l);
+      }
+    }
+    for (int e = tid; e < a.G * a.D; e += NT) {
+      const int g = e / a.D, dd = e - g * a.D;
+      qf[e] = __bfloat162float(a.q[(size_t)(p.b * a.Hq + p.h * a.G + g) * a.D + dd]);
+    }
+    __syncthreads();
+    const float* srow = a.s2 + (size_t)(p.b * a.Hq + p.h * a.G) * a.N;
+    const float invG = 1.0f / (float)a.G;
+    for (int j = tid; j < p.n; j += NT) {
+      float acc = 0.f;
+      for (int g = 0; g < a.G; ++g) acc += exp2f(srow[(size_t)g * a.N + j] - sh.m2[g]) * sh.inv_l[g];
+      acc *= invG;
+      vscr[j] = acc;
+      atomicAdd(&sh.hist[__float_as_uint(acc) >> 21], 1u);
+    }
+    v = vscr;
+  } else {
+    // stage the tile's query rows (bf16) for the fp64 refinement
+    const int nrows = a.G * a.tile;
+    const int vec_per_row = a.D / 8;
+    for (int e = tid; e < nrows * vec_per_row; e += NT) {
+      const int r = e / vec_per_row, c8 = e - r * vec_per_row;
+      const int g = r / a.tile, il = r - g * a.tile;
+      uint4 val = make_uint4(0, 0, 0, 0);
+      if (il < p.rows)
+        val = *reinterpret_cast<const uint4*>(a.q + ((size_t)(p.b * a.Hq + p.h * a.G + g) * a.N + p.i0 + il) * a.D + c8 * 8);
+      *reinterpret_cast<uint4*>(qtile + (size_t)r * a.D + c8 * 8) = val;
+    }
+    for (int j = tid; j < p.n; j += NT) atomicAdd(&sh.hist[__float_as_uint(v[j]) >> 21], 1u);
+  }
+  __syncthreads();
+
+  // radix select: bits [31:21], [20:10], [9:0]
+  int need = p.k;
+  unsigned prefix = 0;
+  find_bin<NT>(sh.hist, need, sh);
+  prefix = (unsigned)sh.bin << 21;
+  need -= sh.above;
+  __syncthreads();
+  clear_hist(sh);
+  for (int j = tid; j < p.n; j += NT) {
+    const unsigned x = __float_as_uint(v[j]);
+    if ((x >> 21) == (prefix >> 21)) atomicAdd(&sh.hist[(x >> 10) & 2047u], 1u);
+  }
+  __syncthreads();
+  find_bin<NT>(sh.hist, need, sh);
+  prefix |= (unsigned)sh.bin << 10;
+  need -= sh.above;
+  __syncthreads();
+  clear_hist(sh);
+  for (int j = tid; j < p.n; j += NT) {
+    const unsigned x = __float_as_uint(v[j]);
+    if ((x >> 10) == (prefix >> 10)) atomicAdd(&sh.hist[x & 1023u], 1u);
+  }
+  __syncthreads();
+  find_bin<NT>(sh.hist, need, sh);
+  prefix |= (unsigned)sh.bin;
+  __syncthreads();
+
+  // band around the k-th fp32 value
+  const float tau = __uint_as_float(prefix);
+  const float lo = tau < kBandFloor ? 0.0f : tau * (1.0f - kBandDelta);
+  const float hi = fmaxf(tau * (1.0f + kBandDelta), kBandFloor);
+  if (tid == 0) {
+    sh.nb = 0;
+    sh.chi = 0;
+  }
+  __syncthreads();
+  int my_hi = 0;
+  for (int j = tid; j < p.n; j += NT) {
+    const float x = v[j];
+    if (x > hi) {
+      ++my_hi;
+    } else if (x >= lo) {
+      const int pos = atomicAdd(&sh.nb, 1);
+      band_idx[pos] = j;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) my_hi += __shfl_xor_sync(0xffffffffu, my_hi, o);
+  if (lane == 0) atomicAdd(&sh.chi, my_hi);
+  __syncthreads();
+  const int nb = sh.nb;
+  const int need_band = p.k - sh.chi;
+
+  // fp64 pooled scores of the band members, one warp per member
+  for (int i = warp; i < nb; i += NT / 32) {
+    const int j = band_idx[i];
+    const double val = a.prefill ? refine_prefill(a, p, j, qtile, kbuf, c2)
+                                 : refine_decode(a, p, j, qf, sh, c2);
+    if (lane == 0) band_val[i] = val;
+  }
+  __syncthreads();
+
+  int need_tie = 0;
+  if (nb <= NT) {
+    // rank by (value desc, index asc)
+    if (tid < nb) {
+      sh.b_idx[tid] = band_idx[tid];
+      sh.b_val[tid] = band_val[tid];
+    }
+    __syncthreads();
+    if (tid < nb) {
+      const double my_v = sh.b_val[tid];
+      const int my_j = sh.b_idx[tid];
+      int rank = 0;
+      for (int m = 0; m < nb; ++m) {
+        const double ov = sh.b_val[m];
+        rank += (ov > my_v) || (ov == my_v && sh.b_idx[m] < my_j);
+      }
+      state[my_j] = rank < need_band ? 1 : 0;
+    }
+  } else {
+    // radix select on the fp64 bit patterns: 11-bit digits from bit 63 down
+    unsigned long long pre = 0;
+    int nd = need_band;
+    const int shifts[6] = {53, 42, 31, 20, 9, 0};
+    for (int pass = 0; pass < 6; ++pass) {
+      const int sft = shifts[pass];
+      clear_hist(sh);
+      for (int i = tid; i < nb; i += NT) {
+        const unsigned long long x = (unsigned long long)__double_as_longlong(band_val[i]);
+        const bool match = pass == 0 || (x >> (shifts[pass - 1])) == (pre >> (shifts[pass - 1]));
+        if (match) atomicAdd(&sh.hist[(x >> sft) & 2047ull], 1u);
+      }
+      __syncthreads();
+      find_bin<NT>(sh.hist, nd, sh);
+      pre |= (unsigned long long)sh.bin << sft;
+      nd -= sh.above;
+      __syncthreads();
+    }
+    const double tau64 = __longlong_as_double((long long)pre);
+    need_tie = nd;
+    for (int i = tid; i < nb; i += NT) {
+      const double x = band_val[i];
+      state[band_idx[i]] = x > tau64 ? 1 : (x == tau64 ? 2 : 0);
+    }
+  }
+  __syncthreads();
+
+  // ascending compaction
+  int written = 0, ties_taken = 0;
+  for (int base = 0; base < p.n; base += NT) {
+    const int j = base + tid;
+    int flag = 0, tie = 0;
+    if (j < p.n) {
+      const float x = v[j];
+      if (x > hi) {
+        flag = 1;
+      } else if (x >= lo) {
+        const uint8_t st = state[j];
+        flag = st == 1;
+        tie = st == 2;
+      }
+    }
+    if (need_tie > 0) {
+      int ties_total;
+      const int tincl = block_inclusive_scan<NT>(tie, sh.scan_buf, &ties_total);
+      if (tie && ties_taken + tincl - 1 < need_tie) flag = 1;
+      ties_taken += ties_total;
+    }
+    int total;
+    const int incl = block_inclusive_scan<NT>(flag, sh.scan_buf, &total);
+    if (flag) p.out[written + incl - 1] = j;
+    written += total;
+  }
+}
+
+template <int NT>
+__global__ void __launch_bounds__(NT) select_kernel(const SelArgs a) {
+  extern __shared__ __align__(128) char smem_raw[];
+  SelShared& sh = *reinterpret_cast<SelShared*>(smem_raw);
+  char* dyn = smem_raw + kSelHead;
+  const int cta = blockIdx.x;
+  float* vscr = a.v_scratch ? a.v_scratch + (size_t)cta * a.n_max : nullptr;
+  int32_t* band_idx = a.band_idx + (size_t)cta * a.n_max;
+  double* band_val = a.band_val + (size_t)cta * a.n_max;
+  uint8_t* state = a.state + (size_t)cta * a.n_max;
+
+  const int BH = a.B * a.Hkv;
+  if (!a.prefill) {
+    const int64_t K = topk_count(a.N, a.num, a.den);
+    for (int prob = cta; prob < BH; prob += gridDim.x) {
+      Problem p;
+      p.b = prob / a.Hkv;
+      p.h = prob - p.b * a.Hkv;
+      p.t = 0;
+      p.n = a.N;
+      p.k = (int)K;
+      p.i0 = 0;
+      p.rows = 1;
+      p.v = vscr;
+      p.out = a.idx + (size_t)prob * K;
+      run_problem<NT>(a, p, sh, vscr, band_idx, band_val, state, dyn);
+      __syncthreads();
+    }
+  } else {
+    const int T = (a.N + a.tile - 1) / a.tile;
+    const int64_t T_last = T - 1;
+    const int64_t row_len = tile_list_offset(T_last, a.tile, a.num, a.den) + topk_count(a.N, a.num, a.den);
+    const int64_t pooled_len = tile_pooled_offset(T_last, a.tile) + a.N;
+    const int64_t total = (int64_t)T * BH;
+    for (int64_t prob = cta; prob < total; prob += gridDim.x) {
+      const int t = T - 1 - (int)(prob / BH);   // longest tiles first
+      const int bh = (int)(prob % BH);
+      Problem p;
+      p.b = bh / a.Hkv;
+      p.h = bh - p.b * a.Hkv;
+      p.t = t;
+      p.i0 = t * a.tile;
+      p.n = min((t + 1) * a.tile, a.N);
+      p.rows = p.n - p.i0;
+      p.k = topk_count(p.n, a.num, a.den);
+      p.v = a.pooled + (size_t)bh * pooled_len + tile_pooled_offset(t, a.tile);
+      p.out = a.idx + (size_t)bh * row_len + tile_list_offset(t, a.tile, a.num, a.den);
+      run_problem<NT>(a, p, sh, vscr, band_idx, band_val, state, dyn);
+      __syncthreads();
+    }
+  }
+}
+
+}  // namespace
+
+size_t select_scratch_bytes_per_cta(int n_max) {
+  return (size_t)n_max * (sizeof(float) + sizeof(int32_t) + sizeof(double) + 1);
+}
+
+int select_grid(bool prefill, int problems, int num_sms) {
+  (void)prefill;
+  const int cap = num_sms;   // one 1024-thread CTA per SM
+  return problems < cap ? problems : cap;
+}
+
+cudaError_t launch_select(const SelArgs& a, cudaStream_t stream) {
+  const size_t smem = sel_dyn_bytes();
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<kSelThreads>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  select_kernel<kSelThreads><<<a.grid, kSelThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace kascade

@@ -1,0 +1,184 @@
+"""ctypes binding of libkascade.so (the C ABI in include/kascade.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library.  Tensors are torch CUDA tensors (used for device memory and
+streams); the library raises if it was not built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+__all__ = ["Shape", "KascadeError", "lib", "OP_SELECT", "OP_SPARSE_DECODE", "OP_SPARSE_PREFILL",
+           "OP_DENSE", "workspace_bytes", "index_count", "index_offsets", "Workspace", "select",
+           "sparse_decode", "sparse_prefill", "dense_ref", "status_str", "EXPORTS", "LIB_PATH"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkascade.so")
+
+OP_SELECT, OP_SPARSE_DECODE, OP_SPARSE_PREFILL, OP_DENSE = 0, 1, 2, 3
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA = 0, 1, 2, 3, 4
+
+EXPORTS = ("kascade_workspace_bytes", "kascade_index_count", "kascade_index_offsets",
+           "kascade_workspace_init", "kascade_select", "kascade_sparse_decode",
+           "kascade_sparse_prefill", "kascade_dense_ref", "kascade_status_str")
+
+
+class KascadeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_str(status)} (status {status})")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    """kascade_shape: B, Hq, Hkv, d, q_len (1 = decode), kv_len, tile, frac."""
+    _fields_ = [("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("q_len", ctypes.c_int32), ("kv_len", ctypes.c_int32), ("tile", ctypes.c_int32),
+                ("topk_num", ctypes.c_int32), ("topk_den", ctypes.c_int32)]
+
+    @classmethod
+    def make(cls, batch, hq, hkv, d, q_len, kv_len, frac=(10, 100), tile=32):
+        return cls(batch, hq, hkv, d, q_len, kv_len, tile, frac[0], frac[1])
+
+    @property
+    def decode(self) -> bool:
+        return self.q_len == 1
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m sparse_attention_long_anchor_b200.build`")
+    so = ctypes.CDLL(LIB_PATH)
+    P = ctypes.c_void_p
+    SP = ctypes.POINTER(Shape)
+    so.kascade_workspace_bytes.argtypes = [SP, ctypes.c_int]
+    so.kascade_workspace_bytes.restype = ctypes.c_size_t
+    so.kascade_index_count.argtypes = [SP]
+    so.kascade_index_count.restype = ctypes.c_int64
+    so.kascade_index_offsets.argtypes = [SP, ctypes.POINTER(ctypes.c_int64)]
+    so.kascade_index_offsets.restype = ctypes.c_int
+    so.kascade_workspace_init.argtypes = [P, ctypes.c_size_t, P]
+    so.kascade_workspace_init.restype = ctypes.c_int
+    so.kascade_select.argtypes = [SP, P, P, P, P, ctypes.c_size_t, P]
+    so.kascade_select.restype = ctypes.c_int
+    for fn in (so.kascade_sparse_decode, so.kascade_sparse_prefill):
+        fn.argtypes = [SP, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        fn.restype = ctypes.c_int
+    so.kascade_dense_ref.argtypes = [SP, P, P, P, ctypes.c_int, P, P, P, ctypes.c_size_t, P]
+    so.kascade_dense_ref.restype = ctypes.c_int
+    so.kascade_status_str.argtypes = [ctypes.c_int]
+    so.kascade_status_str.restype = ctypes.c_char_p
+    return so
+
+
+lib = _load()
+
+
+def status_str(status: int) -> str:
+    return lib.kascade_status_str(status).decode()
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        raise KascadeError(status, where)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def workspace_bytes(shape: Shape, op: int) -> int:
+    return int(lib.kascade_workspace_bytes(ctypes.byref(shape), op))
+
+
+def index_count(shape: Shape) -> int:
+    n = int(lib.kascade_index_count(ctypes.byref(shape)))
+    if n < 0:
+        raise KascadeError(ERR_INVALID_ARG, "kascade_index_count")
+    return n
+
+
+def index_offsets(shape: Shape) -> np.ndarray:
+    n_t = 1 if shape.decode else -(-shape.kv_len // 32)
+    out = np.zeros(n_t + 1, dtype=np.int64)
+    _check(lib.kascade_index_offsets(ctypes.byref(shape), out.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))),
+           "kascade_index_offsets")
+    return out
+
+
+class Workspace:
+    """A zero-initialised device workspace large enough for the given ops."""
+
+    def __init__(self, shape: Shape, ops=(OP_SELECT, OP_SPARSE_DECODE, OP_SPARSE_PREFILL, OP_DENSE),
+                 device="cuda", nbytes=None):
+        need = nbytes if nbytes is not None else max([workspace_bytes(shape, op) for op in ops] + [256])
+        self.buf = torch.zeros(need + 256, dtype=torch.uint8, device=device)
+        base = self.buf.data_ptr()
+        self.ptr = (base + 255) // 256 * 256
+        self.nbytes = need
+
+    def args(self):
+        return self.ptr, self.nbytes
+
+
+def _ws(ws, shape, op):
+    if ws is None:
+        ws = Workspace(shape, (op,))
+    return ws.args()
+
+
+def select(shape: Shape, q, k, idx=None, ws=None, stream=None):
+    """kascade_select: anchor Top-k index sets (int32, ascending)."""
+    if idx is None:
+        idx = torch.empty(index_count(shape), dtype=torch.int32, device=q.device)
+    p, n = _ws(ws, shape, OP_SELECT)
+    _check(lib.kascade_select(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(idx), p, n, _stream(stream)),
+           "kascade_select")
+    return idx
+
+
+def _attn(fn, name, shape, q, k, v, idx, head_map, o, lse, ws, stream, op):
+    if o is None:
+        o = torch.empty_like(q)
+    p, n = _ws(ws, shape, op)
+    _check(fn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(head_map), _ptr(o),
+              _ptr(lse), p, n, _stream(stream)), name)
+    return o
+
+
+def sparse_decode(shape: Shape, q, k, v, idx, head_map=None, o=None, lse=None, ws=None, stream=None):
+    """kascade_sparse_decode: kv head h attends over anchor list head_map[h]."""
+    return _attn(lib.kascade_sparse_decode, "kascade_sparse_decode", shape, q, k, v, idx, head_map, o, lse,
+                 ws, stream, OP_SPARSE_DECODE)
+
+
+def sparse_prefill(shape: Shape, q, k, v, idx, head_map=None, o=None, lse=None, ws=None, stream=None):
+    """kascade_sparse_prefill: causal tile-level sparse attention."""
+    return _attn(lib.kascade_sparse_prefill, "kascade_sparse_prefill", shape, q, k, v, idx, head_map, o,
+                 lse, ws, stream, OP_SPARSE_PREFILL)
+
+
+def dense_ref(shape: Shape, q, k, v, causal=True, o=None, lse=None, ws=None, stream=None):
+    """kascade_dense_ref: dense (causal) attention."""
+    if o is None:
+        o = torch.empty_like(q)
+    p, n = _ws(ws, shape, OP_DENSE)
+    _check(lib.kascade_dense_ref(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), int(bool(causal)), _ptr(o),
+                                 _ptr(lse), p, n, _stream(stream)), "kascade_dense_ref")
+    return o
