@@ -34,13 +34,13 @@
  * All device work is enqueued on `stream` (a cudaStream_t; NULL = legacy
  * default stream) and is asynchronous: results are ready when the stream is.
  *
- * Workspace: each call takes `ws`/`ws_bytes` of device scratch of at least
- * kascade_workspace_bytes() bytes, 256-byte aligned.  Its first bytes hold
- * per-(batch, kv head) ticket counters that the split-K kernels use to find
- * the last CTA; they must be zero before the first call (zero-fill the whole
- * workspace once with kascade_workspace_init) and every call leaves them zero
- * again, so one workspace sized for the largest op can serve every call of a
- * shape.  Calls that may run concurrently must not share a workspace.
+ * Workspace: kascade_select takes `ws`/`ws_bytes` of device scratch of at
+ * least kascade_workspace_bytes(shape, KASCADE_OP_SELECT) bytes, 256-byte
+ * aligned, with no required initial contents.  The attention calls keep
+ * their partial results on chip and need none (their workspace size is 0;
+ * ws may be NULL), but take the same arguments so that callers can pass one
+ * workspace to every call.  Calls that may run concurrently must not share
+ * a workspace.
  *
  * Errors: every call returns KASCADE_OK (0) or a status below; argument
  * errors are detected on the host before anything is launched.  No kernel
@@ -98,7 +98,8 @@ KASCADE_API int64_t kascade_index_count(const kascade_shape* shape);
  * offsets[T] is the row length.  Decode shapes write {0, K}. */
 KASCADE_API int kascade_index_offsets(const kascade_shape* shape, int64_t* offsets);
 
-/* Zero-fills `ws_bytes` bytes of device workspace on `stream`. */
+/* Zero-fills `ws_bytes` bytes of device workspace on `stream` (optional:
+ * no call depends on the workspace's initial contents). */
 KASCADE_API int kascade_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
 /*

@@ -70,19 +70,13 @@ struct SelectPlan {
   double* band_val;
   uint8_t* state;
   int grid;
+  bool cluster;
   size_t bytes;
 };
-
-// Every plan starts with the same counter block, so that one workspace can
-// serve all calls of a shape while the ticket counters stay zero between them.
-int* take_counters(Carver& cv, const kascade_shape* s) {
-  return cv.take<int>((size_t)s->batch * s->num_kv_heads);
-}
 
 SelectPlan plan_select(const kascade_shape* s, void* ws) {
   SelectPlan p{};
   Carver cv{static_cast<char*>(ws)};
-  take_counters(cv, s);
   const size_t B = s->batch, Hq = s->num_q_heads, Hkv = s->num_kv_heads, N = s->kv_len;
   const int n_max = s->kv_len;
   if (is_decode(s)) {
@@ -90,6 +84,14 @@ SelectPlan plan_select(const kascade_shape* s, void* ws) {
     p.s2 = cv.take<float>(B * Hq * N);
     p.m_part = cv.take<float>(B * Hq * p.splits);
     p.l_part = cv.take<double>(B * Hq * p.splits);
+    if (select_decode_cluster_ok(s->kv_len)) {
+      p.cluster = true;
+      const size_t entries = select_decode_cluster_scratch(s->batch, s->num_kv_heads, s->kv_len);
+      p.band_idx = cv.take<int32_t>(entries);
+      p.band_val = cv.take<double>(entries);
+      p.bytes = cv.off;
+      return p;
+    }
     p.grid = select_grid(false, (int)(B * Hkv), kPlanSMs);
     p.v_scratch = cv.take<float>((size_t)p.grid * n_max);
   } else {
@@ -103,27 +105,6 @@ SelectPlan plan_select(const kascade_shape* s, void* ws) {
   p.band_idx = cv.take<int32_t>((size_t)p.grid * n_max);
   p.band_val = cv.take<double>((size_t)p.grid * n_max);
   p.state = cv.take<uint8_t>((size_t)p.grid * n_max);
-  p.bytes = cv.off;
-  return p;
-}
-
-struct AttnPlan {
-  float* part_o;
-  float* part_ml;
-  int* counters;
-  int splits, keys_per_split;
-  size_t bytes;
-};
-
-AttnPlan plan_decode_attn(const kascade_shape* s, int list_len, void* ws) {
-  AttnPlan p{};
-  Carver cv{static_cast<char*>(ws)};
-  const size_t BH = (size_t)s->batch * s->num_kv_heads;
-  const int G = s->num_q_heads / s->num_kv_heads;
-  decode_attn_plan(s->batch, s->num_kv_heads, list_len, kPlanSMs, &p.splits, &p.keys_per_split);
-  p.counters = take_counters(cv, s);      // zero-filled once, kept zero by the kernels
-  p.part_o = cv.take<float>(BH * p.splits * G * s->head_dim);
-  p.part_ml = cv.take<float>(BH * p.splits * G * 2);
   p.bytes = cv.off;
   return p;
 }
@@ -165,20 +146,6 @@ AttnArgs attn_args(const kascade_shape* s, const void* q, const void* k, const v
   return a;
 }
 
-int run_decode_attn(const kascade_shape* s, AttnArgs a, int list_len, void* ws, size_t ws_bytes,
-                    cudaStream_t st) {
-  AttnPlan pl = plan_decode_attn(s, list_len, nullptr);
-  int rc = check_ws(ws, ws_bytes, pl.bytes);
-  if (rc) return rc;
-  pl = plan_decode_attn(s, list_len, ws);
-  a.part_o = pl.part_o;
-  a.part_ml = pl.part_ml;
-  a.counters = pl.counters;
-  a.splits = pl.splits;
-  a.keys_per_split = pl.keys_per_split;
-  return cuda_status(launch_decode_attn(a, st));
-}
-
 }  // namespace
 }  // namespace kascade
 
@@ -192,11 +159,9 @@ size_t kascade_workspace_bytes(const kascade_shape* s, int op) {
     case KASCADE_OP_SELECT:
       return plan_select(s, nullptr).bytes;
     case KASCADE_OP_SPARSE_DECODE:
-      return is_decode(s) ? plan_decode_attn(s, topk_count(s->kv_len, s->topk_num, s->topk_den), nullptr).bytes : 0;
     case KASCADE_OP_SPARSE_PREFILL:
-      return 0;
     case KASCADE_OP_DENSE:
-      return is_decode(s) ? plan_decode_attn(s, s->kv_len, nullptr).bytes : 0;
+      return 0;   // attention kernels keep their partial results on chip
     default:
       return 0;
   }
@@ -280,6 +245,7 @@ int kascade_select(const kascade_shape* s, const void* q, const void* k, int32_t
     a.m_part = pl.m_part;
     a.l_part = pl.l_part;
     a.splits = pl.splits;
+    if (pl.cluster) return cuda_status(launch_select_decode_cluster(a, st));
   } else {
     ScorePoolArgs sp{};
     sp.q = a.q;
@@ -314,9 +280,10 @@ int kascade_sparse_decode(const kascade_shape* s, const void* q, const void* k, 
   if (rc) return rc;
   if (!aligned(idx, 4) || (head_map && !aligned(head_map, 4)) || (lse && !aligned(lse, 4)))
     return KASCADE_ERR_UNSUPPORTED;
+  (void)ws;
+  (void)ws_bytes;
   AttnArgs a = attn_args(s, q, k, v, idx, head_map, o, lse);
-  return run_decode_attn(s, a, topk_count(s->kv_len, s->topk_num, s->topk_den), ws, ws_bytes,
-                         static_cast<cudaStream_t>(stream));
+  return cuda_status(launch_decode_attn(a, static_cast<cudaStream_t>(stream)));
 }
 
 int kascade_sparse_prefill(const kascade_shape* s, const void* q, const void* k, const void* v,
@@ -347,7 +314,9 @@ int kascade_dense_ref(const kascade_shape* s, const void* q, const void* k, cons
   if (lse && !aligned(lse, 4)) return KASCADE_ERR_UNSUPPORTED;
   AttnArgs a = attn_args(s, q, k, v, nullptr, nullptr, o, lse);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (is_decode(s)) return run_decode_attn(s, a, s->kv_len, ws, ws_bytes, st);
+  (void)ws;
+  (void)ws_bytes;
+  if (is_decode(s)) return cuda_status(launch_decode_attn(a, st));
   a.causal = causal != 0;
   return cuda_status(launch_prefill_attn(a, st));
 }

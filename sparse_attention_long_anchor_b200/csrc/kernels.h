@@ -43,6 +43,10 @@ struct SelArgs {
   int32_t* idx;            // output
 };
 size_t select_scratch_bytes_per_cta(int n_max);
+// decode: one 8-CTA cluster per (batch, kv head) when N / 8 <= 16384
+bool select_decode_cluster_ok(int N);
+size_t select_decode_cluster_scratch(int B, int Hkv, int N);   // band entries
+cudaError_t launch_select_decode_cluster(const SelArgs& a, cudaStream_t stream);
 int select_grid(bool prefill, int problems, int num_sms);
 cudaError_t launch_select(const SelArgs& a, cudaStream_t stream);
 
@@ -68,13 +72,8 @@ struct AttnArgs {
   float* lse;                // may be NULL
   int B, Hq, Hkv, G, D, N, tile, num, den;
   bool causal;               // prefill dense only
-  // decode split-K workspace
-  float* part_o;             // [B*Hkv, splits, G, D]
-  float* part_ml;            // [B*Hkv, splits, G, 2]
-  int* counters;             // [B*Hkv], zero between calls
-  int splits, keys_per_split;
 };
-void decode_attn_plan(int B, int Hkv, int list_len, int num_sms, int* splits, int* keys_per_split);
+// decode: one 16-CTA cluster per (batch, kv head), merge over DSMEM
 cudaError_t launch_decode_attn(const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill_attn(const AttnArgs& a, cudaStream_t stream);
 

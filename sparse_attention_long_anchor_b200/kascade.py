@@ -16,7 +16,7 @@ __all__ = ["Shape", "KascadeError", "lib", "OP_SELECT", "OP_SPARSE_DECODE", "OP_
            "OP_DENSE", "workspace_bytes", "index_count", "index_offsets", "Workspace", "select",
            "sparse_decode", "sparse_prefill", "dense_ref", "status_str", "EXPORTS", "LIB_PATH"]
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkascade.so")
+LIB_PATH = os.environ.get("KASCADE_LIB") or os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkascade.so")
 
 OP_SELECT, OP_SPARSE_DECODE, OP_SPARSE_PREFILL, OP_DENSE = 0, 1, 2, 3
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA = 0, 1, 2, 3, 4
@@ -139,6 +139,8 @@ class Workspace:
 
 def _ws(ws, shape, op):
     if ws is None:
+        if workspace_bytes(shape, op) == 0:
+            return None, 0
         ws = Workspace(shape, (op,))
     return ws.args()
 

@@ -48,8 +48,9 @@ def test_index_layout_matches_oracle(n_ctx, frac):
 def test_workspace_sizes_positive():
     kc = _kc()
     s = kc.Shape.make(1, 32, 8, 128, 1, 32768)
-    for op in (kc.OP_SELECT, kc.OP_SPARSE_DECODE, kc.OP_DENSE):
-        assert kc.workspace_bytes(s, op) > 0
+    assert kc.workspace_bytes(s, kc.OP_SELECT) > 0
+    for op in (kc.OP_SPARSE_DECODE, kc.OP_SPARSE_PREFILL, kc.OP_DENSE):
+        assert kc.workspace_bytes(s, op) == 0
     p = kc.Shape.make(1, 32, 8, 128, 32768, 32768)
     assert kc.workspace_bytes(p, kc.OP_SELECT) > 0
 
@@ -82,10 +83,12 @@ def test_null_and_misaligned_pointers_and_small_workspace():
     assert L.kascade_select(sb, 256, 256, 256, None, need, None) == kc.ERR_WORKSPACE
     assert L.kascade_select(sb, 256, 256, 256, 258, need, None) == kc.ERR_WORKSPACE
     nd = kc.workspace_bytes(s, kc.OP_SPARSE_DECODE)
-    assert L.kascade_sparse_decode(sb, 256, 256, 256, None, None, 256, None, 256, nd, None) == kc.ERR_INVALID_ARG
-    assert L.kascade_sparse_decode(sb, 256, 256, None, 256, None, 256, None, 256, nd, None) == kc.ERR_INVALID_ARG
-    assert L.kascade_sparse_decode(sb, 256, 256, 256, 256, None, 256, None, 256, nd - 1, None) == kc.ERR_WORKSPACE
-    assert L.kascade_sparse_decode(sb, 256, 256, 256, 258, None, 256, None, 256, nd, None) == kc.ERR_UNSUPPORTED
+    assert nd == 0   # attention kernels keep partials on chip
+    assert L.kascade_sparse_decode(sb, 256, 256, 256, None, None, 256, None, None, 0, None) == kc.ERR_INVALID_ARG
+    assert L.kascade_sparse_decode(sb, 256, 256, None, 256, None, 256, None, None, 0, None) == kc.ERR_INVALID_ARG
+    assert L.kascade_sparse_decode(sb, None, 256, 256, 256, None, 256, None, None, 0, None) == kc.ERR_INVALID_ARG
+    assert L.kascade_sparse_decode(sb, 256, 256, 256, 258, None, 256, None, None, 0, None) == kc.ERR_UNSUPPORTED
+    assert L.kascade_sparse_decode(sb, 256, 264, 256, 256, None, 256, None, None, 0, None) == kc.ERR_UNSUPPORTED
     # prefill entry points refuse decode shapes and vice versa
     assert L.kascade_sparse_prefill(sb, 256, 256, 256, 256, None, 256, None, None, 0, None) == kc.ERR_UNSUPPORTED
     p = kc.Shape.make(1, 8, 2, 64, 256, 256)
