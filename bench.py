@@ -229,7 +229,7 @@ def build_decode(kc, synth, torch, dev):
     cfg = synth.CONFIGS[DECODE_CFG]
     plan, layers = synth.make_stack(cfg, device=dev)
     frac = (cfg.frac_num, cfg.frac_den)
-    shape = kc.Shape.make(cfg.batch, cfg.hq, cfg.hkv, cfg.d, 1, cfg.n_ctx, frac)
+    shape = kc.Shape.make(cfg.batch, cfg.hq, cfg.hkv, cfg.d, 1, cfg.n_ctx, frac, flags=kc.FLAG_PDL)
     ws = kc.Workspace(shape, device=dev)
     idx = {a: torch.empty(kc.index_count(shape), dtype=torch.int32, device=dev) for a in cfg.anchors}
     hms = {l: torch.tensor(p[2], dtype=torch.int32, device=dev) for l, p in enumerate(plan) if not p[0]}
@@ -238,6 +238,9 @@ def build_decode(kc, synth, torch, dev):
 
 
 def decode_layer(kc, st, l, which="all"):
+    """One decode layer.  Kernels use programmatic dependent launch; a reuse
+    layer reads an index set written at least two launches earlier and a KV
+    cache that no kernel of the step writes, so its gathers may start early."""
     cfg, plan, layers, shape, ws, idx, hms, outs = st
     is_anchor, anchor, _ = plan[l]
     q, k, v = layers[l]
@@ -247,14 +250,15 @@ def decode_layer(kc, st, l, which="all"):
         if which in ("all", "attn"):
             kc.sparse_decode(shape, q, k, v, idx[l], None, o=outs[l], ws=ws)
     elif which in ("all", "attn"):
-        kc.sparse_decode(shape, q, k, v, idx[anchor], hms[l], o=outs[l], ws=ws)
+        stable = shape.with_flags(kc.FLAG_PDL | kc.FLAG_INPUTS_STABLE)
+        kc.sparse_decode(stable, q, k, v, idx[anchor], hms[l], o=outs[l], ws=ws)
 
 
 def build_prefill(kc, synth, torch, dev):
     cfg = synth.CONFIGS[PREFILL_CFG]
     plan, layers = synth.make_stack(cfg, device=dev)
     frac = (cfg.frac_num, cfg.frac_den)
-    shape = kc.Shape.make(cfg.batch, cfg.hq, cfg.hkv, cfg.d, cfg.n_ctx, cfg.n_ctx, frac)
+    shape = kc.Shape.make(cfg.batch, cfg.hq, cfg.hkv, cfg.d, cfg.n_ctx, cfg.n_ctx, frac, flags=kc.FLAG_PDL)
     ws = kc.Workspace(shape, device=dev)
     idx = {a: torch.empty(kc.index_count(shape), dtype=torch.int32, device=dev) for a in cfg.anchors}
     hms = {l: torch.tensor(p[2], dtype=torch.int32, device=dev) for l, p in enumerate(plan) if not p[0]}

@@ -34,17 +34,21 @@
  * All device work is enqueued on `stream` (a cudaStream_t; NULL = legacy
  * default stream) and is asynchronous: results are ready when the stream is.
  *
- * Workspace: kascade_select takes `ws`/`ws_bytes` of device scratch of at
- * least kascade_workspace_bytes(shape, KASCADE_OP_SELECT) bytes, 256-byte
- * aligned, with no required initial contents.  The attention calls keep
- * their partial results on chip and need none (their workspace size is 0;
- * ws may be NULL), but take the same arguments so that callers can pass one
- * workspace to every call.  Calls that may run concurrently must not share
- * a workspace.
+ * Workspace: every call takes `ws`/`ws_bytes` of device scratch of at
+ * least kascade_workspace_bytes(shape, op) bytes, 256-byte aligned.  Its
+ * first int is the device error word: kernels never trap or wait without
+ * bound, and a bounded wait that gives up stores a non-zero code there
+ * (read it with kascade_workspace_error).  Zero the workspace once before
+ * first use (kascade_workspace_init); nothing else depends on its initial
+ * contents.  The attention calls need only this 256-byte header (their
+ * partial results stay on chip) and accept ws = NULL, in which case no error
+ * word is kept.  One workspace sized for the largest op serves every call of
+ * a shape; calls that may run concurrently must not share a workspace.
  *
  * Errors: every call returns KASCADE_OK (0) or a status below; argument
  * errors are detected on the host before anything is launched.  No kernel
- * traps or waits on another kernel.
+ * traps or waits on another kernel; device-side failures go to the error
+ * word described above.
  */
 #ifndef KASCADE_H_
 #define KASCADE_H_
@@ -84,7 +88,24 @@ typedef struct kascade_shape {
   int32_t tile;         /* prefill query tile; must be 32 (ignored in decode) */
   int32_t topk_num;     /* frac = topk_num / topk_den, 0 < frac <= 1, */
   int32_t topk_den;     /*   e.g. 10/100 for the README's Top-k of 10 % */
+  int32_t flags;        /* KASCADE_FLAG_* bits, 0 for plain stream ordering */
 } kascade_shape;
+
+/* Launch the call's kernels with programmatic dependent launch: a kernel may
+ * begin (set-up only) while the previous kernel on the stream finishes; it
+ * waits for that kernel's completion before reading any input, and lets the
+ * next kernel start right after that wait.  Results are the same as without
+ * the flag. */
+#define KASCADE_FLAG_PDL 1
+/* With KASCADE_FLAG_PDL, sparse decode: the caller guarantees that k, v, idx
+ * and head_map were last written at least two kernel launches earlier on the
+ * stream (or before it), so the gathers may start before the previous kernel
+ * completes.  q and the outputs still wait.  Every kernel of this library
+ * releases its successor only after its own wait, which is what makes the
+ * two-launch rule sufficient.  Do not set it when the previous kernel on the
+ * stream wrote any of those inputs (e.g. the anchor layer's own call right
+ * after kascade_select). */
+#define KASCADE_FLAG_INPUTS_STABLE 2
 
 /* Bytes of workspace that `op` needs for `shape` (0 on an invalid shape). */
 KASCADE_API size_t kascade_workspace_bytes(const kascade_shape* shape, int op);
@@ -157,6 +178,11 @@ KASCADE_API int kascade_sparse_prefill(const kascade_shape* shape, const void* q
 KASCADE_API int kascade_dense_ref(const kascade_shape* shape, const void* q, const void* k,
                       const void* v, int causal, void* o, float* lse,
                       void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, copies the device error word (the first int of
+ * `ws`) to *error_out (0 = no failure; 1 = a bounded wait timed out) and, if
+ * `clear` is non-zero, resets it. */
+KASCADE_API int kascade_workspace_error(const void* ws, int* error_out, int clear, void* stream);
 
 /* Static string for a status code. */
 KASCADE_API const char* kascade_status_str(int status);

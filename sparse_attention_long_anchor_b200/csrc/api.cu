@@ -31,6 +31,7 @@ int check_shape(const kascade_shape* s) {
   if (s->topk_den > (1 << 20)) return KASCADE_ERR_UNSUPPORTED;
   if (s->q_len != 1 && s->q_len != s->kv_len) return KASCADE_ERR_UNSUPPORTED;
   if (s->q_len != 1 && s->tile != 32) return KASCADE_ERR_UNSUPPORTED;
+  if (s->flags & ~(KASCADE_FLAG_PDL | KASCADE_FLAG_INPUTS_STABLE)) return KASCADE_ERR_INVALID_ARG;
   return KASCADE_OK;
 }
 
@@ -74,9 +75,14 @@ struct SelectPlan {
   size_t bytes;
 };
 
+// Every workspace starts with a 256-byte header whose first int is the
+// device error word (set when a bounded wait in a kernel gives up).
+constexpr size_t kHeader = 256;
+
 SelectPlan plan_select(const kascade_shape* s, void* ws) {
   SelectPlan p{};
   Carver cv{static_cast<char*>(ws)};
+  cv.take<char>(kHeader);
   const size_t B = s->batch, Hq = s->num_q_heads, Hkv = s->num_kv_heads, N = s->kv_len;
   const int n_max = s->kv_len;
   if (is_decode(s)) {
@@ -107,6 +113,10 @@ SelectPlan plan_select(const kascade_shape* s, void* ws) {
   p.state = cv.take<uint8_t>((size_t)p.grid * n_max);
   p.bytes = cv.off;
   return p;
+}
+
+int* err_word(void* ws, size_t ws_bytes) {
+  return (ws && ws_bytes >= sizeof(int) && aligned(ws, 4)) ? static_cast<int*>(ws) : nullptr;
 }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? KASCADE_OK : KASCADE_ERR_CUDA; }
@@ -143,6 +153,7 @@ AttnArgs attn_args(const kascade_shape* s, const void* q, const void* k, const v
   a.tile = 32;
   a.num = s->topk_num;
   a.den = s->topk_den;
+  a.flags = s->flags;
   return a;
 }
 
@@ -161,7 +172,7 @@ size_t kascade_workspace_bytes(const kascade_shape* s, int op) {
     case KASCADE_OP_SPARSE_DECODE:
     case KASCADE_OP_SPARSE_PREFILL:
     case KASCADE_OP_DENSE:
-      return 0;   // attention kernels keep their partial results on chip
+      return kHeader;   // only the error word: partial results stay on chip
     default:
       return 0;
   }
@@ -226,8 +237,10 @@ int kascade_select(const kascade_shape* s, const void* q, const void* k, int32_t
   a.n_max = s->kv_len;
   a.grid = pl.grid;
   a.idx = idx;
+  a.flags = s->flags & KASCADE_FLAG_PDL;
   if (is_decode(s)) {
     DecodeScoreArgs d{};
+    d.flags = a.flags;
     d.q = a.q;
     d.k = a.k;
     d.s2 = pl.s2;
@@ -248,6 +261,7 @@ int kascade_select(const kascade_shape* s, const void* q, const void* k, int32_t
     if (pl.cluster) return cuda_status(launch_select_decode_cluster(a, st));
   } else {
     ScorePoolArgs sp{};
+    sp.flags = a.flags;
     sp.q = a.q;
     sp.k = a.k;
     sp.row_m2 = pl.row_m2;
@@ -280,17 +294,14 @@ int kascade_sparse_decode(const kascade_shape* s, const void* q, const void* k, 
   if (rc) return rc;
   if (!aligned(idx, 4) || (head_map && !aligned(head_map, 4)) || (lse && !aligned(lse, 4)))
     return KASCADE_ERR_UNSUPPORTED;
-  (void)ws;
-  (void)ws_bytes;
   AttnArgs a = attn_args(s, q, k, v, idx, head_map, o, lse);
+  a.err = err_word(ws, ws_bytes);
   return cuda_status(launch_decode_attn(a, static_cast<cudaStream_t>(stream)));
 }
 
 int kascade_sparse_prefill(const kascade_shape* s, const void* q, const void* k, const void* v,
                            const int32_t* idx, const int32_t* head_map, void* o, float* lse, void* ws,
                            size_t ws_bytes, void* stream) {
-  (void)ws;
-  (void)ws_bytes;
   int rc = check_shape(s);
   if (rc) return rc;
   // N = 1 is both a decode and a prefill shape; both index layouts coincide there
@@ -301,6 +312,7 @@ int kascade_sparse_prefill(const kascade_shape* s, const void* q, const void* k,
   if (!aligned(idx, 4) || (head_map && !aligned(head_map, 4)) || (lse && !aligned(lse, 4)))
     return KASCADE_ERR_UNSUPPORTED;
   AttnArgs a = attn_args(s, q, k, v, idx, head_map, o, lse);
+  a.err = err_word(ws, ws_bytes);
   return cuda_status(launch_prefill_attn(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -313,12 +325,23 @@ int kascade_dense_ref(const kascade_shape* s, const void* q, const void* k, cons
   if (rc) return rc;
   if (lse && !aligned(lse, 4)) return KASCADE_ERR_UNSUPPORTED;
   AttnArgs a = attn_args(s, q, k, v, nullptr, nullptr, o, lse);
+  a.err = err_word(ws, ws_bytes);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  (void)ws;
-  (void)ws_bytes;
   if (is_decode(s)) return cuda_status(launch_decode_attn(a, st));
   a.causal = causal != 0;
   return cuda_status(launch_prefill_attn(a, st));
+}
+
+int kascade_workspace_error(const void* ws, int* error_out, int clear, void* stream) {
+  if (!ws || !error_out) return KASCADE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int host = 0;
+  cudaError_t e = cudaMemcpyAsync(&host, ws, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess && clear && host) e = cudaMemsetAsync(const_cast<void*>(ws), 0, sizeof(int), st);
+  if (e != cudaSuccess) return KASCADE_ERR_CUDA;
+  *error_out = host;
+  return KASCADE_OK;
 }
 
 const char* kascade_status_str(int status) {

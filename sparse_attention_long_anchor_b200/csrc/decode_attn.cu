@@ -3,15 +3,22 @@
 // indices; selection and reuse are head-aware).  With an implicit full key
 // list the same kernel is the dense decode reference.
 //
-// One thread-block cluster per (batch, kv head): the index list is split
-// evenly over the CTAs of the cluster, every warp gathers 16-key slices of
-// K and V rows with 16-byte cp.async into XOR-swizzled shared memory
-// (3-stage pipeline per warp) and runs bf16 MMAs with the G query heads as
-// the rows of a 16-row tile and an fp32 online softmax.  The partial
-// (max, sum, output) of each CTA stays in its shared memory; after a
-// cluster barrier every CTA merges one slice of the output elements from
-// all CTAs over distributed shared memory.  Nothing goes through global
-// scratch and no CTA waits on anything but the cluster barrier.
+// One thread-block cluster per (batch, kv head); the index list is split
+// evenly over the CTAs of the cluster and every warp owns 16-key slices of
+// its CTA's share.  All warps gather at once:
+//   * K rows go straight from global memory into the registers of the
+//     16x8x16 bf16 MMA (the contraction runs over d, so each lane may take
+//     any permutation of d as long as q uses the same: lane (g, c) loads
+//     dims [32s + 8c, +8) of key g, one 16-byte load per 32 dims);
+//   * V rows go through a two-slot cp.async ring per warp (16-byte copies
+//     into rows padded by 16 bytes, conflict-free for ldmatrix.trans);
+//   * the G query rows sit in shared memory and are read with 8-byte loads
+//     in the same permuted order.
+// S = Q K^T (query heads as the MMA rows), fp32 online softmax, O += P V.
+// The partial (max, sum, output) of each CTA is pushed over distributed
+// shared memory to the CTA that owns each output element; after one cluster
+// barrier every CTA merges its slice locally.  No global scratch, no
+// spin-waits.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -23,58 +30,85 @@ namespace kascade {
 
 namespace {
 
-constexpr int kWarps = 4;
-constexpr int kStages = 3;
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
 constexpr int kMaxCS = 16;
+constexpr int kIdxStage = 2048;   // index entries staged in shared memory
 
 template <int D>
-__device__ __forceinline__ uint32_t swz(int r, int ch) {
-  return (uint32_t)(r * (D * 2) + ((ch ^ (r & 7)) << 4));
-}
+struct Lay {
+  static constexpr int ROW = D * 2 + 16;                  // padded V row bytes
+  static constexpr int SLOT = 16 * ROW;                   // one 16-key V slab
+  static constexpr size_t vslots = 0;                     // [W][2] slots
+  static constexpr size_t qs = vslots + (size_t)kWarps * 2 * SLOT;   // [8][D] bf16 query rows
+  static constexpr size_t idx = qs + 8 * D * 2;
+  static constexpr size_t recv_o = idx + kIdxStage * 4;   // [G*D] f32, peers write here
+  static constexpr size_t recv_ml = recv_o + 8 * D * 4;   // [16][8][2]
+  static constexpr size_t total = recv_ml + kMaxCS * 8 * 2 * 4;
+  // after the gather loop, inside the V slots
+  static constexpr int RO = D + 8;                        // padded red_o row (floats)
+  static constexpr size_t red_o = 0;                      // [W][8][RO]
+  static constexpr size_t red_ml = red_o + (size_t)kWarps * 8 * RO * 4;
+  static constexpr size_t wf = red_ml + kWarps * 8 * 2 * 4;
+  static constexpr size_t pml = wf + kWarps * 8 * 4;
+  static constexpr size_t wts = pml + 8 * 2 * 4;
+  static constexpr size_t head = wts + kMaxCS * 8 * 4;
+  static_assert(head + 64 <= qs, "post-loop scratch must fit in the V slots");
+};
 
 __device__ __forceinline__ float scale_from(float m_old, float m_new) {
   return m_old == -INFINITY ? 0.0f : exp2f(m_old - m_new);
 }
 
-template <int D>
-constexpr size_t pipe_bytes() {
-  return (size_t)kWarps * kStages * 2 * 16 * D * 2;
+// Softmax-merge weights of n_slots partial results per head: for every
+// (slot, head) the factor exp2(m - M) against the head's max M, and per head
+// (M, sum of factor * l).  Called by one whole warp.  ml and w are laid out
+// [slot][8][2] and [slot][8]; out is [8][2].
+__device__ void merge_weights(int n_slots, int G, const float* ml, float* w, float* out, int lane) {
+  if (32 % G == 0) {
+    const int gg = lane % G;   // every pair a lane visits belongs to this head
+    float M = -INFINITY;
+    for (int i = lane; i < n_slots * G; i += 32) M = fmaxf(M, ml[((i / G) * 8 + gg) * 2]);
+    for (int o = G; o < 32; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float ls = 0.f;
+    for (int i = lane; i < n_slots * G; i += 32) {
+      const int sl = i / G;
+      const float f = scale_from(ml[(sl * 8 + gg) * 2], M);
+      w[sl * 8 + gg] = f;
+      ls += f * ml[(sl * 8 + gg) * 2 + 1];
+    }
+    for (int o = G; o < 32; o <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+    if (lane < G) {
+      out[gg * 2] = M;
+      out[gg * 2 + 1] = ls;
+    }
+  } else if (lane < G) {
+    const int gg = lane;
+    float M = -INFINITY;
+    for (int sl = 0; sl < n_slots; ++sl) M = fmaxf(M, ml[(sl * 8 + gg) * 2]);
+    float ls = 0.f;
+    for (int sl = 0; sl < n_slots; ++sl) {
+      const float f = scale_from(ml[(sl * 8 + gg) * 2], M);
+      w[sl * 8 + gg] = f;
+      ls += f * ml[(sl * 8 + gg) * 2 + 1];
+    }
+    out[gg * 2] = M;
+    out[gg * 2 + 1] = ls;
+  }
 }
 
-// shared-memory layout after the gather loop (inside the pipeline region):
-//   red_o [W][8][D] | red_ml [W][8][2] | wts [16][8] | head [8][2]
-// and, in a region of their own that peers may write at any time:
-//   recv_o [G*D] f32 ([rank][slice] of this CTA's element slice) | recv_ml [16][8][2]
 template <int D>
-struct Post {
-  static constexpr size_t red_o = 0;
-  static constexpr size_t red_ml = red_o + (size_t)kWarps * 8 * D * 4;
-  static constexpr size_t wts = red_ml + kWarps * 8 * 2 * 4;
-  static constexpr size_t head = wts + kMaxCS * 8 * 4;
-  static constexpr size_t end = head + 8 * 2 * 4;
-};
-
-constexpr int kIdxStage = 2048;   // index entries staged in shared memory
-
-template <int D>
-constexpr size_t main_bytes() {
-  return pipe_bytes<D>() > Post<D>::end ? pipe_bytes<D>() : Post<D>::end;
-}
-template <int D>
-constexpr size_t recv_off() {
-  return main_bytes<D>() + kIdxStage * 4;
-}
-template <int D>
-constexpr size_t smem_bytes() {
-  return recv_off<D>() + 8 * D * 4 + kMaxCS * 8 * 2 * 4;
-}
-
-template <int D>
-__global__ void __launch_bounds__(kWarps * 32) decode_attn_kernel(const AttnArgs a, int per) {
-  constexpr int CH = D / 8;
-  constexpr int SLICE = 16 * D * 2;   // one 16-key slab of K (or V)
+__global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const AttnArgs a, int per) {
+  using L = Lay<D>;
+  constexpr int KS = D / 32;          // 16-byte K loads per key row per lane
   extern __shared__ __align__(128) char smem[];
-
+  // with PDL the gathers may start before the previous kernel completes only
+  // if the caller vouched for k, v, idx and head_map; otherwise wait first
+  const bool early = (a.flags & 3) == 3;
+  if (!early) {
+    pdl_wait();
+    pdl_launch_dependents();
+  }
   cg::cluster_group cluster = cg::this_cluster();
   const int CS = (int)cluster.num_blocks();
   const int rank = (int)cluster.block_rank();
@@ -92,46 +126,44 @@ __global__ void __launch_bounds__(kWarps * 32) decode_attn_kernel(const AttnArgs
   const int32_t* list = a.idx ? a.idx + (size_t)(b * a.Hkv + hm) * list_full : nullptr;
   const int c0 = min(list_len, rank * per);
   const int c1 = min(list_len, c0 + per);
+  const int n_slices = (c1 - c0 + 15) / 16;
+  int* idx_s = reinterpret_cast<int*>(smem + L::idx);
+  const bool staged = list != nullptr && (c1 - c0) <= kIdxStage;
   const __nv_bfloat16* kb = a.k + (size_t)bh * a.N * D;
   const __nv_bfloat16* vb = a.v + (size_t)bh * a.N * D;
 
-  // Q as the A operand: row g = query head g of the group (rows >= G are 0)
-  uint32_t qa[D / 16][2];
-  {
-    const __nv_bfloat16* qrow = a.q + (size_t)(b * a.Hq + h * G + (g < G ? g : 0)) * D;
+  if (staged)
+    for (int i = threadIdx.x; i < c1 - c0; i += kThreads) idx_s[i] = __ldg(list + c0 + i);
+  __syncthreads();
+
+  auto key_of = [&](int rel) -> int {
+    return list ? (staged ? idx_s[rel] : __ldg(list + c0 + rel)) : c0 + rel;
+  };
+  // V rows of slice s into this warp's slot (s / W) & 1; missing rows zero-filled
+  const uint32_t vbase = smem_u32(smem) + (uint32_t)(warp * 2 * L::SLOT);
+  auto issue_v = [&](int s) {
+    const uint32_t dst = vbase + ((s / kWarps) & 1) * L::SLOT;
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      qa[kk][0] = g < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * c) : 0u;
-      qa[kk][1] = g < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * c + 8) : 0u;
+    for (int i = 0; i < D / 16; ++i) {   // 16 rows x D/8 chunks over 32 lanes
+      const int e = lane + 32 * i;
+      const int r = e / (D / 8), ch = e - r * (D / 8);
+      const int rel = s * 16 + r;
+      const bool have = c0 + rel < c1;
+      const int key = have ? key_of(rel) : 0;
+      cp_async_16(dst + r * L::ROW + ch * 16, vb + (size_t)key * D + ch * 8, have ? 16 : 0);
     }
-  }
-
-  const uint32_t wsm = smem_u32(smem) + warp * (kStages * 2 * SLICE);
-  const int n_slices = (c1 - c0 + 15) / 16;
-  const float scale2 = kLog2e * rsqrtf((float)D);
-
-  // this CTA's slice of the index list, staged once with coalesced loads
-  int* idx_s = reinterpret_cast<int*>(smem + main_bytes<D>());
-  const bool staged = list != nullptr && (c1 - c0) <= kIdxStage;
-  if (staged) {
-    for (int i = threadIdx.x; i < c1 - c0; i += blockDim.x) idx_s[i] = __ldg(list + c0 + i);
-    __syncthreads();
-  }
-
-  // lanes 2r, 2r+1 copy row r; each instruction moves 32 contiguous bytes per row
-  auto issue = [&](int slice, int stage) {
-    const int rel = slice * 16 + (lane >> 1);
-    const int pos = c0 + rel;
-    const bool ok = pos < c1;
-    const int key = !ok ? 0 : (list ? (staged ? idx_s[rel] : __ldg(list + pos)) : pos);
-    const uint32_t kdst = wsm + stage * 2 * SLICE;
-    const uint32_t vdst = kdst + SLICE;
-    const int r = lane >> 1;
+    cp_async_commit();
+  };
+  // K rows g and 8+g of slice s into registers (zero past the list end)
+  uint4 kr[2][KS];
+  auto load_k = [&](int s) {
 #pragma unroll
-    for (int i = 0; i < CH / 2; ++i) {
-      const int ch = 2 * i + (lane & 1);
-      cp_async_16(kdst + swz<D>(r, ch), kb + (size_t)key * D + ch * 8, ok ? 16 : 0);
-      cp_async_16(vdst + swz<D>(r, ch), vb + (size_t)key * D + ch * 8, ok ? 16 : 0);
+    for (int t = 0; t < 2; ++t) {
+      const int rel = s * 16 + t * 8 + g;
+      const bool have = c0 + rel < c1;
+      const __nv_bfloat16* row = kb + (size_t)(have ? key_of(rel) : 0) * D + 8 * c;
+#pragma unroll
+      for (int q = 0; q < KS; ++q) kr[t][q] = have ? ldg_nc_v4(row + 32 * q) : make_uint4(0, 0, 0, 0);
     }
   };
 
@@ -139,51 +171,47 @@ __global__ void __launch_bounds__(kWarps * 32) decode_attn_kernel(const AttnArgs
   float oacc[D / 8][2];
 #pragma unroll
   for (int nd = 0; nd < D / 8; ++nd) oacc[nd][0] = oacc[nd][1] = 0.f;
+  const float scale2 = kLog2e * rsqrtf((float)D);
+  const char* qrow = smem + L::qs + (size_t)(g * D + 8 * c) * 2;
 
-  // this warp's slices: warp, warp + W, ...; up to kStages - 1 in flight ahead
-  int s_issue = warp;
-#pragma unroll
-  for (int st = 0; st < kStages - 1; ++st) {
-    if (s_issue < n_slices) issue(s_issue, st);
-    cp_async_commit();
-    s_issue += kWarps;
+  // prologue: V of this warp's first two slices, K of its first slice
+  int s = warp;
+  if (s < n_slices) issue_v(s);
+  if (s + kWarps < n_slices) issue_v(s + kWarps);
+  if (s < n_slices) load_k(s);
+  if (early) {
+    pdl_wait();
+    pdl_launch_dependents();
   }
-  int stage = 0;
-  for (int s = warp; s < n_slices; s += kWarps) {
-    {
-      const int st_next = (stage + kStages - 1) % kStages;
-      if (s_issue < n_slices) issue(s_issue, st_next);
-      cp_async_commit();
-      s_issue += kWarps;
-    }
-    cp_async_wait<kStages - 1>();
-    __syncwarp();
-    const uint32_t ks = wsm + stage * 2 * SLICE;
-    const uint32_t vs = ks + SLICE;
-
-    float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  // the G query rows of this kv head (rows G..7 zero)
+  for (int i = threadIdx.x; i < 8 * (D / 8); i += kThreads) {
+    const int r = i / (D / 8), ch = i - r * (D / 8);
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (r < G) val = *reinterpret_cast<const uint4*>(a.q + (size_t)(b * a.Hq + h * G + r) * D + ch * 8);
+    *reinterpret_cast<uint4*>(smem + L::qs + (r * D + ch * 8) * 2) = val;
+  }
+  __syncthreads();
+  for (; s < n_slices; s += kWarps) {
+    // S = Q K^T: k-step 2q+hf takes dims 32q + 8c + 4hf + {0,1} (a0/b0) and
+    // + {2,3} (a2/b1) of the query rows and key rows
+    float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-      for (int kk = 0; kk < D / 16; kk += 2) {
-        uint32_t r4[4];
-        ldmatrix_x4(r4, ks + swz<D>(nt * 8 + (lane & 7), 2 * kk + (lane >> 3)));
-        const uint32_t a0[4] = {qa[kk][0], 0u, qa[kk][1], 0u};
-        mma_bf16_16816(sacc[nt], a0, r4[0], r4[1]);
-        const uint32_t a1[4] = {qa[kk + 1][0], 0u, qa[kk + 1][1], 0u};
-        mma_bf16_16816(sacc[nt], a1, r4[2], r4[3]);
-      }
+    for (int q = 0; q < KS; ++q) {
+      const uint2 qlo = *reinterpret_cast<const uint2*>(qrow + 64 * q);       // dims 32q+8c+0..3
+      const uint2 qhi = *reinterpret_cast<const uint2*>(qrow + 64 * q + 8);   // dims 32q+8c+4..7
+      const uint32_t a0[4] = {qlo.x, 0u, qlo.y, 0u};
+      const uint32_t a1[4] = {qhi.x, 0u, qhi.y, 0u};
+      mma_bf16_16816(s0, a0, kr[0][q].x, kr[0][q].y);
+      mma_bf16_16816(s1, a0, kr[1][q].x, kr[1][q].y);
+      mma_bf16_16816(s0, a1, kr[0][q].z, kr[0][q].w);
+      mma_bf16_16816(s1, a1, kr[1][q].z, kr[1][q].w);
     }
     const int kbase = c0 + s * 16;
     float sv[4];
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int key = kbase + nt * 8 + 2 * c + e;
-        sv[nt * 2 + e] = key < c1 ? sacc[nt][e] * scale2 : -INFINITY;
-      }
-    }
+    sv[0] = kbase + 2 * c < c1 ? s0[0] * scale2 : -INFINITY;
+    sv[1] = kbase + 2 * c + 1 < c1 ? s0[1] * scale2 : -INFINITY;
+    sv[2] = kbase + 8 + 2 * c < c1 ? s1[0] * scale2 : -INFINITY;
+    sv[3] = kbase + 9 + 2 * c < c1 ? s1[1] * scale2 : -INFINITY;
     float mx = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
@@ -194,19 +222,18 @@ __global__ void __launch_bounds__(kWarps * 32) decode_attn_kernel(const AttnArgs
     for (int e = 0; e < 4; ++e) p[e] = exp2f(sv[e] - m_new);
     l_run = l_run * alpha + (p[0] + p[1] + p[2] + p[3]);
     m_run = m_new;
-#pragma unroll
-    for (int nd = 0; nd < D / 8; ++nd) {
-      oacc[nd][0] *= alpha;
-      oacc[nd][1] *= alpha;
-    }
     const uint32_t pa[4] = {pack_bf16(p[0], p[1]), 0u, pack_bf16(p[2], p[3]), 0u};
+    // V of this slice: its copy group is the oldest one still pending
+    if (s + kWarps < n_slices) cp_async_wait<1>(); else cp_async_wait<0>();
+    __syncwarp();
+    const uint32_t vs = vbase + ((s / kWarps) & 1) * L::SLOT;
 #pragma unroll
     for (int nd = 0; nd < D / 8; nd += 2) {
       uint32_t r4[4];
       const int mi = lane >> 3;
-      ldmatrix_x4_trans(r4, vs + swz<D>((mi & 1) * 8 + (lane & 7), nd + (mi >> 1)));
-      float t0[4] = {oacc[nd][0], oacc[nd][1], 0.f, 0.f};
-      float t1[4] = {oacc[nd + 1][0], oacc[nd + 1][1], 0.f, 0.f};
+      ldmatrix_x4_trans(r4, vs + ((mi & 1) * 8 + (lane & 7)) * L::ROW + (nd + (mi >> 1)) * 16);
+      float t0[4] = {oacc[nd][0] * alpha, oacc[nd][1] * alpha, 0.f, 0.f};
+      float t1[4] = {oacc[nd + 1][0] * alpha, oacc[nd + 1][1] * alpha, 0.f, 0.f};
       mma_bf16_16816(t0, pa, r4[0], r4[1]);
       mma_bf16_16816(t1, pa, r4[2], r4[3]);
       oacc[nd][0] = t0[0];
@@ -215,119 +242,86 @@ __global__ void __launch_bounds__(kWarps * 32) decode_attn_kernel(const AttnArgs
       oacc[nd + 1][1] = t1[1];
     }
     __syncwarp();
-    stage = (stage + 1) % kStages;
+    if (s + 2 * kWarps < n_slices) issue_v(s + 2 * kWarps);   // refill the slot just read
+    if (s + kWarps < n_slices) load_k(s + kWarps);
   }
   cp_async_wait<0>();
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
 
-  // merge the warps of this CTA, then push the partial to the CTAs that own
-  // each output element (remote stores do not stall the issuing thread)
+  // ---------------- merge the warps into this CTA's partial
   __syncthreads();
-  using P = Post<D>;
-  float* recv_o = reinterpret_cast<float*>(smem + recv_off<D>());
-  float* recv_ml = recv_o + 8 * D;
-  float* red_o = reinterpret_cast<float*>(smem + P::red_o);
-  float* red_ml = reinterpret_cast<float*>(smem + P::red_ml);
+  float* red_o = reinterpret_cast<float*>(smem + L::red_o);
+  float* red_ml = reinterpret_cast<float*>(smem + L::red_ml);
   if (g < G) {
 #pragma unroll
-    for (int nd = 0; nd < D / 8; ++nd) {
-      red_o[(warp * 8 + g) * D + nd * 8 + 2 * c] = oacc[nd][0];
-      red_o[(warp * 8 + g) * D + nd * 8 + 2 * c + 1] = oacc[nd][1];
-    }
+    for (int nd = 0; nd < D / 8; ++nd)
+      *reinterpret_cast<float2*>(red_o + (warp * 8 + g) * L::RO + nd * 8 + 2 * c) =
+          make_float2(oacc[nd][0], oacc[nd][1]);
     if (c == 0) {
       red_ml[(warp * 8 + g) * 2] = m_run;
       red_ml[(warp * 8 + g) * 2 + 1] = l_run;
     }
   }
   __syncthreads();
+  // per-head weights of the warps
+  float* wf = reinterpret_cast<float*>(smem + L::wf);
+  float* pml = reinterpret_cast<float*>(smem + L::pml);
+  if (warp == 0) merge_weights(kWarps, G, red_ml, wf, pml, lane);
+  __syncthreads();
+  // push element e to CTA e / en (E is a multiple of the cluster size)
+  float* recv_o = reinterpret_cast<float*>(smem + L::recv_o);
+  float* recv_ml = reinterpret_cast<float*>(smem + L::recv_ml);
   const int E = G * D;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    const int gg = e / D;
-    float M = -INFINITY;
+  const int en = E / CS;
+  for (int e = threadIdx.x; e < E; e += kThreads) {
+    const int gg = e / D, dd = e - gg * D;
+    float acc = 0.f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, red_ml[(w * 8 + gg) * 2]);
-    float acc = 0.f, lsum = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      const float f = scale_from(red_ml[(w * 8 + gg) * 2], M);
-      acc += f * red_o[(w * 8 + gg) * D + (e - gg * D)];
-      lsum += f * red_ml[(w * 8 + gg) * 2 + 1];
-    }
-    // owner of element e and its slot: slices [E*q/CS, E*(q+1)/CS)
-    int q = (int)(((long)e * CS) / E);
-    while ((int)((long)E * (q + 1) / CS) <= e) ++q;
-    while ((int)((long)E * q / CS) > e) --q;
-    const int q0 = (int)((long)E * q / CS), qn = (int)((long)E * (q + 1) / CS) - q0;
-    float* dst = cluster.map_shared_rank(recv_o, q);
-    dst[rank * qn + (e - q0)] = acc;
-    if (e - gg * D == 0) {
-      for (int r = 0; r < CS; ++r) {
-        float* ml = cluster.map_shared_rank(recv_ml, r);
-        ml[(rank * 8 + gg) * 2] = M;
-        ml[(rank * 8 + gg) * 2 + 1] = lsum;
-      }
-    }
+    for (int w = 0; w < kWarps; ++w) acc += wf[w * 8 + gg] * red_o[(w * 8 + gg) * L::RO + dd];
+    const int q = e / en;
+    *cluster.map_shared_rank(recv_o + rank * en + (e - q * en), q) = acc;
+  }
+  if (threadIdx.x < CS * G) {
+    const int r = threadIdx.x / G, gg = threadIdx.x - r * G;
+    float* ml = cluster.map_shared_rank(recv_ml, r);
+    ml[(rank * 8 + gg) * 2] = pml[gg * 2];
+    ml[(rank * 8 + gg) * 2 + 1] = pml[gg * 2 + 1];
   }
   cluster.sync();
 
-  // merge this CTA's element slice from local shared memory
-  float* wts = reinterpret_cast<float*>(smem + P::wts);    // [CS][8]
-  float* head = reinterpret_cast<float*>(smem + P::head);  // [8]: M, L
-  if (threadIdx.x < G) {
-    const int gg = threadIdx.x;
-    float M = -INFINITY;
-    for (int r = 0; r < CS; ++r) M = fmaxf(M, recv_ml[(r * 8 + gg) * 2]);
-    float L = 0.f;
-    for (int r = 0; r < CS; ++r) {
-      const float f = scale_from(recv_ml[(r * 8 + gg) * 2], M);
-      wts[r * 8 + gg] = f;
-      L += f * recv_ml[(r * 8 + gg) * 2 + 1];
-    }
-    head[gg * 2] = M;
-    head[gg * 2 + 1] = L;
-  }
+  // ---------------- merge this CTA's element slice from local shared memory
+  float* wts = reinterpret_cast<float*>(smem + L::wts);
+  float* head = reinterpret_cast<float*>(smem + L::head);
+  if (warp == 0) merge_weights(CS, G, recv_ml, wts, head, lane);
   __syncthreads();
-  const int e0 = (int)((long)E * rank / CS), e1 = (int)((long)E * (rank + 1) / CS);
-  const int en = e1 - e0;
-  for (int e = e0 + (int)threadIdx.x; e < e1; e += blockDim.x) {
+  const int e0 = rank * en, e1 = e0 + en;
+  for (int e = e0 + (int)threadIdx.x; e < e1; e += kThreads) {
     const int gg = e / D, dd = e - gg * D;
     float acc = 0.f;
     for (int r = 0; r < CS; ++r) acc += wts[r * 8 + gg] * recv_o[r * en + (e - e0)];
-    const float L = head[gg * 2 + 1];
+    const float Ls = head[gg * 2 + 1];
     const size_t orow = (size_t)(b * a.Hq + h * G + gg);
-    a.o[orow * D + dd] = __float2bfloat16(L > 0.f ? acc / L : 0.f);
-    if (dd == 0 && a.lse) a.lse[orow] = L > 0.f ? (head[gg * 2] + log2f(L)) * (float)kLn2 : -INFINITY;
+    a.o[orow * D + dd] = __float2bfloat16(Ls > 0.f ? acc / Ls : 0.f);
+    if (dd == 0 && a.lse) a.lse[orow] = Ls > 0.f ? (head[gg * 2] + log2f(Ls)) * (float)kLn2 : -INFINITY;
   }
 }
 
 template <int D>
-cudaError_t launch(const AttnArgs& a, cudaStream_t stream, int cs, int per) {
-  const size_t sm = smem_bytes<D>();
-  cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-  if (e != cudaSuccess) return e;
-  if (cs > 8) {
-    e = cudaFuncSetAttribute(decode_attn_kernel<D>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-  }
+cudaLaunchConfig_t make_cfg(int cs, int bh, cudaStream_t stream, cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(cs, a.B * a.Hkv, 1);
-  cfg.blockDim = dim3(kWarps * 32, 1, 1);
-  cfg.dynamicSmemBytes = sm;
+  cfg.gridDim = dim3(cs, bh, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Lay<D>::total;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = cs;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_attn_kernel<D>, a, per);
+  return cfg;
 }
-
-}  // namespace
-
-int decode_attn_cluster_size() { return kMaxCS; }
 
 // 16-CTA clusters when the device can co-schedule them, else 8
 template <int D>
@@ -337,22 +331,12 @@ int cluster_size_for_device() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 8;
   if (cached[dev]) return cached[dev];
   int cs = 8;
-  const size_t sm = smem_bytes<D>();
-  if (cudaFuncSetAttribute(decode_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) ==
-          cudaSuccess &&
+  if (cudaFuncSetAttribute(decode_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)Lay<D>::total) == cudaSuccess &&
       cudaFuncSetAttribute(decode_attn_kernel<D>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
           cudaSuccess) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(kMaxCS, 1, 1);
-    cfg.blockDim = dim3(kWarps * 32, 1, 1);
-    cfg.dynamicSmemBytes = sm;
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kMaxCS;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cudaLaunchConfig_t cfg = make_cfg<D>(kMaxCS, 1, nullptr, attr);
     int n = 0;
     if (cudaOccupancyMaxActiveClusters(&n, decode_attn_kernel<D>, &cfg) == cudaSuccess && n > 0) cs = kMaxCS;
   }
@@ -361,13 +345,29 @@ int cluster_size_for_device() {
   return cs;
 }
 
-cudaError_t launch_decode_attn(const AttnArgs& a, cudaStream_t stream) {
+template <int D>
+cudaError_t launch(const AttnArgs& a, cudaStream_t stream) {
+  const int cs = cluster_size_for_device<D>();
   const int list_len = a.idx ? topk_count(a.N, a.num, a.den) : a.N;
-  const int cs = a.D == 128 ? cluster_size_for_device<128>() : cluster_size_for_device<64>();
   int per = (list_len + cs - 1) / cs;
   per = (per + 15) / 16 * 16;
   if (per < 16) per = 16;
-  return a.D == 128 ? launch<128>(a, stream, cs, per) : launch<64>(a, stream, cs, per);
+  if ((a.G * D) % cs != 0) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)Lay<D>::total);
+  if (e != cudaSuccess) return e;
+  if (cs > 8) {
+    e = cudaFuncSetAttribute(decode_attn_kernel<D>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_ex(decode_attn_kernel<D>, dim3(cs, a.B * a.Hkv), dim3(kThreads), Lay<D>::total, stream,
+                   (a.flags & 1) != 0, cs, a, per);
+}
+
+}  // namespace
+
+cudaError_t launch_decode_attn(const AttnArgs& a, cudaStream_t stream) {
+  return a.D == 128 ? launch<128>(a, stream) : launch<64>(a, stream);
 }
 
 }  // namespace kascade

@@ -28,6 +28,8 @@ __global__ void __launch_bounds__(kScoreWarps * 32)
                         float* __restrict__ s2, float* __restrict__ m_part,
                         double* __restrict__ l_part, int N, int Hq, int Hkv, int G, int splits,
                         float scale2) {
+  pdl_wait();
+  pdl_launch_dependents();
   constexpr int CH = D / 32;
   constexpr int KEYS = 16 * kScoreWarps * kGroupsPerWarp;
   const int split = blockIdx.x;
@@ -165,13 +167,12 @@ cudaError_t launch_decode_score(const DecodeScoreArgs& a, cudaStream_t stream) {
   const int splits = (a.N + decode_score_keys_per_split() - 1) / decode_score_keys_per_split();
   dim3 grid(splits, a.B * a.Hkv);
   const float scale2 = kLog2e / sqrtf((float)a.D);
+  const bool pdl = (a.flags & 1) != 0;
   if (a.D == 128)
-    decode_score_kernel<128><<<grid, kScoreWarps * 32, 0, stream>>>(
-        a.q, a.k, a.s2, a.m_part, a.l_part, a.N, a.Hq, a.Hkv, a.G, splits, scale2);
-  else
-    decode_score_kernel<64><<<grid, kScoreWarps * 32, 0, stream>>>(
-        a.q, a.k, a.s2, a.m_part, a.l_part, a.N, a.Hq, a.Hkv, a.G, splits, scale2);
-  return cudaGetLastError();
+    return launch_ex(decode_score_kernel<128>, grid, dim3(kScoreWarps * 32), 0, stream, pdl, 1, a.q, a.k, a.s2,
+                     a.m_part, a.l_part, a.N, a.Hq, a.Hkv, a.G, splits, scale2);
+  return launch_ex(decode_score_kernel<64>, grid, dim3(kScoreWarps * 32), 0, stream, pdl, 1, a.q, a.k, a.s2,
+                   a.m_part, a.l_part, a.N, a.Hq, a.Hkv, a.G, splits, scale2);
 }
 
 }  // namespace kascade

@@ -14,6 +14,7 @@ struct DecodeScoreArgs {
   float* m_part;           // [B, Hq, splits]
   double* l_part;          // [B, Hq, splits]
   int B, Hq, Hkv, G, D, N;
+  int flags;
 };
 int decode_score_keys_per_split();
 cudaError_t launch_decode_score(const DecodeScoreArgs& a, cudaStream_t stream);
@@ -41,6 +42,7 @@ struct SelArgs {
   int n_max;
   int grid;
   int32_t* idx;            // output
+  int flags;
 };
 size_t select_scratch_bytes_per_cta(int n_max);
 // decode: one 8-CTA cluster per (batch, kv head) when N / 8 <= 16384
@@ -58,6 +60,7 @@ struct ScorePoolArgs {
   double* row_l;           // [B, Hq, N]
   float* pooled;           // [B, Hkv, sum_t e_t]
   int B, Hq, Hkv, G, D, N, tile;
+  int flags;
 };
 cudaError_t launch_score_pool(const ScorePoolArgs& a, cudaStream_t stream);
 
@@ -72,6 +75,8 @@ struct AttnArgs {
   float* lse;                // may be NULL
   int B, Hq, Hkv, G, D, N, tile, num, den;
   bool causal;               // prefill dense only
+  int* err;                  // device error word (a bounded wait gave up), may be NULL
+  int flags;                 // KASCADE_FLAG_* bits
 };
 // decode: one 16-CTA cluster per (batch, kv head), merge over DSMEM
 cudaError_t launch_decode_attn(const AttnArgs& a, cudaStream_t stream);

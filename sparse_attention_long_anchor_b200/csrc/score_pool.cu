@@ -33,6 +33,8 @@ __device__ __forceinline__ uint32_t sp_swz(int r, int ch) {
 
 template <int D>
 __global__ void __launch_bounds__(kSpWarps * 32) score_pool_kernel(const ScorePoolArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
   constexpr int CH = D / 8;
   constexpr int KBLK_BYTES = kSpKeys * D * 2;
   extern __shared__ __align__(128) char smem[];
@@ -242,11 +244,11 @@ cudaError_t launch_score_pool(const ScorePoolArgs& a, cudaStream_t stream) {
   if (a.D == 128) {
     const size_t sm = score_pool_smem<128>();
     cudaFuncSetAttribute(score_pool_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    score_pool_kernel<128><<<grid, kSpWarps * 32, sm, stream>>>(a);
+    return launch_ex(score_pool_kernel<128>, grid, dim3(kSpWarps * 32), sm, stream, (a.flags & 1) != 0, 1, a);
   } else {
     const size_t sm = score_pool_smem<64>();
     cudaFuncSetAttribute(score_pool_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    score_pool_kernel<64><<<grid, kSpWarps * 32, sm, stream>>>(a);
+    return launch_ex(score_pool_kernel<64>, grid, dim3(kSpWarps * 32), sm, stream, (a.flags & 1) != 0, 1, a);
   }
   return cudaGetLastError();
 }

@@ -103,6 +103,8 @@ __device__ void cluster_exchange(cg::cluster_group& cluster, CSh& sh, int slot, 
 
 __global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(kCNT)
     select_decode_cluster_kernel(const SelArgs a, int keys_per_cta) {
+  pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ __align__(128) char smem_raw[];
   CSh& sh = *reinterpret_cast<CSh*>(smem_raw);
   float* qf = reinterpret_cast<float*>(smem_raw + kCHead);
@@ -362,8 +364,7 @@ cudaError_t launch_select_decode_cluster(const SelArgs& a, cudaStream_t stream) 
                                        (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(kCS, a.B * a.Hkv);
-  select_decode_cluster_kernel<<<grid, kCNT, smem, stream>>>(a, per);
-  return cudaGetLastError();
+  return launch_ex(select_decode_cluster_kernel, grid, dim3(kCNT), smem, stream, (a.flags & 1) != 0, 1, a, per);
 }
 
 }  // namespace kascade

@@ -37,6 +37,8 @@ constexpr int kPreKeys = 64;
 template <int D>
 __global__ void __launch_bounds__(kPreWarps * 32)
     prefill_attn_kernel(const AttnArgs a, int row_blocks) {
+  pdl_wait();
+  pdl_launch_dependents();
   constexpr int CH = D / 8;
   constexpr int MAT_BYTES = kPreKeys * D * 2;   // one stage of K (or V)
   constexpr int STAGE_BYTES = 2 * MAT_BYTES;
@@ -253,11 +255,13 @@ cudaError_t launch_prefill_attn(const AttnArgs& a, cudaStream_t stream) {
   if (a.D == 128) {
     const size_t sm = prefill_smem<128>();
     cudaFuncSetAttribute(prefill_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    prefill_attn_kernel<128><<<grid, kPreWarps * 32, sm, stream>>>(a, row_blocks);
+    return launch_ex(prefill_attn_kernel<128>, grid, dim3(kPreWarps * 32), sm, stream, (a.flags & 1) != 0, 1, a,
+                     row_blocks);
   } else {
     const size_t sm = prefill_smem<64>();
     cudaFuncSetAttribute(prefill_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    prefill_attn_kernel<64><<<grid, kPreWarps * 32, sm, stream>>>(a, row_blocks);
+    return launch_ex(prefill_attn_kernel<64>, grid, dim3(kPreWarps * 32), sm, stream, (a.flags & 1) != 0, 1, a,
+                     row_blocks);
   }
   return cudaGetLastError();
 }

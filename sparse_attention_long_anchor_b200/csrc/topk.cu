@@ -345,6 +345,8 @@ __device__ void run_problem(const SelArgs& a, Problem& p, SelShared& sh, float* 
 
 template <int NT>
 __global__ void __launch_bounds__(NT) select_kernel(const SelArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ __align__(128) char smem_raw[];
   SelShared& sh = *reinterpret_cast<SelShared*>(smem_raw);
   char* dyn = smem_raw + kSelHead;
@@ -413,8 +415,7 @@ cudaError_t launch_select(const SelArgs& a, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(select_kernel<kSelThreads>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  select_kernel<kSelThreads><<<a.grid, kSelThreads, smem, stream>>>(a);
-  return cudaGetLastError();
+  return launch_ex(select_kernel<kSelThreads>, dim3(a.grid), dim3(kSelThreads), smem, stream, (a.flags & 1) != 0, 1, a);
 }
 
 }  // namespace kascade

@@ -20,10 +20,12 @@ LIB_PATH = os.environ.get("KASCADE_LIB") or os.path.join(os.path.dirname(os.path
 
 OP_SELECT, OP_SPARSE_DECODE, OP_SPARSE_PREFILL, OP_DENSE = 0, 1, 2, 3
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA = 0, 1, 2, 3, 4
+FLAG_PDL, FLAG_INPUTS_STABLE = 1, 2
 
 EXPORTS = ("kascade_workspace_bytes", "kascade_index_count", "kascade_index_offsets",
            "kascade_workspace_init", "kascade_select", "kascade_sparse_decode",
-           "kascade_sparse_prefill", "kascade_dense_ref", "kascade_status_str")
+           "kascade_sparse_prefill", "kascade_dense_ref", "kascade_workspace_error",
+           "kascade_status_str")
 
 
 class KascadeError(RuntimeError):
@@ -37,11 +39,15 @@ class Shape(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("q_len", ctypes.c_int32), ("kv_len", ctypes.c_int32), ("tile", ctypes.c_int32),
-                ("topk_num", ctypes.c_int32), ("topk_den", ctypes.c_int32)]
+                ("topk_num", ctypes.c_int32), ("topk_den", ctypes.c_int32), ("flags", ctypes.c_int32)]
 
     @classmethod
-    def make(cls, batch, hq, hkv, d, q_len, kv_len, frac=(10, 100), tile=32):
-        return cls(batch, hq, hkv, d, q_len, kv_len, tile, frac[0], frac[1])
+    def make(cls, batch, hq, hkv, d, q_len, kv_len, frac=(10, 100), tile=32, flags=0):
+        return cls(batch, hq, hkv, d, q_len, kv_len, tile, frac[0], frac[1], flags)
+
+    def with_flags(self, flags: int) -> "Shape":
+        return Shape(self.batch, self.num_q_heads, self.num_kv_heads, self.head_dim, self.q_len,
+                     self.kv_len, self.tile, self.topk_num, self.topk_den, flags)
 
     @property
     def decode(self) -> bool:
@@ -70,6 +76,8 @@ def _load():
         fn.restype = ctypes.c_int
     so.kascade_dense_ref.argtypes = [SP, P, P, P, ctypes.c_int, P, P, P, ctypes.c_size_t, P]
     so.kascade_dense_ref.restype = ctypes.c_int
+    so.kascade_workspace_error.argtypes = [P, ctypes.POINTER(ctypes.c_int), ctypes.c_int, P]
+    so.kascade_workspace_error.restype = ctypes.c_int
     so.kascade_status_str.argtypes = [ctypes.c_int]
     so.kascade_status_str.restype = ctypes.c_char_p
     return so
@@ -136,11 +144,18 @@ class Workspace:
     def args(self):
         return self.ptr, self.nbytes
 
+    def error(self, clear=True, stream=None) -> int:
+        """The device error word (0 = no kernel gave up on a bounded wait)."""
+        out = ctypes.c_int(0)
+        _check(lib.kascade_workspace_error(self.ptr, ctypes.byref(out), int(clear), _stream(stream)),
+               "kascade_workspace_error")
+        return out.value
+
 
 def _ws(ws, shape, op):
     if ws is None:
-        if workspace_bytes(shape, op) == 0:
-            return None, 0
+        if op != OP_SELECT:
+            return None, 0       # attention calls run without an error word
         ws = Workspace(shape, (op,))
     return ws.args()
 

@@ -20,7 +20,7 @@ def _declared():
 def test_library_exports_every_declared_symbol():
     from sparse_attention_long_anchor_b200 import kascade as kc
     names = _declared()
-    assert len(names) >= 9
+    assert len(names) >= 10
     assert set(names) == set(kc.EXPORTS)
     for n in names:
         assert hasattr(kc.lib, n), n
@@ -48,9 +48,9 @@ def test_index_layout_matches_oracle(n_ctx, frac):
 def test_workspace_sizes_positive():
     kc = _kc()
     s = kc.Shape.make(1, 32, 8, 128, 1, 32768)
-    assert kc.workspace_bytes(s, kc.OP_SELECT) > 0
+    assert kc.workspace_bytes(s, kc.OP_SELECT) > 256
     for op in (kc.OP_SPARSE_DECODE, kc.OP_SPARSE_PREFILL, kc.OP_DENSE):
-        assert kc.workspace_bytes(s, op) == 0
+        assert kc.workspace_bytes(s, op) == 256
     p = kc.Shape.make(1, 32, 8, 128, 32768, 32768)
     assert kc.workspace_bytes(p, kc.OP_SELECT) > 0
 
@@ -83,7 +83,7 @@ def test_null_and_misaligned_pointers_and_small_workspace():
     assert L.kascade_select(sb, 256, 256, 256, None, need, None) == kc.ERR_WORKSPACE
     assert L.kascade_select(sb, 256, 256, 256, 258, need, None) == kc.ERR_WORKSPACE
     nd = kc.workspace_bytes(s, kc.OP_SPARSE_DECODE)
-    assert nd == 0   # attention kernels keep partials on chip
+    assert nd == 256   # only the error-word header: attention partials stay on chip
     assert L.kascade_sparse_decode(sb, 256, 256, 256, None, None, 256, None, None, 0, None) == kc.ERR_INVALID_ARG
     assert L.kascade_sparse_decode(sb, 256, 256, None, 256, None, 256, None, None, 0, None) == kc.ERR_INVALID_ARG
     assert L.kascade_sparse_decode(sb, None, 256, 256, 256, None, 256, None, None, 0, None) == kc.ERR_INVALID_ARG
@@ -96,6 +96,9 @@ def test_null_and_misaligned_pointers_and_small_workspace():
         == kc.ERR_UNSUPPORTED
     assert L.kascade_workspace_init(None, 16, None) == kc.ERR_WORKSPACE
     assert L.kascade_index_offsets(sb, None) == kc.ERR_INVALID_ARG
+    out = ctypes.c_int(0)
+    assert L.kascade_workspace_error(None, ctypes.byref(out), 0, None) == kc.ERR_INVALID_ARG
+    assert L.kascade_workspace_error(256, None, 0, None) == kc.ERR_INVALID_ARG
 
 
 def test_status_strings():

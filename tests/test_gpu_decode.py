@@ -33,6 +33,7 @@ def _run_decode(B, Hq, Hkv, d, N, frac, seed=0, zero_q=False, head_map=None, n_s
     o_ref, lse_ref = O.sparse_decode(qn, kn, vn, idx_g, head_map)
     check_out(np64(o).reshape(B, Hq, d), o_ref, "sparse decode")
     check_lse(lse.cpu().numpy(), lse_ref, "sparse decode lse")
+    assert ws.error() == 0
     return q, k, v, idx_g, tally
 
 
@@ -129,3 +130,27 @@ def test_decode_llama_stack_layers():
     check_out(np64(o0).reshape(1, cfg.hq, cfg.d), o_ref, "anchor layer")
     o_ref1, _ = O.sparse_decode(np64(q1), np64(k1), np64(v1), idx_g, hm)
     check_out(np64(o1).reshape(1, cfg.hq, cfg.d), o_ref1, "reuse layer")
+
+
+def test_decode_pdl_flags_give_identical_results():
+    """Programmatic dependent launch (and early gathers for inputs written two
+    launches back) changes scheduling only, never results."""
+    kc = _kc()
+    B, Hq, Hkv, d, N, frac = 1, 32, 8, 128, 8192, (10, 100)
+    q, k, v = gen_inputs(dict(B=B, Hq=Hq, Hkv=Hkv, d=d, N=N), seed=21)
+    q2, k2, v2 = gen_inputs(dict(B=B, Hq=Hq, Hkv=Hkv, d=d, N=N), seed=22)
+    hm = torch.tensor([1, 0, 3, 2, 5, 4, 7, 6], dtype=torch.int32, device="cuda")
+    outs = []
+    for flags in (0, kc.FLAG_PDL, kc.FLAG_PDL | kc.FLAG_INPUTS_STABLE):
+        s = kc.Shape.make(B, Hq, Hkv, d, 1, N, frac, flags=flags & kc.FLAG_PDL)
+        ws = kc.Workspace(s)
+        idx = kc.select(s, q, k, ws=ws)
+        o0 = kc.sparse_decode(s, q, k, v, idx, None, ws=ws)
+        o1 = kc.sparse_decode(s.with_flags(flags), q2, k2, v2, idx, hm, ws=ws)
+        o2 = kc.sparse_decode(s.with_flags(flags), q, k2, v2, idx, hm, ws=ws)
+        torch.cuda.synchronize()
+        assert ws.error() == 0
+        outs.append((idx.clone(), o0.clone(), o1.clone(), o2.clone()))
+    for other in outs[1:]:
+        for x, y in zip(outs[0], other):
+            assert torch.equal(x, y)
