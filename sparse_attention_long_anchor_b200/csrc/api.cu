@@ -115,6 +115,14 @@ SelectPlan plan_select(const kascade_shape* s, void* ws) {
   return p;
 }
 
+int device_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      n <= 0)
+    return kPlanSMs;
+  return n;
+}
+
 int* err_word(void* ws, size_t ws_bytes) {
   return (ws && ws_bytes >= sizeof(int) && aligned(ws, 4)) ? static_cast<int*>(ws) : nullptr;
 }
@@ -274,7 +282,8 @@ int kascade_select(const kascade_shape* s, const void* q, const void* k, int32_t
     sp.D = a.D;
     sp.N = a.N;
     sp.tile = 32;
-    rc = cuda_status(launch_score_pool(sp, st));
+    rc = cuda_status(score_pool_tc_supported(sp) ? launch_score_pool_tc(sp, err_word(ws, ws_bytes), device_sms(), st)
+                                                 : launch_score_pool(sp, st));
     if (rc) return rc;
     a.pooled = pl.pooled;
     a.row_m2 = pl.row_m2;

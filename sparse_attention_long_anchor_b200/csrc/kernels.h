@@ -63,6 +63,9 @@ struct ScorePoolArgs {
   int flags;
 };
 cudaError_t launch_score_pool(const ScorePoolArgs& a, cudaStream_t stream);
+// tcgen05/TMEM + TMA version (G <= 4); err: device error word (may be NULL)
+bool score_pool_tc_supported(const ScorePoolArgs& a);
+cudaError_t launch_score_pool_tc(const ScorePoolArgs& a, int* err, int num_sms, cudaStream_t stream);
 
 // Sparse / dense attention over an index list (decode: split-K + combine).
 struct AttnArgs {
