@@ -15,10 +15,12 @@
 // items longest tile first.  Per CTA:
 //   warp 0      TMA producer: the Q tile (32-row boxes, one per head) and a
 //               ring of kStages K blocks of 128 keys, 128-byte swizzled;
-//   warp 1      single-thread tcgen05.mma issue (M = N = 128, K = 16 steps)
-//               into two 128-column TMEM accumulators; owns TMEM;
-//   warps 2..5  epilogue: tcgen05.ld of one TMEM lane quarter each, online
-//               row statistics (pass 1), masked column sums (pass 2).
+//   warp 1      single-thread tcgen05.mma issue (M = N = 128, K = 16 steps);
+//               owns TMEM;
+//   warps 2..9  epilogue: two warpgroups take alternate K blocks (four
+//               128-column TMEM accumulators); tcgen05.ld of one TMEM lane
+//               quarter per warp, online row statistics (pass 1, merged
+//               across the groups per tile), masked column sums (pass 2).
 // All hand-offs are mbarriers; every wait is bounded and a timeout stops the
 // CTA's loops and records an error code.
 #include "common.cuh"
@@ -31,7 +33,9 @@ namespace {
 
 constexpr int kStages = 4;
 constexpr int kKB = 128;          // keys per block
-constexpr int kThreads = 192;     // 6 warps
+constexpr int kEpiGroups = 2;     // epilogue warpgroups, alternating K blocks
+constexpr int kBufs = 4;          // TMEM accumulators of 128 columns
+constexpr int kThreads = 64 + 128 * kEpiGroups;
 constexpr int kErrTimeout = 2;
 
 template <int D>
@@ -43,19 +47,20 @@ struct SPL {
   static constexpr size_t q = 0;
   static constexpr size_t k = q + QTILE;
   static constexpr size_t bars = k + (size_t)kStages * KTILE;
-  // q_full, q_empty, k_full[S], k_empty[S], acc_full[2], acc_empty[2], drain
-  static constexpr int NBARS = 2 + 2 * kStages + 4 + 1;
+  // q_full, q_empty, k_full[S], k_empty[S], acc_full[B], acc_empty[B], drain
+  static constexpr int NBARS = 2 + 2 * kStages + 2 * kBufs + 1;
   static constexpr size_t tslot = bars + NBARS * 8;
   static constexpr size_t stop = (tslot + 8 + 15) / 16 * 16;
   static constexpr size_t bcol = stop + 16;         // [128] f32, read as float4
   static constexpr size_t rpos = bcol + 128 * 4;    // [128] int, read as int4
-  static constexpr size_t total = rpos + 128 * 4;
+  static constexpr size_t pstat = rpos + 128 * 4;   // [groups][128] (m f32, l f64) row partials
+  static constexpr size_t total = pstat + kEpiGroups * 128 * 16;
   static_assert(bcol % 16 == 0 && rpos % 16 == 0, "vector reads of bcol / rpos need 16-byte alignment");
   static_assert(bars % 8 == 0 && k % 1024 == 0, "mbarriers and swizzled tiles alignment");
   static constexpr size_t alloc = total + 1024;     // slack for 1024-byte alignment
 };
 
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;\n" ::: "memory"); }
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;\n" ::"n"(128 * kEpiGroups) : "memory"); }
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -70,8 +75,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar0 = base + (uint32_t)L::bars;
   const uint32_t q_full = bar0, q_empty = bar0 + 8;
   const uint32_t k_full0 = bar0 + 16, k_empty0 = k_full0 + 8 * kStages;
-  const uint32_t acc_full0 = k_empty0 + 8 * kStages, acc_empty0 = acc_full0 + 16;
-  const uint32_t drain = acc_empty0 + 16;
+  const uint32_t acc_full0 = k_empty0 + 8 * kStages, acc_empty0 = acc_full0 + 8 * kBufs;
+  const uint32_t drain = acc_empty0 + 8 * kBufs;
   volatile int* stop = reinterpret_cast<volatile int*>(sm + L::stop);
   float* bcol = reinterpret_cast<float*>(sm + L::bcol);
   int* rpos = reinterpret_cast<int*>(sm + L::rpos);
@@ -90,9 +95,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(k_full0 + 8 * s, 1);
       mbar_init(k_empty0 + 8 * s, 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kBufs; ++b) {
       mbar_init(acc_full0 + 8 * b, 1);
-      mbar_init(acc_empty0 + 8 * b, 4);
+      mbar_init(acc_empty0 + 8 * b, 4);   // one arrival per warp of the consuming warpgroup
     }
     mbar_init(drain, 1);
     *stop = 0;
@@ -105,7 +110,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     *reinterpret_cast<uint4*>(sm + L::q + cb * L::CBYTES + r * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
   }
   asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-  if (warp == 1) tc::tmem_alloc(base + (uint32_t)L::tslot, 256);
+  if (warp == 1) tc::tmem_alloc(base + (uint32_t)L::tslot, 128 * kBufs);
   pdl_wait();
   pdl_launch_dependents();
   tc::fence_before();
@@ -167,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::fence_after();
         for (int pass = 0; pass < 2 && !*stop; ++pass) {
           for (int blk = 0; blk < nb; ++blk) {
-            const int s = kcount % kStages, buf = acount & 1, ause = acount >> 1;
+            const int s = kcount % kStages, buf = acount % kBufs, ause = acount / kBufs;
             if (!mbar_wait_bounded(k_full0 + 8 * s, (kcount / kStages) & 1)) { fail(); break; }
             if (ause > 0 && !mbar_wait_bounded(acc_empty0 + 8 * buf, (ause - 1) & 1)) { fail(); break; }
             tc::fence_after();
@@ -197,12 +202,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
+    // warpgroup wg takes the K blocks with block sequence number = wg (mod 2);
+    // warp w reads TMEM lanes 32 (w % 4) .. +31
+    const int ew = warp - 2;
+    const int wg = ew >> 2;
+    const int quarter = warp & 3;
     const int r = 32 * quarter + lane;       // pass 1: query row; pass 2: key within the block
     const uint32_t lane_addr = (uint32_t)(32 * quarter) << 16;
     const float scale2 = kLog2e * rsqrtf((float)D);
+    float* pm = reinterpret_cast<float*>(sm + L::pstat);                   // [groups][128]
+    double* pl = reinterpret_cast<double*>(sm + L::pstat + kEpiGroups * 128 * 4);
     int acount = 0;
-    // the four epilogue warps meet at named barriers, so their loops stay
+    // the epilogue warps meet at named barriers, so their loops stay
     // uniform: after a failure the waits are skipped, never the structure
     auto wait_acc = [&](int buf, int par) -> bool {
       if (*stop) return false;
@@ -219,12 +230,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int nb = (e_t + kKB - 1) / kKB;
       const bool valid = quarter < G && lane < rows_t;
       const int pos = i0 + lane;
-      // ---- pass 1: row statistics of row r (head `quarter`, query i0 + lane)
-      float m = -INFINITY;
-      double l = 0.0;
-      for (int blk = 0; blk < nb; ++blk) {
-        const int buf = acount & 1;
-        wait_acc(buf, (acount >> 1) & 1);
+      // ---- pass 1: statistics of row r over this warpgroup's blocks.  The
+      // running shift m2 is the fp32 value that gets stored, and every term is
+      // exp2(fma(dot, scale2, -m2)) with a single rounding, so that the stored
+      // (m2, l) pair is consistent term by term
+      float m2 = -INFINITY;  // running max of dot * scale2 (fp32)
+      double l = 0.0;        // sum of exp2(dot * scale2 - m2)
+      for (int blk = 0; blk < nb; ++blk, ++acount) {
+        if ((acount & 1) != wg) continue;
+        const int buf = acount % kBufs;
+        wait_acc(buf, (acount / kBufs) & 1);
         tc::fence_after();
         const int j0 = blk * kKB;
         const bool diag = j0 + kKB - 1 > i0;   // block reaches the tile: mask j > pos
@@ -233,49 +248,71 @@ __global__ void __launch_bounds__(kThreads, 1)
           float v[32];
           tc::tmem_ld32(tmem + lane_addr + (uint32_t)(buf * 128 + ch * 32), v);
           if (!valid) continue;
-          float cm = -INFINITY;
+          if (diag) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            float s = v[i] * scale2;
-            if (diag && j0 + ch * 32 + i > pos) s = -INFINITY;
-            v[i] = s;
-            cm = fmaxf(cm, s);
+            for (int i = 0; i < 32; ++i)
+              if (j0 + ch * 32 + i > pos) v[i] = -INFINITY;
           }
-          if (cm > m) {
-            if (m != -INFINITY) l *= exp2((double)m - (double)cm);
-            m = cm;
-          }
-          if (m != -INFINITY) {
-            float part = 0.f;
+          float cm = v[0];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) part += exp2f(v[i] - m);
-            l += (double)part;
+          for (int i = 1; i < 32; ++i) cm = fmaxf(cm, v[i]);
+          const float cm2 = cm * scale2;   // scale > 0 keeps the order
+          if (cm2 > m2) {
+            if (m2 != -INFINITY) l *= exp2((double)m2 - (double)cm2);
+            m2 = cm2;
+          }
+          if (m2 != -INFINITY) {
+            const float nm2 = -m2;
+            float p0 = 0.f, p1 = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              p0 += exp2f(fmaf(v[i], scale2, nm2));
+              p1 += exp2f(fmaf(v[i + 1], scale2, nm2));
+            }
+            l += (double)(p0 + p1);
           }
         }
         tc::fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_empty0 + 8 * buf);
-        ++acount;
       }
-      epi_bar();   // everyone finished reading the previous item's bcol / rpos
-      if (valid) {
-        const size_t srow = (size_t)(b * a.Hq + h * G + quarter) * a.N + pos;
-        a.row_m2[srow] = m;
-        a.row_l[srow] = l;
-      }
-      bcol[r] = valid ? (float)((double)m + log2(l)) : INFINITY;
-      rpos[r] = valid ? pos : -1;
+      // merge the two warpgroups' row statistics (after every reader of the
+      // previous item's bcol / rpos is done)
+      pm[wg * 128 + r] = m2;
+      pl[wg * 128 + r] = l;
       epi_bar();
-      // ---- pass 2: pooled score of key j0 + r
+      if (wg == 0) {
+        float M2 = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < kEpiGroups; ++e) M2 = fmaxf(M2, pm[e * 128 + r]);
+        double Ls = 0.0;
+        if (M2 != -INFINITY) {
+#pragma unroll
+          for (int e = 0; e < kEpiGroups; ++e) {
+            const float me = pm[e * 128 + r];
+            if (me != -INFINITY) Ls += pl[e * 128 + r] * exp2((double)me - (double)M2);
+          }
+        }
+        if (valid) {
+          const size_t srow = (size_t)(b * a.Hq + h * G + quarter) * a.N + pos;
+          a.row_m2[srow] = M2;
+          a.row_l[srow] = Ls;
+        }
+        bcol[r] = valid ? (float)((double)M2 + log2(Ls)) : INFINITY;
+        rpos[r] = valid ? pos : -1;
+      }
+      epi_bar();
+      // ---- pass 2: pooled score of key j0 + r over this warpgroup's blocks
       const float inv_rows = 1.0f / (float)(G * rows_t);
       float* pooled = a.pooled + (size_t)bh * (tile_pooled_offset(T - 1, a.tile) + a.N) + tile_pooled_offset(t, a.tile);
-      for (int blk = 0; blk < nb; ++blk) {
-        const int buf = acount & 1;
-        wait_acc(buf, (acount >> 1) & 1);
+      for (int blk = 0; blk < nb; ++blk, ++acount) {
+        if ((acount & 1) != wg) continue;
+        const int buf = acount % kBufs;
+        wait_acc(buf, (acount / kBufs) & 1);
         tc::fence_after();
         const int j = blk * kKB + r;
         const bool diag = blk * kKB + kKB - 1 > i0;
-        float colsum = 0.f;
+        float c0 = 0.f, c1 = 0.f;
 #pragma unroll 1
         for (int ch = 0; ch < 4; ++ch) {
           float v[32];
@@ -285,24 +322,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int q4 = 0; q4 < 8; ++q4) {
             const float4 bb = bc[q4];
-            const float b4[4] = {bb.x, bb.y, bb.z, bb.w};
+            float e0 = exp2f(fmaf(v[q4 * 4 + 0], scale2, -bb.x));
+            float e1 = exp2f(fmaf(v[q4 * 4 + 1], scale2, -bb.y));
+            float e2 = exp2f(fmaf(v[q4 * 4 + 2], scale2, -bb.z));
+            float e3 = exp2f(fmaf(v[q4 * 4 + 3], scale2, -bb.w));
             if (diag) {
               const int4 pp = rp[q4];
-              const int p4[4] = {pp.x, pp.y, pp.z, pp.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                colsum += j <= p4[e] ? exp2f(v[q4 * 4 + e] * scale2 - b4[e]) : 0.f;
-            } else {
-#pragma unroll
-              for (int e = 0; e < 4; ++e) colsum += exp2f(v[q4 * 4 + e] * scale2 - b4[e]);
+              e0 = j <= pp.x ? e0 : 0.f;
+              e1 = j <= pp.y ? e1 : 0.f;
+              e2 = j <= pp.z ? e2 : 0.f;
+              e3 = j <= pp.w ? e3 : 0.f;
             }
+            c0 += e0 + e1;
+            c1 += e2 + e3;
           }
         }
         tc::fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_empty0 + 8 * buf);
-        ++acount;
-        if (j < e_t) pooled[j] = colsum * inv_rows;
+        if (j < e_t) pooled[j] = (c0 + c1) * inv_rows;
       }
     }
   }
@@ -312,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc::fence_after();
-    tc::tmem_dealloc(tmem, 256);
+    tc::tmem_dealloc(tmem, 128 * kBufs);
   }
 }
 
