@@ -71,6 +71,7 @@ extern "C" {
 #define KASCADE_ERR_UNSUPPORTED 2  /* d not 64/128, tile != 32, G > 8, q_len not 1 or N, misaligned pointer */
 #define KASCADE_ERR_WORKSPACE 3    /* ws NULL, misaligned or smaller than kascade_workspace_bytes() */
 #define KASCADE_ERR_CUDA 4         /* a CUDA launch or device query failed */
+#define KASCADE_ERR_TOO_LARGE 5    /* the shape needs more scratch than a fixed library buffer holds */
 
 /* Operations for kascade_workspace_bytes(). */
 #define KASCADE_OP_SELECT 0
@@ -178,6 +179,26 @@ KASCADE_API int kascade_sparse_prefill(const kascade_shape* shape, const void* q
 KASCADE_API int kascade_dense_ref(const kascade_shape* shape, const void* q, const void* k,
                       const void* v, int causal, void* o, float* lse,
                       void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Decode anchor selection that allocates nothing and takes no workspace.
+ * The paper has no counterpart: this serves callers that can neither pass
+ * device scratch nor allocate (e.g. an operator inside a host runtime that
+ * pre-plans all device memory).  Same inputs, outputs and results as
+ * kascade_select for a decode shape (q_len == 1).  Its scratch is a fixed
+ * array of kascade_select_decode_static_max_bytes() bytes (8 MiB) inside the
+ * library, held by every GPU that loads the library until the process exits.
+ * The first call on a device looks up the array's device address with that
+ * device current; make that first call before any stream capture.  All calls
+ * share the array: calls that may overlap on the GPU race and must be
+ * serialised by the caller.  Returns KASCADE_ERR_TOO_LARGE, before launching
+ * anything, when the shape needs more than the array holds, and
+ * KASCADE_ERR_UNSUPPORTED for prefill shapes.
+ */
+KASCADE_API int kascade_select_decode_static(const kascade_shape* shape, const void* q, const void* k,
+                                             int32_t* idx, void* stream);
+/* Size in bytes of the fixed scratch array of kascade_select_decode_static. */
+KASCADE_API size_t kascade_select_decode_static_max_bytes(void);
 
 /* Synchronises `stream`, copies the device error word (the first int of
  * `ws`) to *error_out (0 = no failure; 1 = a bounded wait timed out) and, if

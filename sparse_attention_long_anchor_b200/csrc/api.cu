@@ -365,6 +365,8 @@ const char* kascade_status_str(int status) {
       return "workspace missing, misaligned or too small";
     case KASCADE_ERR_CUDA:
       return "CUDA launch or device error";
+    case KASCADE_ERR_TOO_LARGE:
+      return "shape needs more scratch than the library's fixed buffer holds";
     default:
       return "unknown status";
   }

@@ -19,13 +19,13 @@ __all__ = ["Shape", "KascadeError", "lib", "OP_SELECT", "OP_SPARSE_DECODE", "OP_
 LIB_PATH = os.environ.get("KASCADE_LIB") or os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkascade.so")
 
 OP_SELECT, OP_SPARSE_DECODE, OP_SPARSE_PREFILL, OP_DENSE = 0, 1, 2, 3
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA = 0, 1, 2, 3, 4
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TOO_LARGE = 0, 1, 2, 3, 4, 5
 FLAG_PDL, FLAG_INPUTS_STABLE = 1, 2
 
 EXPORTS = ("kascade_workspace_bytes", "kascade_index_count", "kascade_index_offsets",
            "kascade_workspace_init", "kascade_select", "kascade_sparse_decode",
            "kascade_sparse_prefill", "kascade_dense_ref", "kascade_workspace_error",
-           "kascade_status_str")
+           "kascade_status_str", "kascade_select_decode_static", "kascade_select_decode_static_max_bytes")
 
 
 class KascadeError(RuntimeError):
@@ -78,6 +78,10 @@ def _load():
     so.kascade_dense_ref.restype = ctypes.c_int
     so.kascade_workspace_error.argtypes = [P, ctypes.POINTER(ctypes.c_int), ctypes.c_int, P]
     so.kascade_workspace_error.restype = ctypes.c_int
+    so.kascade_select_decode_static.argtypes = [SP, P, P, P, P]
+    so.kascade_select_decode_static.restype = ctypes.c_int
+    so.kascade_select_decode_static_max_bytes.argtypes = []
+    so.kascade_select_decode_static_max_bytes.restype = ctypes.c_size_t
     so.kascade_status_str.argtypes = [ctypes.c_int]
     so.kascade_status_str.restype = ctypes.c_char_p
     return so
@@ -167,6 +171,16 @@ def select(shape: Shape, q, k, idx=None, ws=None, stream=None):
     p, n = _ws(ws, shape, OP_SELECT)
     _check(lib.kascade_select(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(idx), p, n, _stream(stream)),
            "kascade_select")
+    return idx
+
+
+def select_decode_static(shape: Shape, q, k, idx=None, stream=None):
+    """kascade_select_decode_static: decode anchor selection with the library's
+    fixed scratch array instead of a workspace (nothing is allocated)."""
+    if idx is None:
+        idx = torch.empty(index_count(shape), dtype=torch.int32, device=q.device)
+    _check(lib.kascade_select_decode_static(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(idx), _stream(stream)),
+           "kascade_select_decode_static")
     return idx
 
 
