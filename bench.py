@@ -385,7 +385,7 @@ def run_kascade(args, rank, world, local):
     attn_us_per_launch = attn_ms * 1e3 / n_dec
     n_anchor = len(dcfg.anchors)
     attn_gbs = reuse_bytes / (attn_us_per_launch * 1e-6) / 1e9
-    traffic = profiled_traffic("decode_attn_llama8b_n32k.md", "sparse_attn.cu")
+    traffic = profiled_traffic("decode_attn_llama8b_n32k.md", "decode_attn.cu")
     roofline = {"bound": "hbm", "kernel": "decode_attn_kernel (sparse decode, row a6)",
                 "achieved": attn_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": attn_gbs / pk["hbm_gbs"],
                 "traffic": traffic, "peak_source": pk["source"] + " hbm_gbs (burst copy)",
