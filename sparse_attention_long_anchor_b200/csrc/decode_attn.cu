@@ -4,22 +4,32 @@
 // list the same kernel is the dense decode reference.
 //
 // One thread-block cluster per (batch, kv head); the index list is split
-// evenly over the CTAs of the cluster and every warp owns 16-key slices of
-// its CTA's share.  All warps gather at once:
-//   * K rows go straight from global memory into the registers of the
-//     16x8x16 bf16 MMA (the contraction runs over d, so each lane may take
-//     any permutation of d as long as q uses the same: lane (g, c) loads
-//     dims [32s + 8c, +8) of key g, one 16-byte load per 32 dims);
-//   * V rows go through a two-slot cp.async ring per warp (16-byte copies
-//     into rows padded by 16 bytes, conflict-free for ldmatrix.trans);
-//   * the G query rows sit in shared memory and are read with 8-byte loads
-//     in the same permuted order.
-// S = Q K^T (query heads as the MMA rows), fp32 online softmax, O += P V.
-// The partial (max, sum, output) of each CTA is pushed over distributed
-// shared memory to the CTA that owns each output element; after one cluster
-// barrier every CTA merges its slice locally.  No global scratch, no
-// spin-waits.
+// evenly over the CTAs of the cluster and every warp owns the 16-key slices
+// s = warp, warp + 8, ... of its CTA's share.  Each warp keeps its first two
+// slices in flight from the start:
+//   * K rows of its even slices go straight from global memory into the
+//     registers of the 16x8x16 bf16 MMA (the contraction runs over d, so each
+//     lane may take any permutation of d as long as q uses the same: lane
+//     (g, c) loads dims [32s + 8c, +8) of key g, one 16-byte load per 32
+//     dims); K rows of its odd slices go through a shared-memory slot and are
+//     read back in the same permuted order;
+//   * V rows go through a two-slot cp.async ring (16-byte chunks XOR-swizzled
+//     by row, conflict-free for ldmatrix.trans);
+//   * the G query rows sit in shared memory, read with 8-byte loads.
+// With programmatic dependent launch and inputs the caller vouches for, all
+// of that is issued before the kernel waits for its predecessor, so for the
+// usual list lengths every byte a CTA needs lands while the previous layer
+// is still running.
+// S^T = K Q^T and O^T += V^T P^T with the keys, then the head dims, as the
+// MMA rows and the query heads of the group as its columns; fp32 online
+// softmax per head.
+// The partial (max, sum, output) of each CTA is pushed with st.async into
+// the shared memory of the CTA that owns each output element, completing on
+// the owner's mbarrier; every CTA waits only for its own bytes and merges its
+// slice.  No global scratch; the one wait is bounded.
 #include <cooperative_groups.h>
+
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -33,74 +43,125 @@ namespace {
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kMaxCS = 16;
-constexpr int kIdxStage = 2048;   // index entries staged in shared memory
+constexpr int kIdxStage = 512;      // index entries staged in shared memory
+constexpr int kErrMergeTimeout = 3; // device error word: a merge wait gave up
 
 template <int D>
 struct Lay {
-  static constexpr int ROW = D * 2 + 16;                  // padded V row bytes
-  static constexpr int SLOT = 16 * ROW;                   // one 16-key V slab
-  static constexpr size_t vslots = 0;                     // [W][2] slots
-  static constexpr size_t qs = vslots + (size_t)kWarps * 2 * SLOT;   // [8][D] bf16 query rows
+  static constexpr int ROWB = D * 2;                       // K / V row bytes (chunks swizzled)
+  static constexpr int SLAB = 16 * ROWB;                   // one 16-key slab
+  static constexpr int WARPB = 3 * SLAB;                   // V slot 0, V slot 1, K slot
+  static constexpr size_t slabs = 0;
+  static constexpr size_t qs = slabs + (size_t)kWarps * WARPB;   // [8][D] bf16 query rows
   static constexpr size_t idx = qs + 8 * D * 2;
-  static constexpr size_t recv_o = idx + kIdxStage * 4;   // [G*D] f32, peers write here
-  static constexpr size_t recv_ml = recv_o + 8 * D * 4;   // [16][8][2]
-  static constexpr size_t total = recv_ml + kMaxCS * 8 * 2 * 4;
-  // after the gather loop, inside the V slots
-  static constexpr int RO = D + 8;                        // padded red_o row (floats)
-  static constexpr size_t red_o = 0;                      // [W][8][RO]
-  static constexpr size_t red_ml = red_o + (size_t)kWarps * 8 * RO * 4;
-  static constexpr size_t wf = red_ml + kWarps * 8 * 2 * 4;
-  static constexpr size_t pml = wf + kWarps * 8 * 4;
-  static constexpr size_t wts = pml + 8 * 2 * 4;
-  static constexpr size_t head = wts + kMaxCS * 8 * 4;
-  static_assert(head + 64 <= qs, "post-loop scratch must fit in the V slots");
+  static constexpr size_t recv_o = idx + kIdxStage * 4;    // [G*D] f32, written by the peers
+  static constexpr size_t recv_ml = recv_o + 8 * D * 4;    // [16][8] (m, l)
+  static constexpr size_t bar = recv_ml + kMaxCS * 8 * 8;  // mbarrier of the incoming partials
+  static constexpr size_t total = bar + 16;
+  // after the gather loop, inside the slabs
+  static constexpr int RO = D + 4;                         // padded red_o row (floats)
+  static constexpr size_t red_o = 0;                       // [W][8][RO]
+  static constexpr size_t red_ml = red_o + (size_t)kWarps * 8 * RO * 4;   // [W][8] (m, l)
+  static constexpr size_t wf = red_ml + kWarps * 8 * 8;    // [W][8] weight of each warp's partial
+  static constexpr size_t pml = wf + kWarps * 8 * 4;       // [8] (m, l) of this CTA
+  static constexpr size_t wts = pml + 8 * 8;               // [16][8] weight of each CTA's partial
+  static constexpr size_t head = wts + kMaxCS * 8 * 4;     // [8] (m, l) of the whole list
+  static_assert(head + 8 * 8 <= qs, "post-loop scratch must fit in the slabs");
+  static_assert(recv_o % 16 == 0 && recv_ml % 8 == 0 && bar % 8 == 0, "alignment");
 };
 
 __device__ __forceinline__ float scale_from(float m_old, float m_new) {
   return m_old == -INFINITY ? 0.0f : exp2f(m_old - m_new);
 }
 
-// Softmax-merge weights of n_slots partial results per head: for every
-// (slot, head) the factor exp2(m - M) against the head's max M, and per head
-// (M, sum of factor * l).  Called by one whole warp.  ml and w are laid out
-// [slot][8][2] and [slot][8]; out is [8][2].
-__device__ void merge_weights(int n_slots, int G, const float* ml, float* w, float* out, int lane) {
-  if (32 % G == 0) {
-    const int gg = lane % G;   // every pair a lane visits belongs to this head
-    float M = -INFINITY;
-    for (int i = lane; i < n_slots * G; i += 32) M = fmaxf(M, ml[((i / G) * 8 + gg) * 2]);
-    for (int o = G; o < 32; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float ls = 0.f;
-    for (int i = lane; i < n_slots * G; i += 32) {
-      const int sl = i / G;
-      const float f = scale_from(ml[(sl * 8 + gg) * 2], M);
-      w[sl * 8 + gg] = f;
-      ls += f * ml[(sl * 8 + gg) * 2 + 1];
-    }
-    for (int o = G; o < 32; o <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
-    if (lane < G) {
-      out[gg * 2] = M;
-      out[gg * 2 + 1] = ls;
-    }
-  } else if (lane < G) {
-    const int gg = lane;
-    float M = -INFINITY;
-    for (int sl = 0; sl < n_slots; ++sl) M = fmaxf(M, ml[(sl * 8 + gg) * 2]);
-    float ls = 0.f;
-    for (int sl = 0; sl < n_slots; ++sl) {
-      const float f = scale_from(ml[(sl * 8 + gg) * 2], M);
-      w[sl * 8 + gg] = f;
-      ls += f * ml[(sl * 8 + gg) * 2 + 1];
-    }
-    out[gg * 2] = M;
-    out[gg * 2 + 1] = ls;
-  }
+// Softmax-merge weights of n <= 32 partial results (m, l) of one head,
+// strided by 8 entries: lane i < n takes exp2(m_i - M) against the max M and
+// writes it to w[8 i]; lane 0 writes (M, sum of w_i l_i).  Whole warp.
+__device__ __forceinline__ void merge_weights(int n, const float2* ml, float* w, float2* out, int lane) {
+  const float2 v = lane < n ? ml[lane * 8] : make_float2(-INFINITY, 0.f);
+  float M = v.x;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  const float f = scale_from(v.x, M);
+  float ls = f * v.y;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+  if (lane < n) w[lane * 8] = f;
+  if (lane == 0) *out = make_float2(M, ls);
 }
 
-template <int D>
+// 8x8 b16 transpose across the warp: lane (g, c) passes row g, columns
+// 2c and 2c+1, and receives row 2c and 2c+1 of column g
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t r;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(r) : "r"(x));
+  return r;
+}
+
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+  uint4 r;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];\n"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "r"(addr));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t mapa(uint32_t addr, int rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+// asynchronous store into another CTA's shared memory, completing on that
+// CTA's mbarrier (both addresses in the shared::cluster window)
+__device__ __forceinline__ void st_async_v4(uint32_t raddr, float4 v, uint32_t rbar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];\n" ::"r"(raddr),
+      "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(rbar)
+      : "memory");
+}
+__device__ __forceinline__ void st_async_v2(uint32_t raddr, float2 v, uint32_t rbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];\n" ::"r"(raddr),
+               "f"(v.x), "f"(v.y), "r"(rbar)
+               : "memory");
+}
+
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// bounded wait (about 2^32 SM clocks) for data other CTAs of the cluster
+// stored into this CTA
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait_cluster(bar, parity)) {
+    if (clock64() - t0 > (1ll << 32)) return false;
+  }
+  return true;
+}
+
+// kRing = false: every warp owns at most two slices (per <= 16 * 2 * kWarps),
+// all issued up front; kRing = true: the slabs are refilled two slices ahead.
+template <int D, bool kRing>
 __global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const AttnArgs a, int per) {
   using L = Lay<D>;
   constexpr int KS = D / 32;          // 16-byte K loads per key row per lane
+  constexpr int CH = D / 8;           // 16-byte chunks per row
   extern __shared__ __align__(128) char smem[];
   // with PDL the gathers may start before the previous kernel completes only
   // if the caller vouched for k, v, idx and head_map; otherwise wait first
@@ -117,6 +178,18 @@ __global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const AttnArgs
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, c = lane & 3;
   const int G = a.G;
+  const int E = G * D;
+  const int en = E / CS;              // output elements owned by each CTA (a multiple of 4)
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar = sbase + (uint32_t)L::bar;
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    mbar_fence_init();
+    // every CTA of the cluster sends en outputs and G (m, l) pairs
+    mbar_arrive_expect_tx(bar, (uint32_t)(E * 4 + CS * G * 8));
+  }
+  cluster_arrive_release();   // the matching wait comes before the first push
+
   // an out-of-range head_map entry reads as an empty list (output 0, lse -inf)
   const int hm_raw = a.head_map ? a.head_map[h] : h;
   const bool hm_ok = hm_raw >= 0 && hm_raw < a.Hkv;
@@ -139,20 +212,22 @@ __global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const AttnArgs
   auto key_of = [&](int rel) -> int {
     return list ? (staged ? idx_s[rel] : __ldg(list + c0 + rel)) : c0 + rel;
   };
-  // V rows of slice s into this warp's slot (s / W) & 1; missing rows zero-filled
-  const uint32_t vbase = smem_u32(smem) + (uint32_t)(warp * 2 * L::SLOT);
-  auto issue_v = [&](int s) {
-    const uint32_t dst = vbase + ((s / kWarps) & 1) * L::SLOT;
+  const uint32_t wbase = sbase + (uint32_t)(L::slabs + warp * L::WARPB);
+  const uint32_t kslot = wbase + 2 * L::SLAB;
+  // 16 rows of slice s (K or V) into a slab; rows past the list zero-filled.
+  // V chunks are swizzled by row & 7 (ldmatrix.trans), K chunks by
+  // (row & 1) * 4 (the permuted 16-byte reads of two rows per quarter warp).
+  auto issue_rows = [&](int s, uint32_t dst, const __nv_bfloat16* base, bool is_k) {
 #pragma unroll
-    for (int i = 0; i < D / 16; ++i) {   // 16 rows x D/8 chunks over 32 lanes
+    for (int i = 0; i < D / 16; ++i) {   // 16 rows x CH chunks over 32 lanes
       const int e = lane + 32 * i;
-      const int r = e / (D / 8), ch = e - r * (D / 8);
+      const int r = e / CH, ch = e - r * CH;
       const int rel = s * 16 + r;
       const bool have = c0 + rel < c1;
       const int key = have ? key_of(rel) : 0;
-      cp_async_16(dst + r * L::ROW + ch * 16, vb + (size_t)key * D + ch * 8, have ? 16 : 0);
+      const int pch = is_k ? (ch ^ ((r & 1) << 2)) : (ch ^ (r & 7));
+      cp_async_16(dst + r * L::ROWB + pch * 16, base + (size_t)key * D + ch * 8, have ? 16 : 0);
     }
-    cp_async_commit();
   };
   // K rows g and 8+g of slice s into registers (zero past the list end)
   uint4 kr[2][KS];
@@ -167,147 +242,212 @@ __global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const AttnArgs
     }
   };
 
-  float m_run = -INFINITY, l_run = 0.f;
-  float oacc[D / 8][2];
+  // per lane: heads 2c and 2c+1 (running max in log2 units, partial sums
+  // over this lane's keys) and O^T for dims 16i + g (+8) of those heads
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+  float oacc[D / 16][4];
 #pragma unroll
-  for (int nd = 0; nd < D / 8; ++nd) oacc[nd][0] = oacc[nd][1] = 0.f;
+  for (int i = 0; i < D / 16; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
   const float scale2 = kLog2e * rsqrtf((float)D);
   const char* qrow = smem + L::qs + (size_t)(g * D + 8 * c) * 2;
 
-  // prologue: V of this warp's first two slices, K of its first slice
-  int s = warp;
-  if (s < n_slices) issue_v(s);
-  if (s + kWarps < n_slices) issue_v(s + kWarps);
-  if (s < n_slices) load_k(s);
+  // prologue: this warp's first two slices (one cp.async group each)
+  if (warp < n_slices) issue_rows(warp, wbase, vb, false);
+  if constexpr (kRing) cp_async_commit();
+  if (warp + kWarps < n_slices) {
+    issue_rows(warp + kWarps, wbase + L::SLAB, vb, false);
+    issue_rows(warp + kWarps, kslot, kb, true);
+  }
+  cp_async_commit();
+  if (warp < n_slices) load_k(warp);
   if (early) {
     pdl_wait();
     pdl_launch_dependents();
   }
   // the G query rows of this kv head (rows G..7 zero)
-  for (int i = threadIdx.x; i < 8 * (D / 8); i += kThreads) {
-    const int r = i / (D / 8), ch = i - r * (D / 8);
+  for (int i = threadIdx.x; i < 8 * CH; i += kThreads) {
+    const int r = i / CH, ch = i - r * CH;
     uint4 val = make_uint4(0, 0, 0, 0);
     if (r < G) val = *reinterpret_cast<const uint4*>(a.q + (size_t)(b * a.Hq + h * G + r) * D + ch * 8);
     *reinterpret_cast<uint4*>(smem + L::qs + (r * D + ch * 8) * 2) = val;
   }
   __syncthreads();
-  for (; s < n_slices; s += kWarps) {
-    // S = Q K^T: k-step 2q+hf takes dims 32q + 8c + 4hf + {0,1} (a0/b0) and
-    // + {2,3} (a2/b1) of the query rows and key rows
-    float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+
+  // One slice, both products transposed so that the 16 keys (and then the
+  // head dims) fill the MMA rows and the <= 8 query heads its columns:
+  // S^T = K q^T (A = K rows, B = q^T), then O^T += V^T P^T (A = V^T by
+  // ldmatrix.trans, B = P^T moved from accumulator to operand layout by
+  // movmatrix).  K fragments come from registers (even iterations) or the
+  // K slot (odd iterations).
+  auto step = [&](int s, int slot, auto from_slot) {
+    constexpr bool kSlot = decltype(from_slot)::value;
+    // k-step 2q+t takes dims 32q + 8c + 4t + {0,1} (logical k 2c, 2c+1) and
+    // + {2,3} (logical k 2c+8, 2c+9) of the key rows and the query rows
+    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int q = 0; q < KS; ++q) {
       const uint2 qlo = *reinterpret_cast<const uint2*>(qrow + 64 * q);       // dims 32q+8c+0..3
       const uint2 qhi = *reinterpret_cast<const uint2*>(qrow + 64 * q + 8);   // dims 32q+8c+4..7
-      const uint32_t a0[4] = {qlo.x, 0u, qlo.y, 0u};
-      const uint32_t a1[4] = {qhi.x, 0u, qhi.y, 0u};
-      mma_bf16_16816(s0, a0, kr[0][q].x, kr[0][q].y);
-      mma_bf16_16816(s1, a0, kr[1][q].x, kr[1][q].y);
-      mma_bf16_16816(s0, a1, kr[0][q].z, kr[0][q].w);
-      mma_bf16_16816(s1, a1, kr[1][q].z, kr[1][q].w);
+      uint4 k0, k1;
+      if constexpr (kSlot) {
+        const int pch = (4 * q + c) ^ ((g & 1) << 2);   // rows g and 8 + g share parity
+        k0 = lds_v4(kslot + g * L::ROWB + pch * 16);
+        k1 = lds_v4(kslot + (8 + g) * L::ROWB + pch * 16);
+      } else {
+        k0 = kr[0][q];
+        k1 = kr[1][q];
+      }
+      const uint32_t a0[4] = {k0.x, k1.x, k0.y, k1.y};
+      const uint32_t a1[4] = {k0.z, k1.z, k0.w, k1.w};
+      mma_bf16_16816(q & 1 ? sb : sa, a0, qlo.x, qlo.y);
+      mma_bf16_16816(q & 1 ? sb : sa, a1, qhi.x, qhi.y);
     }
+    // sv: (key g, head 2c), (key g, head 2c+1), (key g+8, head 2c), (key g+8, head 2c+1)
     const int kbase = c0 + s * 16;
+    const bool v_lo = kbase + g < c1, v_hi = kbase + 8 + g < c1;
     float sv[4];
-    sv[0] = kbase + 2 * c < c1 ? s0[0] * scale2 : -INFINITY;
-    sv[1] = kbase + 2 * c + 1 < c1 ? s0[1] * scale2 : -INFINITY;
-    sv[2] = kbase + 8 + 2 * c < c1 ? s1[0] * scale2 : -INFINITY;
-    sv[3] = kbase + 9 + 2 * c < c1 ? s1[1] * scale2 : -INFINITY;
-    float mx = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    const float m_new = fmaxf(m_run, mx);
-    const float alpha = scale_from(m_run, m_new);
-    float p[4];
+    sv[0] = v_lo ? (sa[0] + sb[0]) * scale2 : -INFINITY;
+    sv[1] = v_lo ? (sa[1] + sb[1]) * scale2 : -INFINITY;
+    sv[2] = v_hi ? (sa[2] + sb[2]) * scale2 : -INFINITY;
+    sv[3] = v_hi ? (sa[3] + sb[3]) * scale2 : -INFINITY;
+    float mx0 = fmaxf(sv[0], sv[2]), mx1 = fmaxf(sv[1], sv[3]);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) p[e] = exp2f(sv[e] - m_new);
-    l_run = l_run * alpha + (p[0] + p[1] + p[2] + p[3]);
-    m_run = m_new;
-    const uint32_t pa[4] = {pack_bf16(p[0], p[1]), 0u, pack_bf16(p[2], p[3]), 0u};
-    // V of this slice: its copy group is the oldest one still pending
-    if (s + kWarps < n_slices) cp_async_wait<1>(); else cp_async_wait<0>();
-    __syncwarp();
-    const uint32_t vs = vbase + ((s / kWarps) & 1) * L::SLOT;
-#pragma unroll
-    for (int nd = 0; nd < D / 8; nd += 2) {
-      uint32_t r4[4];
-      const int mi = lane >> 3;
-      ldmatrix_x4_trans(r4, vs + ((mi & 1) * 8 + (lane & 7)) * L::ROW + (nd + (mi >> 1)) * 16);
-      float t0[4] = {oacc[nd][0] * alpha, oacc[nd][1] * alpha, 0.f, 0.f};
-      float t1[4] = {oacc[nd + 1][0] * alpha, oacc[nd + 1][1] * alpha, 0.f, 0.f};
-      mma_bf16_16816(t0, pa, r4[0], r4[1]);
-      mma_bf16_16816(t1, pa, r4[2], r4[3]);
-      oacc[nd][0] = t0[0];
-      oacc[nd][1] = t0[1];
-      oacc[nd + 1][0] = t1[0];
-      oacc[nd + 1][1] = t1[1];
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
     }
+    // key s*16 is always in the list, so the slice maxima are finite
+    const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+    const float al0 = scale_from(m_run[0], mn0), al1 = scale_from(m_run[1], mn1);
+    const float p0 = exp2f(sv[0] - mn0), p1 = exp2f(sv[1] - mn1);
+    const float p2 = exp2f(sv[2] - mn0), p3 = exp2f(sv[3] - mn1);
+    l_run[0] = l_run[0] * al0 + (p0 + p2);
+    l_run[1] = l_run[1] * al1 + (p1 + p3);
+    m_run[0] = mn0;
+    m_run[1] = mn1;
+    // P^T rows (keys) x columns (heads) -> B fragments (k = keys, n = heads)
+    const uint32_t b0 = movmatrix_trans(pack_bf16(p0, p1));   // keys 0..7
+    const uint32_t b1 = movmatrix_trans(pack_bf16(p2, p3));   // keys 8..15
+    const uint32_t vs = wbase + slot * L::SLAB;
+    const int vrow = ((lane >> 4) << 3) + (lane & 7);         // key of this lane's ldmatrix row
+    const int vch = (lane >> 3) & 1;                           // dims +0 / +8 of the tile
+#pragma unroll
+    for (int i = 0; i < D / 16; ++i) {
+      uint32_t r4[4];
+      ldmatrix_x4_trans(r4, vs + vrow * L::ROWB + (((2 * i + vch) ^ (lane & 7)) * 16));
+      float t[4] = {oacc[i][0] * al0, oacc[i][1] * al1, oacc[i][2] * al0, oacc[i][3] * al1};
+      mma_bf16_16816(t, r4, b0, b1);
+      oacc[i][0] = t[0];
+      oacc[i][1] = t[1];
+      oacc[i][2] = t[2];
+      oacc[i][3] = t[3];
+    }
+  };
+
+  if constexpr (kRing) {
+    int it = 0;
+    for (int s = warp; s < n_slices; s += kWarps, ++it) {
+      cp_async_wait<1>();   // the group of slice `it`; one later group is always committed
+      __syncwarp();
+      const int slot = it & 1;
+      if (slot) step(s, 1, std::true_type{});
+      else step(s, 0, std::false_type{});
+      __syncwarp();
+      // refill what this slice used with the slice two iterations ahead
+      const int s2 = s + 2 * kWarps;
+      if (s2 < n_slices) {
+        issue_rows(s2, wbase + slot * L::SLAB, vb, false);
+        if (slot) issue_rows(s2, kslot, kb, true);
+      }
+      cp_async_commit();
+      if (!slot && s2 < n_slices) load_k(s2);
+    }
+  } else {
+    cp_async_wait<0>();
     __syncwarp();
-    if (s + 2 * kWarps < n_slices) issue_v(s + 2 * kWarps);   // refill the slot just read
-    if (s + kWarps < n_slices) load_k(s + kWarps);
+    if (warp < n_slices) step(warp, 0, std::false_type{});
+    if (warp + kWarps < n_slices) step(warp + kWarps, 1, std::true_type{});
   }
   cp_async_wait<0>();
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], o);
+    l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], o);
+  }
 
   // ---------------- merge the warps into this CTA's partial
-  __syncthreads();
+  __syncthreads();   // every warp is done with its slabs
   float* red_o = reinterpret_cast<float*>(smem + L::red_o);
-  float* red_ml = reinterpret_cast<float*>(smem + L::red_ml);
-  if (g < G) {
+  float2* red_ml = reinterpret_cast<float2*>(smem + L::red_ml);
 #pragma unroll
-    for (int nd = 0; nd < D / 8; ++nd)
-      *reinterpret_cast<float2*>(red_o + (warp * 8 + g) * L::RO + nd * 8 + 2 * c) =
-          make_float2(oacc[nd][0], oacc[nd][1]);
-    if (c == 0) {
-      red_ml[(warp * 8 + g) * 2] = m_run;
-      red_ml[(warp * 8 + g) * 2 + 1] = l_run;
+  for (int j = 0; j < 2; ++j) {
+    const int hh = 2 * c + j;
+    if (hh < G) {
+      float* ro = red_o + (warp * 8 + hh) * L::RO + g;
+#pragma unroll
+      for (int i = 0; i < D / 16; ++i) {
+        ro[16 * i] = oacc[i][j];
+        ro[16 * i + 8] = oacc[i][2 + j];
+      }
+      if (g == 0) red_ml[warp * 8 + hh] = make_float2(m_run[j], l_run[j]);
     }
   }
   __syncthreads();
-  // per-head weights of the warps
+  // softmax-merge weights of the warps' partials, one warp per head
   float* wf = reinterpret_cast<float*>(smem + L::wf);
-  float* pml = reinterpret_cast<float*>(smem + L::pml);
-  if (warp == 0) merge_weights(kWarps, G, red_ml, wf, pml, lane);
+  float2* pml = reinterpret_cast<float2*>(smem + L::pml);
+  if (warp < G) merge_weights(kWarps, red_ml + warp, wf + warp, pml + warp, lane);
   __syncthreads();
-  // push element e to CTA e / en (E is a multiple of the cluster size)
-  float* recv_o = reinterpret_cast<float*>(smem + L::recv_o);
-  float* recv_ml = reinterpret_cast<float*>(smem + L::recv_ml);
-  const int E = G * D;
-  const int en = E / CS;
-  for (int e = threadIdx.x; e < E; e += kThreads) {
+  cluster_wait_acquire();   // every peer's mbarrier is initialised
+  const uint32_t recv_o = sbase + (uint32_t)L::recv_o;
+  const uint32_t recv_ml = sbase + (uint32_t)L::recv_ml;
+  // four consecutive output elements per thread, pushed to their owner e / en
+  if (threadIdx.x * 4 < E) {
+    const int e = threadIdx.x * 4;
+    const int gg = e / D, dd = e - gg * D;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const float f = wf[w * 8 + gg];
+      const float4 v = *reinterpret_cast<const float4*>(red_o + (w * 8 + gg) * L::RO + dd);
+      acc.x += f * v.x;
+      acc.y += f * v.y;
+      acc.z += f * v.z;
+      acc.w += f * v.w;
+    }
+    const int q = e / en;
+    const uint32_t off = (uint32_t)(rank * en + (e - q * en)) * 4;
+    st_async_v4(mapa(recv_o + off, q), acc, mapa(bar, q));
+  }
+  // this CTA's (max, sum) of every head, to every CTA of the cluster
+  if (threadIdx.x < CS * G) {
+    const int r = threadIdx.x / G, gg = threadIdx.x - r * G;
+    st_async_v2(mapa(recv_ml + (uint32_t)(rank * 8 + gg) * 8, r), pml[gg], mapa(bar, r));
+  }
+
+  // ---------------- merge this CTA's element slice once every peer's bytes landed
+  if (!mbar_wait_cluster_bounded(bar, 0)) raise_error(a.err, kErrMergeTimeout);
+  float* wts = reinterpret_cast<float*>(smem + L::wts);
+  float2* head = reinterpret_cast<float2*>(smem + L::head);
+  const float2* rml = reinterpret_cast<const float2*>(smem + L::recv_ml);
+  if (warp < G) merge_weights(CS, rml + warp, wts + warp, head + warp, lane);
+  __syncthreads();
+  if ((int)threadIdx.x < en) {
+    const float* ro = reinterpret_cast<const float*>(smem + L::recv_o);
+    const int e = rank * en + threadIdx.x;
     const int gg = e / D, dd = e - gg * D;
     float acc = 0.f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) acc += wf[w * 8 + gg] * red_o[(w * 8 + gg) * L::RO + dd];
-    const int q = e / en;
-    *cluster.map_shared_rank(recv_o + rank * en + (e - q * en), q) = acc;
-  }
-  if (threadIdx.x < CS * G) {
-    const int r = threadIdx.x / G, gg = threadIdx.x - r * G;
-    float* ml = cluster.map_shared_rank(recv_ml, r);
-    ml[(rank * 8 + gg) * 2] = pml[gg * 2];
-    ml[(rank * 8 + gg) * 2 + 1] = pml[gg * 2 + 1];
-  }
-  cluster.sync();
-
-  // ---------------- merge this CTA's element slice from local shared memory
-  float* wts = reinterpret_cast<float*>(smem + L::wts);
-  float* head = reinterpret_cast<float*>(smem + L::head);
-  if (warp == 0) merge_weights(CS, G, recv_ml, wts, head, lane);
-  __syncthreads();
-  const int e0 = rank * en, e1 = e0 + en;
-  for (int e = e0 + (int)threadIdx.x; e < e1; e += kThreads) {
-    const int gg = e / D, dd = e - gg * D;
-    float acc = 0.f;
-    for (int r = 0; r < CS; ++r) acc += wts[r * 8 + gg] * recv_o[r * en + (e - e0)];
-    const float Ls = head[gg * 2 + 1];
+    for (int r = 0; r < kMaxCS; ++r)
+      if (r < CS) acc += wts[r * 8 + gg] * ro[r * en + threadIdx.x];
+    const float2 ml = head[gg];
     const size_t orow = (size_t)(b * a.Hq + h * G + gg);
-    a.o[orow * D + dd] = __float2bfloat16(Ls > 0.f ? acc / Ls : 0.f);
-    if (dd == 0 && a.lse) a.lse[orow] = Ls > 0.f ? (head[gg * 2] + log2f(Ls)) * (float)kLn2 : -INFINITY;
+    a.o[orow * D + dd] = __float2bfloat16(ml.y > 0.f ? acc / ml.y : 0.f);
+    if (dd == 0 && a.lse) a.lse[orow] = ml.y > 0.f ? (ml.x + log2f(ml.y)) * (float)kLn2 : -INFINITY;
   }
 }
 
-template <int D>
+template <int D, bool kRing>
 cudaLaunchConfig_t make_cfg(int cs, int bh, cudaStream_t stream, cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cs, bh, 1);
@@ -324,44 +464,52 @@ cudaLaunchConfig_t make_cfg(int cs, int bh, cudaStream_t stream, cudaLaunchAttri
 }
 
 // 16-CTA clusters when the device can co-schedule them, else 8
-template <int D>
+template <int D, bool kRing>
 int cluster_size_for_device() {
   static int cached[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 8;
   if (cached[dev]) return cached[dev];
   int cs = 8;
-  if (cudaFuncSetAttribute(decode_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(decode_attn_kernel<D, kRing>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)Lay<D>::total) == cudaSuccess &&
-      cudaFuncSetAttribute(decode_attn_kernel<D>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+      cudaFuncSetAttribute(decode_attn_kernel<D, kRing>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
           cudaSuccess) {
     cudaLaunchAttribute attr[1];
-    cudaLaunchConfig_t cfg = make_cfg<D>(kMaxCS, 1, nullptr, attr);
+    cudaLaunchConfig_t cfg = make_cfg<D, kRing>(kMaxCS, 1, nullptr, attr);
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, decode_attn_kernel<D>, &cfg) == cudaSuccess && n > 0) cs = kMaxCS;
+    if (cudaOccupancyMaxActiveClusters(&n, decode_attn_kernel<D, kRing>, &cfg) == cudaSuccess && n > 0)
+      cs = kMaxCS;
   }
   cudaGetLastError();
   cached[dev] = cs;
   return cs;
 }
 
+template <int D, bool kRing>
+cudaError_t launch_cs(const AttnArgs& a, int cs, int per, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<D, kRing>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)Lay<D>::total);
+  if (e != cudaSuccess) return e;
+  if (cs > 8) {
+    e = cudaFuncSetAttribute(decode_attn_kernel<D, kRing>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_ex(decode_attn_kernel<D, kRing>, dim3(cs, a.B * a.Hkv), dim3(kThreads), Lay<D>::total, stream,
+                   (a.flags & 1) != 0, cs, a, per);
+}
+
 template <int D>
 cudaError_t launch(const AttnArgs& a, cudaStream_t stream) {
-  const int cs = cluster_size_for_device<D>();
+  // both variants share the shared-memory size and cluster shape, so one
+  // occupancy answer serves both
+  const int cs = cluster_size_for_device<D, false>();
   const int list_len = a.idx ? topk_count(a.N, a.num, a.den) : a.N;
   int per = (list_len + cs - 1) / cs;
   per = (per + 15) / 16 * 16;
   if (per < 16) per = 16;
   if ((a.G * D) % cs != 0) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)Lay<D>::total);
-  if (e != cudaSuccess) return e;
-  if (cs > 8) {
-    e = cudaFuncSetAttribute(decode_attn_kernel<D>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-  }
-  return launch_ex(decode_attn_kernel<D>, dim3(cs, a.B * a.Hkv), dim3(kThreads), Lay<D>::total, stream,
-                   (a.flags & 1) != 0, cs, a, per);
+  return per <= 2 * 16 * kWarps ? launch_cs<D, false>(a, cs, per, stream) : launch_cs<D, true>(a, cs, per, stream);
 }
 
 }  // namespace
