@@ -123,6 +123,12 @@ int device_sms() {
   return n;
 }
 
+// sparse / dense prefill: the tcgen05 kernel where it applies, else the
+// warp-MMA kernel
+cudaError_t launch_prefill(const AttnArgs& a, cudaStream_t st) {
+  return prefill_attn_tc_supported(a) ? launch_prefill_attn_tc(a, device_sms(), st) : launch_prefill_attn(a, st);
+}
+
 int* err_word(void* ws, size_t ws_bytes) {
   return (ws && ws_bytes >= sizeof(int) && aligned(ws, 4)) ? static_cast<int*>(ws) : nullptr;
 }
@@ -322,7 +328,7 @@ int kascade_sparse_prefill(const kascade_shape* s, const void* q, const void* k,
     return KASCADE_ERR_UNSUPPORTED;
   AttnArgs a = attn_args(s, q, k, v, idx, head_map, o, lse);
   a.err = err_word(ws, ws_bytes);
-  return cuda_status(launch_prefill_attn(a, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_prefill(a, static_cast<cudaStream_t>(stream)));
 }
 
 int kascade_dense_ref(const kascade_shape* s, const void* q, const void* k, const void* v, int causal,
@@ -338,7 +344,7 @@ int kascade_dense_ref(const kascade_shape* s, const void* q, const void* k, cons
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (is_decode(s)) return cuda_status(launch_decode_attn(a, st));
   a.causal = causal != 0;
-  return cuda_status(launch_prefill_attn(a, st));
+  return cuda_status(launch_prefill(a, st));
 }
 
 int kascade_workspace_error(const void* ws, int* error_out, int clear, void* stream) {

@@ -84,5 +84,8 @@ struct AttnArgs {
 // decode: one 16-CTA cluster per (batch, kv head), merge over DSMEM
 cudaError_t launch_decode_attn(const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill_attn(const AttnArgs& a, cudaStream_t stream);
+// prefill on tcgen05 (G <= 4 or a multiple of 4, d in {64, 128}, tile 32)
+bool prefill_attn_tc_supported(const AttnArgs& a);
+cudaError_t launch_prefill_attn_tc(const AttnArgs& a, int num_sms, cudaStream_t stream);
 
 }  // namespace kascade
