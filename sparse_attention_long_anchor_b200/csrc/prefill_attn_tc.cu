@@ -10,21 +10,25 @@
 // Work item = (query tile, row block, batch x kv head): 128 MMA rows = 4
 // query heads x 32 queries (rows of absent heads are zero and never stored).
 // Persistent CTAs take items head by head, longest tile first.  Per CTA:
-//   warps 0..3  softmax: one TMEM lane (= one query row) per thread; reads S
+//   warps 0..7  softmax, two warpgroups splitting the columns: one TMEM
+//               lane (= one query row) per thread of each group; reads S
 //               with tcgen05.ld, applies the causal mask by original key
 //               index, keeps the running max and sum, writes P (bf16) into
-//               shared memory as the A operand of the second product, and
+//               TMEM as the A operand of the second product, and
 //               finally reads O, normalises and stores it.  The running max
 //               used for the exponent is raised (and O, l rescaled in TMEM)
 //               only when a row's max grows by more than 2^8, which keeps
 //               the result exact and P within bf16 range;
-//   warps 4..7  gather: 64 selected K and V rows per block, 16-byte
+//   warps 8..11 gather: 64 selected K and V rows per block, 16-byte
 //               cp.async into 128-byte-swizzled shared memory, a ring of
-//               kStages blocks; one thread also issues the TMA loads of the
-//               item's Q tile (double-buffered);
-//   warp 8      single-thread tcgen05.mma issue and TMEM owner:
+//               kStages blocks, completion tracked per thread on the stage's
+//               mbarrier; one thread also issues the TMA loads of the item's
+//               Q tile (double-buffered);
+//   warp 12     single-thread tcgen05.mma issue (whichever product is
+//               ready first) and TMEM owner:
 //               S = Q K^T (M = 128, N = 64, into one of two TMEM buffers),
-//               O += P V (M = 128, N = d, V as an MN-major operand, into
+//               O += P V (M = 128, N = d, P from TMEM, V as an MN-major
+//               shared-memory operand, into
 //               one of two TMEM output buffers, one per item in flight).
 // All hand-offs are mbarriers; every wait is bounded and a timeout stops the
 // CTA's waits and records an error code in the workspace error word.
@@ -37,11 +41,15 @@ namespace kascade {
 namespace {
 
 constexpr int kKB = 64;          // keys per block
-constexpr int kStages = 4;       // K/V ring; >= 3 keeps the MMA issue order deadlock-free
-constexpr int kThreads = 288;    // 4 softmax warps, 4 gather warps, 1 MMA warp
+constexpr int kStages = 5;       // K/V ring; >= 3 keeps the MMA issue order deadlock-free
+constexpr int kThreads = 416;    // 8 softmax warps, 4 gather warps, 1 MMA warp
+constexpr int kGather0 = 256;    // first gather thread
+constexpr int kMmaWarp = 12;
 constexpr int kErrTimeout = 4;
 constexpr float kRescale = 8.0f; // log2 growth of a row max that forces a rescale
 constexpr int kNoKey = 0x7fffffff;
+// TMEM columns: S[2] (kKB each), O[2] (128 each), P[2] (kKB / 2 each, bf16 pairs)
+constexpr uint32_t kColS = 0, kColO = 128, kColP = 384;
 
 template <int D>
 struct PAL {
@@ -49,18 +57,16 @@ struct PAL {
   static constexpr int QCB = 128 * 128;             // one 64-column block of the Q tile
   static constexpr int KB = kKB * D * 2;            // K (or V) of one block
   static constexpr int KVCB = kKB * 128;            // one 64-column block of K (or V)
-  static constexpr int PB = 128 * kKB * 2;          // P of one block
   static constexpr size_t q = 0;                     // [2] Q
   static constexpr size_t kv = q + 2 * (size_t)QB;   // [S] K then V
-  static constexpr size_t p = kv + (size_t)kStages * 2 * KB;   // [2] P
-  static constexpr size_t keys = p + 2 * (size_t)PB; // [S][64] key index per row (kNoKey past the list)
-  static constexpr size_t bars = keys + (size_t)kStages * kKB * 4;
+  static constexpr size_t bars = kv + (size_t)kStages * 2 * KB;
   static constexpr int NBARS = 4 + 2 * kStages + 12 + 1;
-  static constexpr size_t tslot = bars + NBARS * 8;
+  static constexpr size_t xch = bars + NBARS * 8;     // [2][128] f32 row maxima / sums of the two softmax groups
+  static constexpr size_t tslot = xch + 2 * 128 * 4;
   static constexpr size_t stop = tslot + 8;
   static constexpr size_t total = stop + 8;
   static constexpr size_t alloc = total + 1024;      // slack for 1024-byte alignment
-  static_assert(kv % 1024 == 0 && p % 1024 == 0 && KB % 1024 == 0 && PB % 1024 == 0, "swizzled tiles");
+  static_assert(kv % 1024 == 0 && KB % 1024 == 0, "swizzled tiles");
   static_assert(bars % 8 == 0, "mbarrier alignment");
   static_assert(alloc <= 232448, "more than 227 KB of shared memory per block");
 };
@@ -107,9 +113,6 @@ __device__ __forceinline__ Item item_of(const AttnArgs& a, int it, int T, int RB
 
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
-}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -120,8 +123,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   char* sm = smem_raw + (base - raw);
-  const uint32_t q_s = base + (uint32_t)L::q, kv_s = base + (uint32_t)L::kv, p_s = base + (uint32_t)L::p;
-  int* keys_s = reinterpret_cast<int*>(sm + L::keys);
+  const uint32_t q_s = base + (uint32_t)L::q, kv_s = base + (uint32_t)L::kv;
   const uint32_t bar0 = base + (uint32_t)L::bars;
   auto bar = [&](int slot) { return bar0 + 8u * (uint32_t)slot; };
   volatile int* stop = reinterpret_cast<volatile int*>(sm + L::stop);
@@ -138,11 +140,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(bQFull + i), 1);
       mbar_init(bar(bQEmpty + i), 1);
       mbar_init(bar(bSFull + i), 1);
-      mbar_init(bar(bSEmpty + i), 4);
-      mbar_init(bar(bPFull + i), 4);
+      mbar_init(bar(bSEmpty + i), 8);
+      mbar_init(bar(bPFull + i), 8);
       mbar_init(bar(bPEmpty + i), 1);
       mbar_init(bar(bODone + i), 1);
-      mbar_init(bar(bOEmpty + i), 4);
+      mbar_init(bar(bOEmpty + i), 8);
     }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bar(bKVFull + s), 128);
@@ -162,7 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         make_uint4(0, 0, 0, 0);
   }
   fence_async_smem();
-  if (warp == 8) tc::tmem_alloc(base + (uint32_t)L::tslot, 512);
+  if (warp == kMmaWarp) tc::tmem_alloc(base + (uint32_t)L::tslot, 512);
   pdl_wait();
   pdl_launch_dependents();
   tc::fence_before();
@@ -180,65 +182,86 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   };
 
-  if (warp >= 4 && warp < 8) {
+  if (warp >= 8 && warp < kMmaWarp) {
     // ------------------------------------------------------------ gather
     // thread -> 16-byte chunk c of rows r0, r0 + RPP, ...: one warp
-    // instruction copies whole 256-byte rows
-    constexpr int CH = D / 8, RPP = 128 / CH;
-    const int pt = threadIdx.x - 128;
+    // instruction copies whole 256-byte rows.  The key indices of the next
+    // block are loaded one block ahead, and every thread arrives on the
+    // stage's barrier asynchronously when its copies land, so the gather
+    // only ever waits for a free stage.
+    constexpr int CH = D / 8, RPP = 128 / CH, KR = kKB / RPP;
+    const int pt = threadIdx.x - kGather0;
     const int c = pt % CH, r0 = pt / CH;
     const int cb = c >> 3, cc = c & 7;
-    const __nv_bfloat16* kbase = a.k;
-    const __nv_bfloat16* vbase = a.v;
-    int n = 0, qn = 0, pend = -1;
+    auto load_keys = [&](const Item& I, int j, int (&kk)[KR]) {
+#pragma unroll
+      for (int u = 0; u < KR; ++u) {
+        const int pos = j * kKB + r0 + RPP * u;
+        kk[u] = pos < I.list_len ? (I.list ? __ldg(I.list + pos) : pos) : kNoKey;
+      }
+    };
+    int cur[KR], nxt[KR];
+    int pf_it = -1, pf_j = 0;   // block whose keys sit in cur
+    int n = 0, qn = 0;
+    if (blockIdx.x < items) {
+      const Item I0 = item_of(a, blockIdx.x, T, RB);
+      if (I0.nb > 0) {
+        load_keys(I0, 0, cur);
+        pf_it = blockIdx.x;
+      }
+    }
     for (int it = blockIdx.x; it < items; it += gridDim.x, ++qn) {
       const Item I = item_of(a, it, T, RB);
+      const int it2 = it + gridDim.x;
+      const Item I2 = item_of(a, it2 < items ? it2 : it, T, RB);
+      const bool have2 = it2 < items && I2.nb > 0;
       if (pt == 0) {
         const int qb = qn & 1;
         if (qn >= 2) wait(bQEmpty + qb, (qn >> 1) - 1);
         mbar_arrive_expect_tx(bar(bQFull + qb), (uint32_t)(CB * heads_rb * 32 * 128));
-        for (int cb = 0; cb < CB; ++cb)
+        for (int b = 0; b < CB; ++b)
           for (int g = 0; g < heads_rb; ++g)
-            tc::tma_load_3d(q_s + qb * L::QB + cb * L::QCB + g * 4096, &mq, cb * 64, I.i0,
+            tc::tma_load_3d(q_s + qb * L::QB + b * L::QCB + g * 4096, &mq, b * 64, I.i0,
                             I.b * a.Hq + I.hq0 + g, bar(bQFull + qb));
       }
       const size_t bhoff = (size_t)(I.b * a.Hkv + I.h) * a.N * D;
       for (int j = 0; j < I.nb; ++j, ++n) {
+        if (pf_it != it || pf_j != j) load_keys(I, j, cur);   // not prefetched (rare)
+        // keys of the following block
+        int nx_it = -1, nx_j = 0;
+        if (j + 1 < I.nb) {
+          load_keys(I, j + 1, nxt);
+          nx_it = it;
+          nx_j = j + 1;
+        } else if (have2) {
+          load_keys(I2, 0, nxt);
+          nx_it = it2;
+        }
         const int s = n % kStages;
         if (n >= kStages) wait(bKVEmpty + s, n / kStages - 1);
         const uint32_t kd = kv_s + (uint32_t)(s * 2 * L::KB);
         const uint32_t vd = kd + L::KB;
 #pragma unroll
-        for (int u = 0; u < kKB / RPP; ++u) {
+        for (int u = 0; u < KR; ++u) {
           const int row = r0 + RPP * u;
-          const int pos = j * kKB + row;
-          const bool ok = pos < I.list_len;
-          const int key = ok ? (I.list ? __ldg(I.list + pos) : pos) : 0;
-          if (c == 0) keys_s[s * kKB + row] = ok ? key : kNoKey;
-          const size_t src = bhoff + (size_t)key * D + c * 8;
+          const bool ok = cur[u] != kNoKey;
+          const size_t src = bhoff + (size_t)(ok ? cur[u] : 0) * D + c * 8;
           const uint32_t off = (uint32_t)(cb * L::KVCB + row * 128 + ((cc ^ (row & 7)) << 4));
-          cp_async_16(kd + off, kbase + src, ok ? 16 : 0);
-          cp_async_16(vd + off, vbase + src, ok ? 16 : 0);
+          cp_async_16(kd + off, a.k + src, ok ? 16 : 0);
+          cp_async_16(vd + off, a.v + src, ok ? 16 : 0);
         }
-        cp_async_commit();
-        // the previous block of this thread has landed: publish it
-        if (pend >= 0) {
-          cp_async_wait<1>();
-          fence_async_smem();
-          mbar_arrive(bar(bKVFull + pend));
-        }
-        pend = s;
+        cp_async_mbar_arrive(bar(bKVFull + s));
+#pragma unroll
+        for (int u = 0; u < KR; ++u) cur[u] = nxt[u];
+        pf_it = nx_it;
+        pf_j = nx_j;
       }
     }
-    cp_async_wait<0>();
-    if (pend >= 0) {
-      fence_async_smem();
-      mbar_arrive(bar(bKVFull + pend));
-    }
+    asm volatile("cp.async.wait_all;\n" ::: "memory");
     // no TMA copy may still be in flight when the CTA exits
     if (pt == 0 && qn > 0 && !mbar_wait_bounded(bar(bQFull + ((qn - 1) & 1)), ((qn - 1) >> 1) & 1))
       raise_error(a.err, kErrTimeout);
-  } else if (warp == 8) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
       const uint32_t id1 = tc::idesc_bf16_f32(128, kKB);
@@ -251,10 +274,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::fence_after();
         auto mma1 = [&](int m) {   // S[m & 1] = Q K_m^T
           const int s = m % kStages, sb = m & 1;
-          wait(bKVFull + s, m / kStages);
-          if (m >= 2) wait(bSEmpty + sb, (m >> 1) - 1);
+          fence_async_smem();   // K / V arrived by cp.async
           tc::fence_after();
-          const uint32_t d = tmem + (uint32_t)(sb * kKB);
+          const uint32_t d = tmem + kColS + (uint32_t)(sb * kKB);
           const uint32_t ks = kv_s + (uint32_t)(s * 2 * L::KB);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
@@ -265,25 +287,50 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc::commit(bar(bSFull + sb));
         };
-        auto mma2 = [&](int m, int j) {   // O[ob] += P[m & 1] V_m
+        auto mma2 = [&](int m, int j) {   // O[ob] += P[m & 1] V_m, P from TMEM
           const int s = m % kStages, pb = m & 1;
-          wait(bPFull + pb, m >> 1);
-          if (j == 0 && qn >= 2) wait(bOEmpty + ob, (qn >> 1) - 1);
           tc::fence_after();
-          const uint32_t d = tmem + 128u + (uint32_t)(ob * 128);
+          const uint32_t d = tmem + kColO + (uint32_t)(ob * 128);
+          const uint32_t pa = tmem + kColP + (uint32_t)(pb * (kKB / 2));
           const uint32_t vs = kv_s + (uint32_t)(s * 2 * L::KB + L::KB);
 #pragma unroll
           for (int kk = 0; kk < kKB / 16; ++kk)
-            tc::mma_bf16(d, tc::smem_desc_sw128(p_s + pb * L::PB + kk * 32),
-                         tc::smem_desc_sw128_mn(vs + kk * 2048, L::KVCB), id2, (j > 0 || kk > 0) ? 1u : 0u);
+            tc::mma_bf16_ts(d, pa + (uint32_t)(kk * 8), tc::smem_desc_sw128_mn(vs + kk * 2048, L::KVCB), id2,
+                            (j > 0 || kk > 0) ? 1u : 0u);
           tc::commit(bar(bKVEmpty + s));
           tc::commit(bar(bPEmpty + pb));
           tc::commit(bar(bODone + ob));
         };
-        if (I.nb > 0) mma1(n);
-        for (int j = 0; j < I.nb; ++j) {
-          if (j + 1 < I.nb) mma1(n + j + 1);
-          mma2(n + j, j);
+        // issue whichever product is ready: S of a later block (up to two
+        // ahead of P V) or P V of the oldest block whose P is published
+        int i1 = 0, i2 = 0;
+        long long t_last = clock64();
+        while (i2 < I.nb && !*stop) {
+          bool did = false;
+          if (i1 < I.nb && i1 <= i2 + 2) {
+            const int m = n + i1;
+            if (mbar_test(bar(bKVFull + m % kStages), (uint32_t)((m / kStages) & 1)) &&
+                (m < 2 || mbar_test(bar(bSEmpty + (m & 1)), (uint32_t)(((m >> 1) - 1) & 1)))) {
+              mma1(m);
+              ++i1;
+              did = true;
+            }
+          }
+          if (!did && i2 < i1) {
+            const int m = n + i2;
+            if (mbar_test(bar(bPFull + (m & 1)), (uint32_t)((m >> 1) & 1)) &&
+                (i2 > 0 || qn < 2 || mbar_test(bar(bOEmpty + ob), (uint32_t)(((qn >> 1) - 1) & 1)))) {
+              mma2(m, i2);
+              ++i2;
+              did = true;
+            }
+          }
+          if (did) {
+            t_last = clock64();
+          } else if (clock64() - t_last > (1ll << 32)) {
+            *stop = 1;
+            raise_error(a.err, kErrTimeout);
+          }
         }
         tc::commit(bar(bQEmpty + qb));
         n += I.nb;
@@ -294,9 +341,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int r = threadIdx.x;                        // TMEM lane = MMA row
-    const uint32_t lane_addr = (uint32_t)(32 * warp) << 16;
+    // two warpgroups share every row: group wg takes S columns
+    // [32 wg, 32 wg + 32) of each block and O columns [wg D/2, (wg+1) D/2);
+    // they exchange row maxima (and at the end row sums) through shared
+    // memory at a named barrier
+    const int wg = warp >> 2;
+    const int r = threadIdx.x & 127;                  // TMEM lane = MMA row
+    const uint32_t lane_addr = (uint32_t)(32 * (warp & 3)) << 16;
     const float scale2 = kLog2e * rsqrtf((float)D);
+    float* xch = reinterpret_cast<float*>(sm + L::xch);   // [2 groups][128]
+    constexpr int OC = D / 2;                             // O columns per group
     int n = 0, qn = 0;
     int ocnt[2] = {0, 0};                             // completed MMA2 groups per O buffer
     for (int it = blockIdx.x; it < items; it += gridDim.x, ++qn) {
@@ -306,43 +360,50 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int pos = I.i0 + qi;
       const bool valid = g < heads_rb && qi < I.rows_t;
       float m_used = -INFINITY, l = 0.f;
+      // last key of block j (lists are ascending), loaded one block ahead
+      auto last_key = [&](int j) {
+        const int q = min(j * kKB + kKB, I.list_len) - 1;
+        return I.list ? __ldg(I.list + q) : q;
+      };
+      int last_next = I.nb > 0 ? last_key(0) : 0;
       for (int j = 0; j < I.nb; ++j) {
         const int m = n + j;
-        const int sb = m & 1, s = m % kStages, pb = m & 1;
+        const int sb = m & 1, pb = m & 1;
+        // the block needs a per-key check if it holds keys past the list
+        // end or (causal) keys after the tile start
+        const int pos0 = j * kKB;
+        const bool tail = pos0 + kKB > I.list_len;
+        const int last = last_next;
+        if (j + 1 < I.nb) last_next = last_key(j + 1);
+        const bool check = tail || (causal && last > I.i0);
         wait(bSFull + sb, m >> 1);
-        wait(bKVFull + s, m / kStages);   // the block's key indices
         tc::fence_after();
-        float v[kKB];
-        tc::tmem_ld32(tmem + lane_addr + (uint32_t)(sb * kKB), *reinterpret_cast<float(*)[32]>(v));
-        tc::tmem_ld32(tmem + lane_addr + (uint32_t)(sb * kKB + 32), *reinterpret_cast<float(*)[32]>(v + 32));
+        float v[32];
+        tc::tmem_ld32(tmem + lane_addr + kColS + (uint32_t)(sb * kKB + 32 * wg), v);
         tc::fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(bSEmpty + sb));
-        // mask: lists are ascending with kNoKey past the end, so the last
-        // entry tells whether any key of the block needs a check
-        const int* kb = keys_s + s * kKB;
-        const int last = kb[kKB - 1];
-        if (causal ? last > I.i0 : last == kNoKey) {
+        if (check) {
 #pragma unroll
-          for (int c4 = 0; c4 < kKB; c4 += 4) {
-            const int4 kk = *reinterpret_cast<const int4*>(kb + c4);
-            if (causal) {
-              if (kk.x > pos) v[c4] = -INFINITY;
-              if (kk.y > pos) v[c4 + 1] = -INFINITY;
-              if (kk.z > pos) v[c4 + 2] = -INFINITY;
-              if (kk.w > pos) v[c4 + 3] = -INFINITY;
-            } else {
-              if (kk.x == kNoKey) v[c4] = -INFINITY;
-              if (kk.y == kNoKey) v[c4 + 1] = -INFINITY;
-              if (kk.z == kNoKey) v[c4 + 2] = -INFINITY;
-              if (kk.w == kNoKey) v[c4 + 3] = -INFINITY;
-            }
+          for (int c = 0; c < 32; ++c) {
+            const int q = pos0 + 32 * wg + c;
+            const int key = q < I.list_len ? (I.list ? __ldg(I.list + q) : q) : kNoKey;
+            if (key == kNoKey || (causal && key > pos)) v[c] = -INFINITY;
           }
         }
-        float mx = v[0];
+        float mx4[4] = {v[0], v[1], v[2], v[3]};
 #pragma unroll
-        for (int c = 1; c < kKB; ++c) mx = fmaxf(mx, v[c]);
-        const float mx2 = mx * scale2;   // scale > 0 keeps the order; -inf stays -inf
+        for (int c = 4; c < 32; c += 4) {
+          mx4[0] = fmaxf(mx4[0], v[c]);
+          mx4[1] = fmaxf(mx4[1], v[c + 1]);
+          mx4[2] = fmaxf(mx4[2], v[c + 2]);
+          mx4[3] = fmaxf(mx4[3], v[c + 3]);
+        }
+        const float mine = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        xch[wg * 128 + r] = mine;
+        asm volatile("bar.sync 1, 256;\n" ::: "memory");
+        const float mx2 = fmaxf(mine, xch[(wg ^ 1) * 128 + r]) * scale2;   // scale > 0 keeps the order
+        asm volatile("bar.sync 1, 256;\n" ::: "memory");   // xch is rewritten next
         float m_new = m_used;
         bool resc = false;
         if (mx2 > m_used) {
@@ -354,14 +415,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (__any_sync(0xffffffffu, resc)) {
-          // rescale O (and l) once the previous block's P V has landed
+          // rescale this group's half of O (and l) once the previous
+          // block's P V has landed
           wait(bODone + ob, ocnt[ob] + j - 1);
           tc::fence_after();
           const float alpha = resc ? exp2f(m_used - m_new) : 1.0f;
 #pragma unroll 1
-          for (int c32 = 0; c32 < D / 32; ++c32) {
+          for (int c32 = 0; c32 < OC / 32; ++c32) {
             float o[32];
-            const uint32_t ta = tmem + lane_addr + 128u + (uint32_t)(ob * 128 + c32 * 32);
+            const uint32_t ta = tmem + lane_addr + kColO + (uint32_t)(ob * 128 + wg * OC + c32 * 32);
             tc::tmem_ld32(ta, o);
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] *= alpha;
@@ -370,46 +432,54 @@ __global__ void __launch_bounds__(kThreads, 1)
           l *= alpha;
         }
         m_used = m_new;
-        // P = exp2(s * scale2 - m_used) in bf16, row r of the block's A tile
-        uint32_t pk[kKB / 2];
-        float ps = 0.f;
+        // P = exp2(s * scale2 - m_used) in bf16: this group's 32 columns of
+        // row r of the block's A tile
+        uint32_t pk[16];
         if (m_used == -INFINITY) {
 #pragma unroll
-          for (int c = 0; c < kKB / 2; ++c) pk[c] = 0u;
+          for (int c = 0; c < 16; ++c) pk[c] = 0u;
         } else {
           const float nm = -m_used;
+          float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int c = 0; c < kKB; c += 2) {
+          for (int c = 0; c < 32; c += 4) {
             const float p0 = exp2f(fmaf(v[c], scale2, nm));
             const float p1 = exp2f(fmaf(v[c + 1], scale2, nm));
-            ps += p0 + p1;
+            const float p2 = exp2f(fmaf(v[c + 2], scale2, nm));
+            const float p3 = exp2f(fmaf(v[c + 3], scale2, nm));
+            ps[0] += p0;
+            ps[1] += p1;
+            ps[2] += p2;
+            ps[3] += p3;
             pk[c / 2] = pack_bf16(p0, p1);
+            pk[c / 2 + 1] = pack_bf16(p2, p3);
           }
+          l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
         }
-        l += ps;
         if (m >= 2) wait(bPEmpty + pb, (m >> 1) - 1);
-        const uint32_t prow = p_s + (uint32_t)(pb * L::PB + r * 128);
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc)
-          st_shared_v4(prow + ((cc ^ (r & 7)) << 4), pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
-        fence_async_smem();
-        tc::fence_before();   // orders a TMEM rescale of O before the next P V
+        // this group's 16 columns of P (bf16 pairs) in TMEM, row r
+        tc::tmem_st16(tmem + lane_addr + kColP + (uint32_t)(pb * (kKB / 2) + 16 * wg), pk);
+        tc::fence_before();   // orders the P store and a TMEM rescale of O before the next P V
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(bPFull + pb));
       }
-      // ---- output rows: O / l, bf16
+      // ---- output rows: O / l, bf16 (row sums of both groups)
+      xch[wg * 128 + r] = l;
+      asm volatile("bar.sync 1, 256;\n" ::: "memory");
+      const float lt = l + xch[(wg ^ 1) * 128 + r];
+      asm volatile("bar.sync 1, 256;\n" ::: "memory");   // xch is rewritten next
       if (I.nb > 0) {
         wait(bODone + ob, ocnt[ob] + I.nb - 1);
         tc::fence_after();
       }
       ocnt[ob] += I.nb;
-      const float inv = l > 0.f ? 1.0f / l : 0.0f;
-      __nv_bfloat16* orow = a.o + ((size_t)(I.b * a.Hq + I.hq0 + g) * a.N + pos) * D;
+      const float inv = lt > 0.f ? 1.0f / lt : 0.0f;
+      __nv_bfloat16* orow = a.o + ((size_t)(I.b * a.Hq + I.hq0 + g) * a.N + pos) * D + wg * OC;
 #pragma unroll 1
-      for (int c32 = 0; c32 < D / 32; ++c32) {
+      for (int c32 = 0; c32 < OC / 32; ++c32) {
         float o[32];
         if (I.nb > 0) {
-          tc::tmem_ld32(tmem + lane_addr + 128u + (uint32_t)(ob * 128 + c32 * 32), o);
+          tc::tmem_ld32(tmem + lane_addr + kColO + (uint32_t)(ob * 128 + wg * OC + c32 * 32), o);
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = 0.f;
@@ -426,9 +496,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (valid && a.lse)
+      if (valid && wg == 0 && a.lse)
         a.lse[(size_t)(I.b * a.Hq + I.hq0 + g) * a.N + pos] =
-            l > 0.f ? (m_used + log2f(l)) * (float)kLn2 : -INFINITY;
+            lt > 0.f ? (m_used + log2f(lt)) * (float)kLn2 : -INFINITY;
       tc::fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(bOEmpty + ob));
@@ -439,7 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ------------------------------------------------------------ teardown
   tc::fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == kMmaWarp) {
     tc::fence_after();
     tc::tmem_dealloc(tmem, 512);
   }
