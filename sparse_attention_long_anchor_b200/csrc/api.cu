@@ -252,7 +252,9 @@ int kascade_select(const kascade_shape* s, const void* q, const void* k, int32_t
   a.grid = pl.grid;
   a.idx = idx;
   a.flags = s->flags & KASCADE_FLAG_PDL;
+  a.err = err_word(ws, ws_bytes);
   if (is_decode(s)) {
+    if (pl.cluster && anchor_select_fused_ok(a)) return cuda_status(launch_anchor_select_fused(a, st));
     DecodeScoreArgs d{};
     d.flags = a.flags;
     d.q = a.q;

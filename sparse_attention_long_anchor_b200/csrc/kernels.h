@@ -43,12 +43,18 @@ struct SelArgs {
   int grid;
   int32_t* idx;            // output
   int flags;
+  int* err;                // device error word (a bounded wait gave up), may be NULL
 };
 size_t select_scratch_bytes_per_cta(int n_max);
-// decode: one 8-CTA cluster per (batch, kv head) when N / 8 <= 16384
+// decode: one 8-CTA cluster per (batch, kv head) when N / 8 <= 16384 (band
+// scratch also sized for the fused kernel)
 bool select_decode_cluster_ok(int N);
 size_t select_decode_cluster_scratch(int B, int Hkv, int N);   // band entries
 cudaError_t launch_select_decode_cluster(const SelArgs& a, cudaStream_t stream);
+// decode: fused scoring + selection (one cluster per (batch, kv head), K
+// streamed once, scores kept on chip) when the shape and device allow it
+bool anchor_select_fused_ok(const SelArgs& a);
+cudaError_t launch_anchor_select_fused(const SelArgs& a, cudaStream_t stream);
 int select_grid(bool prefill, int problems, int num_sms);
 cudaError_t launch_select(const SelArgs& a, cudaStream_t stream);
 

@@ -2,18 +2,25 @@
 // (batch, kv head) (Kascade README, Abstract: exact Top-k indices computed in
 // the anchor layers; selection is head-aware).
 //
-// The N candidate keys are split across the kCS CTAs of a cluster; each CTA
+// The N candidate keys are split across the CS CTAs of a cluster; each CTA
 // keeps the fp32 pooled scores of its keys in shared memory:
-//   P_j = (1/G) sum_g exp2(s2_gj - m2_g) / l_g
-// (s2 and the per-split softmax statistics come from the scoring kernel).
-// Radix select runs on the fp32 bit patterns with 8-bit digits: every CTA
-// histograms its own keys, the histograms are summed over distributed
-// shared memory, and every CTA derives the same digit.  The band of keys
-// within delta (relative) of the k-th fp32 value is then re-scored in fp64
-// (exact bf16 products, fp64 sums and exp2) and settled by (value desc,
-// index asc); counts are exchanged over DSMEM and each CTA writes its
-// selected keys, ascending, at its prefix offset.  No CTA waits on anything
-// but cluster barriers, which every CTA of the cluster reaches.
+//   P_j = (1/G) sum_g exp2(s2_gj - m2_g) / l_g,   s2 = q . k_j log2(e)/sqrt(d)
+// Two kernels produce them:
+//   * anchor_select_kernel (the usual path) streams the CTA's contiguous K
+//     rows into shared memory with bulk TMA copies, scores them with warp
+//     MMAs (keys as the MMA rows, the <= 8 query heads of the group as its
+//     columns), keeps the scores in shared memory and takes the softmax
+//     statistics of every head over the cluster through distributed shared
+//     memory: one launch, no score round trip through global memory;
+//   * select_decode_cluster_kernel (fallback for contexts too long to keep
+//     the scores on chip, or devices without 16-CTA clusters) reads the
+//     scores and per-split statistics written by the scoring kernel.
+// Both then run the same cluster Top-k: radix select on the fp32 bit
+// patterns with 8-bit digits, histograms summed over distributed shared
+// memory; the band of keys within delta (relative) of the k-th fp32 value is
+// re-scored in fp64 (exact bf16 products, fp64 sums and exp2) and settled by
+// (value desc, index asc); counts are exchanged over DSMEM and each CTA
+// writes its selected keys, ascending, at its prefix offset.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -25,12 +32,15 @@ namespace kascade {
 
 namespace {
 
-constexpr int kCS = 8;            // CTAs per cluster
 constexpr int kCNT = 512;         // threads per CTA
+constexpr int kWarpsC = kCNT / 32;
 constexpr int kCBins = 256;       // 8-bit digits
 constexpr int kSmallBand = 1024;  // band sizes settled by direct ranking
 constexpr float kBandDelta = 1.0f / 8192.0f;
 constexpr float kBandFloor = 0x1p-96f;
+constexpr int kFallbackCS = 8;    // cluster size of the fallback kernel
+constexpr int kRoundKeys = 256;   // fused kernel: K rows per streamed round
+constexpr int kErrTimeout = 5;
 
 struct CSh {
   unsigned hist[2][kCBins];
@@ -41,19 +51,21 @@ struct CSh {
   float m2[8];
   double l[8];
   float inv_l[8];
+  float cmax[8];          // fused: this CTA's max score of each head (read by the cluster)
+  double csum[8];         // fused: this CTA's sum of exp2(s2 - cmax) of each head
+  float wpool[8];         // fused: weight exp2(cmax - m2) / l of the stored terms
+  float wmax[kWarpsC][8];
+  double wsum[kWarpsC][8];
+  unsigned long long full[2];   // fused: K round barriers
   int b_idx[kSmallBand];
   double b_val[kSmallBand];
 };
 
 constexpr size_t kCHead = (sizeof(CSh) + 127) / 128 * 128;
 
-__host__ __device__ constexpr size_t cluster_dyn_bytes(int keys_per_cta) {
-  // q rows fp32 [8][128], v[keys] fp32, state[keys] bytes
-  return kCHead + 8 * 128 * 4 + (size_t)keys_per_cta * 4 + (size_t)keys_per_cta;
-}
-
 // Sum the cluster's histograms (buffer `buf`) and find the digit holding the
 // need-th largest element.  Every CTA computes the same (bin, above).
+template <int CS>
 __device__ void cluster_find_bin(cg::cluster_group& cluster, CSh& sh, int buf, int need) {
   __syncthreads();
   cluster.sync();
@@ -63,7 +75,7 @@ __device__ void cluster_find_bin(cg::cluster_group& cluster, CSh& sh, int buf, i
   if (t < kCBins) {
     bin = kCBins - 1 - t;   // thread 0 holds the largest digit
 #pragma unroll
-    for (int r = 0; r < kCS; ++r) {
+    for (int r = 0; r < CS; ++r) {
       const unsigned* rh = cluster.map_shared_rank(&sh.hist[buf][0], r);
       local += (int)rh[bin];
     }
@@ -84,15 +96,19 @@ __device__ __forceinline__ void clear_hist(CSh& sh, int buf) {
   __syncthreads();
 }
 
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.aligned;\n" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;\n" ::: "memory"); }
+
 // exchange one int per CTA: returns the total and the sum over lower ranks
-__device__ void cluster_exchange(cg::cluster_group& cluster, CSh& sh, int slot, int mine, int rank,
-                                 int* total, int* below) {
+template <int CS>
+__device__ void cluster_exchange(cg::cluster_group& cluster, CSh& sh, int slot, int mine, int rank, int* total,
+                                 int* below) {
   if (threadIdx.x == 0) sh.xchg[slot] = mine;
   __syncthreads();
   cluster.sync();
   int tot = 0, bel = 0;
 #pragma unroll
-  for (int r = 0; r < kCS; ++r) {
+  for (int r = 0; r < CS; ++r) {
     const int x = *cluster.map_shared_rank(&sh.xchg[slot], r);
     tot += x;
     bel += r < rank ? x : 0;
@@ -101,70 +117,21 @@ __device__ void cluster_exchange(cg::cluster_group& cluster, CSh& sh, int slot, 
   *below = bel;
 }
 
-__global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(kCNT)
-    select_decode_cluster_kernel(const SelArgs a, int keys_per_cta) {
-  pdl_wait();
-  pdl_launch_dependents();
-  extern __shared__ __align__(128) char smem_raw[];
-  CSh& sh = *reinterpret_cast<CSh*>(smem_raw);
-  float* qf = reinterpret_cast<float*>(smem_raw + kCHead);
-  float* v = qf + 8 * 128;
-  uint8_t* st = reinterpret_cast<uint8_t*>(v + keys_per_cta);
-
-  cg::cluster_group cluster = cg::this_cluster();
-  const int rank = (int)cluster.block_rank();
+// Everything after the pooled scores: exact Top-K over the cluster of the
+// pooled values v[0, cnt) of this CTA (keys j0 + i), written ascending into
+// out[0, K).  sh.m2 / sh.l hold the softmax statistics of the G heads and
+// qf the fp32 query rows (for the fp64 band).  Band scratch: this CTA's
+// `per` entries at band_idx / band_val; the cluster's CS * per entries start
+// at band_idx0 / band_val0.
+template <int CS>
+__device__ void cluster_topk(cg::cluster_group& cluster, CSh& sh, const float* v, uint8_t* st, int cnt, int j0,
+                             int rank, int K, int per, int32_t* out, int32_t* band_idx, double* band_val,
+                             const int32_t* band_idx0, const double* band_val0, const float* qf,
+                             const __nv_bfloat16* kb, int G, int D) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int bh = blockIdx.y;
-  const int b = bh / a.Hkv, h = bh - b * a.Hkv;
-  const int G = a.G, D = a.D, N = a.N;
-  const int K = topk_count(N, a.num, a.den);
-  const int j0 = rank * keys_per_cta;
-  const int j1 = min(N, j0 + keys_per_cta);
-  const int cnt = max(0, j1 - j0);
-  int32_t* out = a.idx + (size_t)bh * K;
-  int32_t* band_idx = a.band_idx + (size_t)bh * kCS * keys_per_cta + (size_t)rank * keys_per_cta;
-  double* band_val = a.band_val + (size_t)bh * kCS * keys_per_cta + (size_t)rank * keys_per_cta;
-
-  if (K >= N) {   // everything is selected (same branch in every CTA)
-    for (int i = tid; i < cnt; i += kCNT) out[j0 + i] = j0 + i;
-    return;
-  }
-
-  // softmax statistics of the G query heads from the scoring kernel's splits
-  for (int g = warp; g < G; g += kCNT / 32) {
-    const size_t row = (size_t)(b * a.Hq + h * G + g) * a.splits;
-    float m = -INFINITY;
-    for (int s = lane; s < a.splits; s += 32) m = fmaxf(m, a.m_part[row + s]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    double l = 0.0;
-    for (int s = lane; s < a.splits; s += 32) l += a.l_part[row + s] * exp2((double)a.m_part[row + s] - (double)m);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    if (lane == 0) {
-      sh.m2[g] = m;
-      sh.l[g] = l;
-      sh.inv_l[g] = (float)(1.0 / l);
-    }
-  }
-  for (int e = tid; e < G * D; e += kCNT) {
-    const int g = e / D, dd = e - g * D;
-    qf[e] = __bfloat162float(a.q[(size_t)(b * a.Hq + h * G + g) * D + dd]);
-  }
   clear_hist(sh, 0);
   clear_hist(sh, 1);
-  __syncthreads();
-
-  // pooled fp32 scores of this CTA's keys + histogram of the top digit
-  const float* srow = a.s2 + (size_t)(b * a.Hq + h * G) * N;
-  const float invG = 1.0f / (float)G;
-  for (int i = tid; i < cnt; i += kCNT) {
-    float acc = 0.f;
-    for (int g = 0; g < G; ++g) acc += exp2f(srow[(size_t)g * N + j0 + i] - sh.m2[g]) * sh.inv_l[g];
-    acc *= invG;
-    v[i] = acc;
-    atomicAdd(&sh.hist[0][__float_as_uint(acc) >> 24], 1u);
-  }
+  for (int i = tid; i < cnt; i += kCNT) atomicAdd(&sh.hist[0][__float_as_uint(v[i]) >> 24], 1u);
 
   // radix select over the cluster: digits [31:24] [23:16] [15:8] [7:0]
   int need = K;
@@ -178,7 +145,7 @@ __global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(kCNT)
         if ((x >> (shift + 8)) == (prefix >> (shift + 8))) atomicAdd(&sh.hist[buf][(x >> shift) & 255u], 1u);
       }
     }
-    cluster_find_bin(cluster, sh, buf, need);
+    cluster_find_bin<CS>(cluster, sh, buf, need);
     prefix |= (unsigned)sh.bin << shift;
     need -= sh.above;
     clear_hist(sh, buf ^ 1);   // the other buffer's readers have all passed this pass's barrier
@@ -207,15 +174,28 @@ __global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(kCNT)
   if (lane == 0 && my_hi) atomicAdd(&sh.chi, my_hi);
   __syncthreads();
   const int nb = sh.nb, chi = sh.chi;
-  int chi_total, chi_below, nb_total, nb_below;
-  cluster_exchange(cluster, sh, 0, chi, rank, &chi_total, &chi_below);
-  cluster_exchange(cluster, sh, 1, nb, rank, &nb_total, &nb_below);
+  // one exchange of (count above the band, band size)
+  if (tid == 0) {
+    sh.xchg[0] = chi;
+    sh.xchg[1] = nb;
+  }
+  __syncthreads();
+  cluster.sync();
+  int chi_total = 0, chi_below = 0, nb_total = 0, nb_below = 0;
+#pragma unroll
+  for (int r = 0; r < CS; ++r) {
+    const int x = *cluster.map_shared_rank(&sh.xchg[0], r);
+    const int y = *cluster.map_shared_rank(&sh.xchg[1], r);
+    chi_total += x;
+    nb_total += y;
+    chi_below += r < rank ? x : 0;
+    nb_below += r < rank ? y : 0;
+  }
   const int need_band = K - chi_total;
 
   // fp64 pooled scores of this CTA's band members, one warp per member
   const double c2 = 1.4426950408889634 / sqrt((double)D);
-  const __nv_bfloat16* kb = a.k + (size_t)bh * N * D;
-  for (int i = warp; i < nb; i += kCNT / 32) {
+  for (int i = warp; i < nb; i += kWarpsC) {
     const int j = band_idx[i];
     const __nv_bfloat16* krow = kb + (size_t)j * D;
     float kv[4];
@@ -237,34 +217,47 @@ __global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(kCNT)
   __syncthreads();
   cluster.sync();
 
-  int tie_quota = 0;
+  int tie_quota = 0, sel_below = 0;
+  auto flag_of = [&](int i) -> int {
+    const float x = v[i];
+    return x > hi || (x >= lo && st[i] == 1);
+  };
   if (nb_total <= kSmallBand) {
-    // every CTA gathers the whole band and ranks its own members
-    const int32_t* base_idx = a.band_idx + (size_t)bh * kCS * keys_per_cta;
-    const double* base_val = a.band_val + (size_t)bh * kCS * keys_per_cta;
+    // every CTA gathers the whole band (ordered by CTA rank) and ranks the
+    // members of the lower CTAs and its own: its own are marked, the lower
+    // ones give this CTA's output offset
     for (int t = tid; t < nb_total; t += kCNT) {
       int r = 0, off = t;
-      while (r < kCS) {
+      while (r < CS) {
         const int nr = *cluster.map_shared_rank(&sh.xchg[1], r);
         if (off < nr) break;
         off -= nr;
         ++r;
       }
-      sh.b_idx[t] = __ldcg(base_idx + (size_t)r * keys_per_cta + off);
-      sh.b_val[t] = __ldcg(base_val + (size_t)r * keys_per_cta + off);
+      sh.b_idx[t] = __ldcg(band_idx0 + (size_t)r * per + off);
+      sh.b_val[t] = __ldcg(band_val0 + (size_t)r * per + off);
     }
+    cluster_arrive();   // the last reads of other CTAs' shared memory
     __syncthreads();
-    for (int i = tid; i < nb; i += kCNT) {
-      const int me = nb_below + i;
-      const double mv = sh.b_val[me];
-      const int mj = sh.b_idx[me];
+    int low_sel = 0;
+    for (int t = tid; t < nb_below + nb; t += kCNT) {
+      const double mv = sh.b_val[t];
+      const int mj = sh.b_idx[t];
       int rk = 0;
-      for (int t = 0; t < nb_total; ++t) {
-        const double ov = sh.b_val[t];
-        rk += (ov > mv) || (ov == mv && sh.b_idx[t] < mj);
+      for (int u = 0; u < nb_total; ++u) {
+        const double ov = sh.b_val[u];
+        rk += (ov > mv) || (ov == mv && sh.b_idx[u] < mj);
       }
-      st[mj - j0] = rk < need_band ? 1 : 0;
+      if (t < nb_below) low_sel += rk < need_band;
+      else st[mj - j0] = rk < need_band ? 1 : 0;
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) low_sel += __shfl_xor_sync(0xffffffffu, low_sel, o);
+    if (tid == 0) sh.chi = 0;
+    __syncthreads();
+    if (lane == 0 && low_sel) atomicAdd(&sh.chi, low_sel);
+    __syncthreads();
+    sel_below = chi_below + sh.chi;
   } else {
     // large band (degenerate inputs): cluster radix select on the fp64 bits
     unsigned long long pre = 0;
@@ -280,7 +273,7 @@ __global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(kCNT)
         if (pass == 0 || (x >> (shift + 8)) == (pre >> (shift + 8)))
           atomicAdd(&sh.hist[buf][(x >> shift) & 255ull], 1u);
       }
-      cluster_find_bin(cluster, sh, buf, nd);
+      cluster_find_bin<CS>(cluster, sh, buf, nd);
       pre |= (unsigned long long)sh.bin << shift;
       nd -= sh.above;
       clear_hist(sh, buf ^ 1);
@@ -300,61 +293,435 @@ __global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(kCNT)
     if (lane == 0 && my_ties) atomicAdd(&sh.nb, my_ties);
     __syncthreads();
     int ties_total, ties_below;
-    cluster_exchange(cluster, sh, 2, sh.nb, rank, &ties_total, &ties_below);
+    cluster_exchange<CS>(cluster, sh, 2, sh.nb, rank, &ties_total, &ties_below);
     tie_quota = min(max(nd - ties_below, 0), sh.nb);   // lower ranks hold lower indices
+    __syncthreads();
+    int mine = 0;
+    for (int i = tid; i < cnt; i += kCNT) mine += flag_of(i);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
+    if (tid == 0) sh.chi = 0;
+    __syncthreads();
+    if (lane == 0 && mine) atomicAdd(&sh.chi, mine);
+    __syncthreads();
+    int sel_total;
+    cluster_exchange<CS>(cluster, sh, 3, sh.chi + tie_quota, rank, &sel_total, &sel_below);
+    cluster_arrive();   // the last reads of other CTAs' shared memory
   }
   __syncthreads();
 
-  // count, exchange offsets, then write ascending
-  int mine = 0;
-  for (int i = tid; i < cnt; i += kCNT) {
-    const float x = v[i];
-    mine += x > hi || (x >= lo && st[i] == 1);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
-  if (tid == 0) sh.chi = 0;
-  __syncthreads();
-  if (lane == 0 && mine) atomicAdd(&sh.chi, mine);
-  __syncthreads();
-  int sel_total, sel_below;
-  cluster_exchange(cluster, sh, 3, sh.chi + tie_quota, rank, &sel_total, &sel_below);
-  int written = sel_below, ties_taken = 0;
-  for (int base = 0; base < cnt; base += kCNT) {
-    const int i = base + tid;
-    int flag = 0, tie = 0;
-    if (i < cnt) {
-      const float x = v[i];
-      if (x > hi) {
-        flag = 1;
-      } else if (x >= lo) {
-        flag = st[i] == 1;
-        tie = st[i] == 2;
+  // write ascending at this CTA's offset
+  if (tie_quota == 0) {
+    // one scan: thread t owns the consecutive keys [t * kpt, (t + 1) * kpt)
+    const int kpt = (cnt + kCNT - 1) / kCNT;
+    const int b0 = min(cnt, tid * kpt), b1 = min(cnt, b0 + kpt);
+    int c = 0;
+    for (int i = b0; i < b1; ++i) c += flag_of(i);
+    const int incl = block_inclusive_scan<kCNT>(c, sh.scan_buf, nullptr);
+    int w = sel_below + incl - c;
+    for (int i = b0; i < b1; ++i)
+      if (flag_of(i)) out[w++] = j0 + i;
+  } else {
+    int written = sel_below, ties_taken = 0;
+    for (int base = 0; base < cnt; base += kCNT) {
+      const int i = base + tid;
+      int flag = 0, tie = 0;
+      if (i < cnt) {
+        const float x = v[i];
+        if (x > hi) {
+          flag = 1;
+        } else if (x >= lo) {
+          flag = st[i] == 1;
+          tie = st[i] == 2;
+        }
       }
-    }
-    if (tie_quota > 0) {
       int tt;
       const int tincl = block_inclusive_scan<kCNT>(tie, sh.scan_buf, &tt);
       if (tie && ties_taken + tincl - 1 < tie_quota) flag = 1;
       ties_taken += tt;
+      int total;
+      const int incl = block_inclusive_scan<kCNT>(flag, sh.scan_buf, &total);
+      if (flag) out[written + incl - 1] = j0 + i;
+      written += total;
     }
-    int total;
-    const int incl = block_inclusive_scan<kCNT>(flag, sh.scan_buf, &total);
-    if (flag) out[written + incl - 1] = j0 + i;
-    written += total;
   }
   // no CTA may leave while another can still read its shared memory
+  cluster_wait();
+}
+
+// ---------------------------------------------------------------- fallback
+
+__host__ __device__ constexpr size_t cluster_dyn_bytes(int keys_per_cta) {
+  // q rows fp32 [8][128], v[keys] fp32, state[keys] bytes
+  return kCHead + 8 * 128 * 4 + (size_t)keys_per_cta * 4 + (size_t)keys_per_cta;
+}
+
+__global__ void __cluster_dims__(kFallbackCS, 1, 1) __launch_bounds__(kCNT)
+    select_decode_cluster_kernel(const SelArgs a, int keys_per_cta) {
+  pdl_wait();
+  pdl_launch_dependents();
+  extern __shared__ __align__(128) char smem_raw[];
+  CSh& sh = *reinterpret_cast<CSh*>(smem_raw);
+  float* qf = reinterpret_cast<float*>(smem_raw + kCHead);
+  float* v = qf + 8 * 128;
+  uint8_t* st = reinterpret_cast<uint8_t*>(v + keys_per_cta);
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int bh = blockIdx.y;
+  const int b = bh / a.Hkv, h = bh - b * a.Hkv;
+  const int G = a.G, D = a.D, N = a.N;
+  const int K = topk_count(N, a.num, a.den);
+  const int j0 = rank * keys_per_cta;
+  const int j1 = min(N, j0 + keys_per_cta);
+  const int cnt = max(0, j1 - j0);
+  int32_t* out = a.idx + (size_t)bh * K;
+  const size_t bbase = (size_t)bh * kFallbackCS * keys_per_cta;
+
+  if (K >= N) {   // everything is selected (same branch in every CTA)
+    for (int i = tid; i < cnt; i += kCNT) out[j0 + i] = j0 + i;
+    return;
+  }
+
+  // softmax statistics of the G query heads from the scoring kernel's splits
+  for (int g = warp; g < G; g += kWarpsC) {
+    const size_t row = (size_t)(b * a.Hq + h * G + g) * a.splits;
+    float m = -INFINITY;
+    for (int s = lane; s < a.splits; s += 32) m = fmaxf(m, a.m_part[row + s]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    double l = 0.0;
+    for (int s = lane; s < a.splits; s += 32) l += a.l_part[row + s] * exp2((double)a.m_part[row + s] - (double)m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane == 0) {
+      sh.m2[g] = m;
+      sh.l[g] = l;
+      sh.inv_l[g] = (float)(1.0 / l);
+    }
+  }
+  for (int e = tid; e < G * D; e += kCNT) {
+    const int g = e / D, dd = e - g * D;
+    qf[e] = __bfloat162float(a.q[(size_t)(b * a.Hq + h * G + g) * D + dd]);
+  }
+  __syncthreads();
+
+  // pooled fp32 scores of this CTA's keys
+  const float* srow = a.s2 + (size_t)(b * a.Hq + h * G) * N;
+  const float invG = 1.0f / (float)G;
+  for (int i = tid; i < cnt; i += kCNT) {
+    float acc = 0.f;
+    for (int g = 0; g < G; ++g) acc += exp2f(srow[(size_t)g * N + j0 + i] - sh.m2[g]) * sh.inv_l[g];
+    v[i] = acc * invG;
+  }
+  __syncthreads();
+  cluster_topk<kFallbackCS>(cluster, sh, v, st, cnt, j0, rank, K, keys_per_cta, out,
+                            a.band_idx + bbase + (size_t)rank * keys_per_cta,
+                            a.band_val + bbase + (size_t)rank * keys_per_cta, a.band_idx + bbase,
+                            a.band_val + bbase, qf, a.k + (size_t)bh * N * D, G, D);
+}
+
+// ------------------------------------------------------------ fused select
+
+template <int D>
+struct ASL {
+  static constexpr size_t qf = kCHead;                               // [8][128] f32
+  static constexpr size_t ring = qf + 8 * 128 * 4;                    // [2][kRoundKeys][D] bf16
+  static constexpr size_t RB = (size_t)kRoundKeys * D * 2;
+  static constexpr size_t sc = ring + 2 * RB;                         // [G][per + 4] f32 scores
+  static size_t bytes(int G, int per) { return sc + (size_t)G * (per + 4) * 4 + (size_t)per + 16; }
+  static_assert(ring % 128 == 0, "bulk copy destination alignment");
+};
+
+template <int CS, int D>
+__global__ void __launch_bounds__(kCNT, 1) anchor_select_kernel(const SelArgs a, int per) {
+  using L = ASL<D>;
+  constexpr int KS = D / 32;
+  pdl_wait();
+  pdl_launch_dependents();
+  extern __shared__ __align__(128) char smem_raw[];
+  CSh& sh = *reinterpret_cast<CSh*>(smem_raw);
+  float* qf = reinterpret_cast<float*>(smem_raw + L::qf);
+  const uint32_t ring = smem_u32(smem_raw) + (uint32_t)L::ring;
+  float* sc = reinterpret_cast<float*>(smem_raw + L::sc);
+  const int SCS = per + 4;   // score row stride (floats)
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, c = lane & 3;
+  const int bh = blockIdx.y;
+  const int b = bh / a.Hkv, h = bh - b * a.Hkv;
+  const int G = a.G, N = a.N;
+  const int K = topk_count(N, a.num, a.den);
+  const int j0 = rank * per;
+  const int j1 = min(N, j0 + per);
+  const int cnt = max(0, j1 - j0);
+  uint8_t* st = reinterpret_cast<uint8_t*>(sc + (size_t)G * SCS);
+  int32_t* out = a.idx + (size_t)bh * K;
+  const size_t bbase = (size_t)bh * CS * per;
+  const __nv_bfloat16* kb = a.k + (size_t)bh * N * D;
+
+  if (K >= N) {   // everything is selected (same branch in every CTA)
+    for (int i = tid; i < cnt; i += kCNT) out[j0 + i] = j0 + i;
+    return;
+  }
+
+  // ---- stream this CTA's K rows in rounds of kRoundKeys (two in flight)
+  const uint32_t full0 = smem_u32(&sh.full[0]);
+  const int nr = (cnt + kRoundKeys - 1) / kRoundKeys;
+  if (tid == 0) {
+    mbar_init(full0, 1);
+    mbar_init(full0 + 8, 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  auto issue = [&](int r) {   // thread 0 only
+    const int k0 = r * kRoundKeys, nk = min(kRoundKeys, cnt - k0);
+    const uint32_t bytes = (uint32_t)nk * D * 2;
+    const uint32_t bar = full0 + 8u * (uint32_t)(r & 1);
+    const uint32_t dst = ring + (uint32_t)((r & 1) * L::RB);
+    const char* src = reinterpret_cast<const char*>(kb + (size_t)(j0 + k0) * D);
+    mbar_arrive_expect_tx(bar, bytes);
+    for (uint32_t off = 0; off < bytes; off += 16384u) bulk_g2s(dst + off, src + off, min(16384u, bytes - off), bar);
+  };
+  if (tid == 0) {
+    if (nr > 0) issue(0);
+    if (nr > 1) issue(1);
+  }
+  // query rows: fp32 copy for the fp64 band, MMA B fragments in registers
+  // (lane (g, c) holds dims [32 s + 8 c, +8) of head g; heads >= G zero)
+  for (int e = tid; e < G * D; e += kCNT) {
+    const int gg = e / D, dd = e - gg * D;
+    qf[e] = __bfloat162float(a.q[(size_t)(b * a.Hq + h * G + gg) * D + dd]);
+  }
+  uint4 qb[KS];
+#pragma unroll
+  for (int s = 0; s < KS; ++s)
+    qb[s] = g < G ? *reinterpret_cast<const uint4*>(a.q + (size_t)(b * a.Hq + h * G + g) * D + 32 * s + 8 * c)
+                  : make_uint4(0, 0, 0, 0);
+  const float scale2 = kLog2e * rsqrtf((float)D);
+  float mx0 = -INFINITY, mx1 = -INFINITY;   // heads 2c, 2c+1
+  for (int r = 0; r < nr; ++r) {
+    if (!mbar_wait_bounded(full0 + 8u * (uint32_t)(r & 1), (uint32_t)((r >> 1) & 1))) raise_error(a.err, kErrTimeout);
+    const int k0 = r * kRoundKeys, nk = min(kRoundKeys, cnt - k0);
+    const uint32_t slot = ring + (uint32_t)((r & 1) * L::RB);
+    if (16 * warp < nk) {
+      // S^T for 16 keys: A = K rows g and g + 8 of the group (d-permuted
+      // 16-byte loads), B = q^T; k-step 2s+t takes dims 32s + 8c + 4t + {0..3}
+      const uint32_t row0 = slot + (uint32_t)((16 * warp + g) * D * 2 + 16 * c);
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int s = 0; s < KS; ++s) {
+        uint4 ka, kc;
+        asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];\n"
+                     : "=r"(ka.x), "=r"(ka.y), "=r"(ka.z), "=r"(ka.w)
+                     : "r"(row0 + 64 * s));
+        asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];\n"
+                     : "=r"(kc.x), "=r"(kc.y), "=r"(kc.z), "=r"(kc.w)
+                     : "r"(row0 + 8 * D * 2 + 64 * s));
+        const uint32_t a0[4] = {ka.x, kc.x, ka.y, kc.y};
+        const uint32_t a1[4] = {ka.z, kc.z, ka.w, kc.w};
+        mma_bf16_16816(acc, a0, qb[s].x, qb[s].y);
+        mma_bf16_16816(acc, a1, qb[s].z, qb[s].w);
+      }
+      const int i0 = k0 + 16 * warp + g, i1 = i0 + 8;   // local key indices
+      if (i0 < cnt) {
+        const float s0 = acc[0] * scale2, s1 = acc[1] * scale2;
+        if (2 * c < G) sc[(2 * c) * SCS + i0] = s0;
+        if (2 * c + 1 < G) sc[(2 * c + 1) * SCS + i0] = s1;
+        mx0 = fmaxf(mx0, s0);
+        mx1 = fmaxf(mx1, s1);
+      }
+      if (i1 < cnt) {
+        const float s0 = acc[2] * scale2, s1 = acc[3] * scale2;
+        if (2 * c < G) sc[(2 * c) * SCS + i1] = s0;
+        if (2 * c + 1 < G) sc[(2 * c + 1) * SCS + i1] = s1;
+        mx0 = fmaxf(mx0, s0);
+        mx1 = fmaxf(mx1, s1);
+      }
+    }
+    __syncthreads();   // every warp is done with this slot
+    if (tid == 0 && r + 2 < nr) {
+      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+      issue(r + 2);
+    }
+  }
+
+  // ---- softmax statistics of every head over the cluster: each CTA
+  // publishes its own (max, sum of exp2(s - max)); one exchange, partial sums
+  // rescaled to the cluster max in fp64
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+  }
+  if (g == 0) {
+    sh.wmax[warp][2 * c] = mx0;
+    sh.wmax[warp][2 * c + 1] = mx1;
+  }
+  __syncthreads();
+  float cm[8];
+#pragma unroll
+  for (int hh = 0; hh < 8; ++hh) {
+    cm[hh] = -INFINITY;
+    if (hh < G) {
+#pragma unroll
+      for (int w = 0; w < kWarpsC; ++w) cm[hh] = fmaxf(cm[hh], sh.wmax[w][hh]);
+    }
+  }
+  float ps[8];
+#pragma unroll
+  for (int hh = 0; hh < 8; ++hh) ps[hh] = 0.f;
+  for (int i = tid; i < cnt; i += kCNT) {
+#pragma unroll
+    for (int hh = 0; hh < 8; ++hh)
+      if (hh < G) {
+        const float e = exp2f(sc[hh * SCS + i] - cm[hh]);   // kept for the pooled scores
+        sc[hh * SCS + i] = e;
+        ps[hh] += e;
+      }
+  }
+#pragma unroll
+  for (int hh = 0; hh < 8; ++hh) {
+    if (hh < G) {
+      double d = ps[hh];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+      if (lane == 0) sh.wsum[warp][hh] = d;
+    }
+  }
+  __syncthreads();
+  if (tid < G) {
+    double s = 0.0;
+#pragma unroll
+    for (int w = 0; w < kWarpsC; ++w) s += sh.wsum[w][tid];
+#pragma unroll
+    for (int hh = 0; hh < 8; ++hh)
+      if (hh == tid) sh.cmax[hh] = cm[hh];
+    sh.csum[tid] = s;
+  }
   cluster.sync();
+  // warp hh (< G): lane r < CS takes CTA r's (max, sum) of head hh
+  if (warp < G) {
+    const float mr = lane < CS ? *cluster.map_shared_rank(&sh.cmax[warp], lane) : -INFINITY;
+    const double sr = lane < CS ? *cluster.map_shared_rank(&sh.csum[warp], lane) : 0.0;
+    float m = mr;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    double l = mr != -INFINITY ? sr * exp2((double)mr - (double)m) : 0.0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane == 0) {
+      sh.m2[warp] = m;
+      sh.l[warp] = l;
+      sh.inv_l[warp] = (float)(1.0 / l);
+      // pooled weight of this CTA's stored terms exp2(s - cm)
+      const float cmh = sh.cmax[warp];
+      sh.wpool[warp] = cmh == -INFINITY ? 0.f : (float)(exp2((double)cmh - (double)m) / l);
+    }
+  }
+  __syncthreads();
+
+  // ---- pooled scores, in place of head 0's scores
+  float* v = sc;
+  const float invG = 1.0f / (float)G;
+  float wh[8];
+#pragma unroll
+  for (int hh = 0; hh < 8; ++hh) wh[hh] = hh < G ? sh.wpool[hh] : 0.f;
+  for (int i = tid; i < cnt; i += kCNT) {
+    float acc = 0.f;
+#pragma unroll
+    for (int hh = 0; hh < 8; ++hh)
+      if (hh < G) acc += sc[hh * SCS + i] * wh[hh];
+    v[i] = acc * invG;
+  }
+  __syncthreads();
+  cluster_topk<CS>(cluster, sh, v, st, cnt, j0, rank, K, per, out, a.band_idx + bbase + (size_t)rank * per,
+                   a.band_val + bbase + (size_t)rank * per, a.band_idx + bbase, a.band_val + bbase, qf, kb, G, D);
+}
+
+int fused_per(int N, int cs) {
+  const int per = (N + cs - 1) / cs;
+  return (per + 63) / 64 * 64;
+}
+
+// How many clusters of `cs` CTAs of the fused kernel (one CTA per SM at
+// these shared-memory sizes) the current device runs at once; 0 if none.
+template <int CS, int D>
+int fused_active_clusters(size_t smem) {
+  if (cudaFuncSetAttribute(anchor_select_kernel<CS, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return 0;
+  if (CS > 8 &&
+      cudaFuncSetAttribute(anchor_select_kernel<CS, D>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+    return 0;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(CS, 1, 1);
+  cfg.blockDim = dim3(kCNT, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, anchor_select_kernel<CS, D>, &cfg) != cudaSuccess) n = 0;
+  return n;
+}
+
+// Cluster size of the fused kernel for this shape on the current device:
+// 16 when every (batch, kv head) cluster runs at once (one wave), else 8;
+// 0 when the scores do not fit on chip.
+template <int D>
+int fused_cluster_size(const SelArgs& a) {
+  static int cached[64][2] = {{0}};   // max active clusters of 16 and of 8 (+1; 0 = unknown)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  const size_t max_smem = 227 * 1024;
+  const size_t s16 = ASL<D>::bytes(a.G, fused_per(a.N, 16)), s8 = ASL<D>::bytes(a.G, fused_per(a.N, 8));
+  if (!cached[dev][0]) {
+    cached[dev][0] = 1 + fused_active_clusters<16, D>(max_smem);
+    cached[dev][1] = 1 + fused_active_clusters<8, D>(max_smem);
+    cudaGetLastError();
+  }
+  const int n16 = cached[dev][0] - 1, n8 = cached[dev][1] - 1;
+  const int problems = a.B * a.Hkv;
+  const bool ok16 = s16 <= max_smem && n16 > 0, ok8 = s8 <= max_smem && n8 > 0;
+  if (ok16 && (problems <= n16 || !ok8)) return 16;
+  if (ok8) return 8;
+  return ok16 ? 16 : 0;
+}
+
+template <int CS, int D>
+cudaError_t launch_fused(const SelArgs& a, cudaStream_t stream) {
+  const int per = fused_per(a.N, CS);
+  const size_t smem = ASL<D>::bytes(a.G, per);
+  cudaError_t e = cudaFuncSetAttribute(anchor_select_kernel<CS, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  if (CS > 8) {
+    e = cudaFuncSetAttribute(anchor_select_kernel<CS, D>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_ex(anchor_select_kernel<CS, D>, dim3(CS, a.B * a.Hkv), dim3(kCNT), smem, stream,
+                   (a.flags & 1) != 0, CS, a, per);
 }
 
 }  // namespace
 
-int select_decode_cluster_keys(int N) { return (N + kCS - 1) / kCS; }
+int select_decode_cluster_keys(int N) { return (N + kFallbackCS - 1) / kFallbackCS; }
 
 bool select_decode_cluster_ok(int N) { return select_decode_cluster_keys(N) <= 16384; }
 
 size_t select_decode_cluster_scratch(int B, int Hkv, int N) {
-  return (size_t)B * Hkv * kCS * select_decode_cluster_keys(N);
+  // band entries for the fallback layout and both fused cluster sizes
+  const size_t fb = (size_t)kFallbackCS * select_decode_cluster_keys(N);
+  const size_t f16 = (size_t)16 * fused_per(N, 16), f8 = (size_t)8 * fused_per(N, 8);
+  return (size_t)B * Hkv * (fb > f16 ? (fb > f8 ? fb : f8) : (f16 > f8 ? f16 : f8));
 }
 
 cudaError_t launch_select_decode_cluster(const SelArgs& a, cudaStream_t stream) {
@@ -363,8 +730,26 @@ cudaError_t launch_select_decode_cluster(const SelArgs& a, cudaStream_t stream) 
   cudaError_t e = cudaFuncSetAttribute(select_decode_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(kCS, a.B * a.Hkv);
+  dim3 grid(kFallbackCS, a.B * a.Hkv);
   return launch_ex(select_decode_cluster_kernel, grid, dim3(kCNT), smem, stream, (a.flags & 1) != 0, 1, a, per);
+}
+
+bool anchor_select_fused_ok(const SelArgs& a) {
+  if (a.G > 8 || !(a.D == 64 || a.D == 128)) return false;
+  return (a.D == 128 ? fused_cluster_size<128>(a) : fused_cluster_size<64>(a)) > 0;
+}
+
+cudaError_t launch_anchor_select_fused(const SelArgs& a, cudaStream_t stream) {
+  if (a.D == 128) {
+    const int cs = fused_cluster_size<128>(a);
+    if (cs == 16) return launch_fused<16, 128>(a, stream);
+    if (cs == 8) return launch_fused<8, 128>(a, stream);
+  } else {
+    const int cs = fused_cluster_size<64>(a);
+    if (cs == 16) return launch_fused<16, 64>(a, stream);
+    if (cs == 8) return launch_fused<8, 64>(a, stream);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace kascade
