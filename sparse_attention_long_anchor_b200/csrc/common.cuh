@@ -61,6 +61,16 @@ __host__ __device__ inline int64_t tile_pooled_offset(int64_t t, int tile) {
 // ---------------------------------------------------------------------------
 // bf16 helpers
 
+// 2^x as the single MUFU instruction ex2.approx.ftz.f32 (relative error
+// about 2^-22; subnormal results flush to zero).  For epilogues that are
+// bound by instruction issue; exp2f adds range handling around the same
+// instruction.
+__device__ __forceinline__ float ex2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

@@ -443,10 +443,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int c = 0; c < 32; c += 4) {
-            const float p0 = exp2f(fmaf(v[c], scale2, nm));
-            const float p1 = exp2f(fmaf(v[c + 1], scale2, nm));
-            const float p2 = exp2f(fmaf(v[c + 2], scale2, nm));
-            const float p3 = exp2f(fmaf(v[c + 3], scale2, nm));
+            const float p0 = ex2_fast(fmaf(v[c], scale2, nm));
+            const float p1 = ex2_fast(fmaf(v[c + 1], scale2, nm));
+            const float p2 = ex2_fast(fmaf(v[c + 2], scale2, nm));
+            const float p3 = ex2_fast(fmaf(v[c + 3], scale2, nm));
             ps[0] += p0;
             ps[1] += p1;
             ps[2] += p2;

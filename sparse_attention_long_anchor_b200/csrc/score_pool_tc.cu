@@ -266,8 +266,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             float p0 = 0.f, p1 = 0.f;
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
-              p0 += exp2f(fmaf(v[i], scale2, nm2));
-              p1 += exp2f(fmaf(v[i + 1], scale2, nm2));
+              p0 += ex2_fast(fmaf(v[i], scale2, nm2));
+              p1 += ex2_fast(fmaf(v[i + 1], scale2, nm2));
             }
             l += (double)(p0 + p1);
           }
@@ -322,10 +322,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int q4 = 0; q4 < 8; ++q4) {
             const float4 bb = bc[q4];
-            float e0 = exp2f(fmaf(v[q4 * 4 + 0], scale2, -bb.x));
-            float e1 = exp2f(fmaf(v[q4 * 4 + 1], scale2, -bb.y));
-            float e2 = exp2f(fmaf(v[q4 * 4 + 2], scale2, -bb.z));
-            float e3 = exp2f(fmaf(v[q4 * 4 + 3], scale2, -bb.w));
+            float e0 = ex2_fast(fmaf(v[q4 * 4 + 0], scale2, -bb.x));
+            float e1 = ex2_fast(fmaf(v[q4 * 4 + 1], scale2, -bb.y));
+            float e2 = ex2_fast(fmaf(v[q4 * 4 + 2], scale2, -bb.z));
+            float e3 = ex2_fast(fmaf(v[q4 * 4 + 3], scale2, -bb.w));
             if (diag) {
               const int4 pp = rp[q4];
               e0 = j <= pp.x ? e0 : 0.f;

@@ -578,7 +578,7 @@ __global__ void __launch_bounds__(kCNT, 1) anchor_select_kernel(const SelArgs a,
 #pragma unroll
     for (int hh = 0; hh < 8; ++hh)
       if (hh < G) {
-        const float e = exp2f(sc[hh * SCS + i] - cm[hh]);   // kept for the pooled scores
+        const float e = ex2_fast(sc[hh * SCS + i] - cm[hh]);   // kept for the pooled scores
         sc[hh * SCS + i] = e;
         ps[hh] += e;
       }
