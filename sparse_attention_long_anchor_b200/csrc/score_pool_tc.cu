@@ -17,7 +17,7 @@
 //               ring of kStages K blocks of 128 keys, 128-byte swizzled;
 //   warp 1      single-thread tcgen05.mma issue (M = N = 128, K = 16 steps);
 //               owns TMEM;
-//   warps 2..9  epilogue: two warpgroups take alternate K blocks (four
+//   warps 2..17 epilogue: four warpgroups take the K blocks in turn (four
 //               128-column TMEM accumulators); tcgen05.ld of one TMEM lane
 //               quarter per warp, online row statistics (pass 1, merged
 //               across the groups per tile), masked column sums (pass 2).
@@ -33,7 +33,7 @@ namespace {
 
 constexpr int kStages = 4;
 constexpr int kKB = 128;          // keys per block
-constexpr int kEpiGroups = 2;     // epilogue warpgroups, alternating K blocks
+constexpr int kEpiGroups = 4;     // epilogue warpgroups, taking K blocks in turn
 constexpr int kBufs = 4;          // TMEM accumulators of 128 columns
 constexpr int kThreads = 64 + 128 * kEpiGroups;
 constexpr int kErrTimeout = 2;
@@ -202,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // warpgroup wg takes the K blocks with block sequence number = wg (mod 2);
+    // warpgroup wg takes the K blocks with block sequence number = wg (mod kEpiGroups);
     // warp w reads TMEM lanes 32 (w % 4) .. +31
     const int ew = warp - 2;
     const int wg = ew >> 2;
@@ -237,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m2 = -INFINITY;  // running max of dot * scale2 (fp32)
       double l = 0.0;        // sum of exp2(dot * scale2 - m2)
       for (int blk = 0; blk < nb; ++blk, ++acount) {
-        if ((acount & 1) != wg) continue;
+        if (acount % kEpiGroups != wg) continue;
         const int buf = acount % kBufs;
         wait_acc(buf, (acount / kBufs) & 1);
         tc::fence_after();
@@ -276,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_empty0 + 8 * buf);
       }
-      // merge the two warpgroups' row statistics (after every reader of the
+      // merge the warpgroups' row statistics (after every reader of the
       // previous item's bcol / rpos is done)
       pm[wg * 128 + r] = m2;
       pl[wg * 128 + r] = l;
@@ -306,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv_rows = 1.0f / (float)(G * rows_t);
       float* pooled = a.pooled + (size_t)bh * (tile_pooled_offset(T - 1, a.tile) + a.N) + tile_pooled_offset(t, a.tile);
       for (int blk = 0; blk < nb; ++blk, ++acount) {
-        if ((acount & 1) != wg) continue;
+        if (acount % kEpiGroups != wg) continue;
         const int buf = acount % kBufs;
         wait_acc(buf, (acount / kBufs) & 1);
         tc::fence_after();
