@@ -394,7 +394,8 @@ def run_kascade(args, rank, world, local):
                   "anchor_select_us_per_anchor": sel_ms * 1e3 / n_anchor,
                   "anchor_scoring_bytes": anchor_score_bytes,
                   "anchor_select_GBps_on_K": anchor_score_bytes / (sel_ms * 1e-3 / n_anchor) / 1e9}
-    launches = n_anchor * 3 + (n_dec - n_anchor)
+    # kernels per step, as the library reports them for these shapes on this device
+    launches = n_anchor * (kc.launch_count(dec[3], kc.OP_SELECT) + 1) + (n_dec - n_anchor)
 
     prefill_obj = None
     if g_pre is not None:
@@ -419,7 +420,7 @@ def run_kascade(args, rank, world, local):
                                         "frac": gather / (pattn_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
                                         "tensor_tflops": sp_flops / (pattn_ms * 1e-3) / 1e12},
         }
-        launches += len(pcfg.anchors) * 3 + (pcfg.n_layers - len(pcfg.anchors))
+        launches += len(pcfg.anchors) * (kc.launch_count(pre[3], kc.OP_SELECT) + 1) + (pcfg.n_layers - len(pcfg.anchors))
 
     # ---- end to end through the public API: pinned host q -> device, step, outputs -> host
     cfg, plan, layers, shape, ws, idx, hms, outs = dec

@@ -111,6 +111,15 @@ typedef struct kascade_shape {
 /* Bytes of workspace that `op` needs for `shape` (0 on an invalid shape). */
 KASCADE_API size_t kascade_workspace_bytes(const kascade_shape* shape, int op);
 
+/* Number of kernels that `op` launches for `shape` on the current device
+ * (what a CUDA graph capturing the call will hold): KASCADE_OP_SELECT
+ * launches 1 for decode shapes whose scores fit on chip (fused scoring and
+ * selection in one cluster launch) and 2 otherwise (scoring, then
+ * selection); the attention ops launch 1.  Host-only query (it reads the
+ * device's cluster occupancy once).  Returns -1 on an invalid shape or op.
+ * The pages describe no such call; it exists for callers that size graphs. */
+KASCADE_API int kascade_launch_count(const kascade_shape* shape, int op);
+
 /* Number of int32 entries of the index buffer: B * Hkv * K (decode) or
  * B * Hkv * sum_t k_t (prefill).  Returns -1 on an invalid shape. */
 KASCADE_API int64_t kascade_index_count(const kascade_shape* shape);

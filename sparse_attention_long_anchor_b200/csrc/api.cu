@@ -214,6 +214,22 @@ int kascade_index_offsets(const kascade_shape* s, int64_t* offsets) {
   return KASCADE_OK;
 }
 
+int kascade_launch_count(const kascade_shape* s, int op) {
+  if (check_shape(s)) return -1;
+  if (op == KASCADE_OP_SPARSE_DECODE || op == KASCADE_OP_SPARSE_PREFILL || op == KASCADE_OP_DENSE) return 1;
+  if (op != KASCADE_OP_SELECT) return -1;
+  if (!is_decode(s)) return 2;
+  if (!select_decode_cluster_ok(s->kv_len)) return 2;
+  SelArgs a{};
+  a.B = s->batch;
+  a.Hq = s->num_q_heads;
+  a.Hkv = s->num_kv_heads;
+  a.G = a.Hq / a.Hkv;
+  a.D = s->head_dim;
+  a.N = s->kv_len;
+  return anchor_select_fused_ok(a) ? 1 : 2;
+}
+
 int kascade_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   if (!ws && ws_bytes) return KASCADE_ERR_WORKSPACE;
   if (!ws_bytes) return KASCADE_OK;

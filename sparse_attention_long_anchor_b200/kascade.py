@@ -14,7 +14,7 @@ import torch
 
 __all__ = ["Shape", "KascadeError", "lib", "OP_SELECT", "OP_SPARSE_DECODE", "OP_SPARSE_PREFILL",
            "OP_DENSE", "workspace_bytes", "index_count", "index_offsets", "Workspace", "select",
-           "sparse_decode", "sparse_prefill", "dense_ref", "status_str", "EXPORTS", "LIB_PATH"]
+           "sparse_decode", "sparse_prefill", "dense_ref", "status_str", "launch_count", "EXPORTS", "LIB_PATH"]
 
 LIB_PATH = os.environ.get("KASCADE_LIB") or os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkascade.so")
 
@@ -25,7 +25,8 @@ FLAG_PDL, FLAG_INPUTS_STABLE = 1, 2
 EXPORTS = ("kascade_workspace_bytes", "kascade_index_count", "kascade_index_offsets",
            "kascade_workspace_init", "kascade_select", "kascade_sparse_decode",
            "kascade_sparse_prefill", "kascade_dense_ref", "kascade_workspace_error",
-           "kascade_status_str", "kascade_select_decode_static", "kascade_select_decode_static_max_bytes")
+           "kascade_status_str", "kascade_select_decode_static", "kascade_select_decode_static_max_bytes",
+           "kascade_launch_count")
 
 
 class KascadeError(RuntimeError):
@@ -82,6 +83,8 @@ def _load():
     so.kascade_select_decode_static.restype = ctypes.c_int
     so.kascade_select_decode_static_max_bytes.argtypes = []
     so.kascade_select_decode_static_max_bytes.restype = ctypes.c_size_t
+    so.kascade_launch_count.argtypes = [SP, ctypes.c_int]
+    so.kascade_launch_count.restype = ctypes.c_int
     so.kascade_status_str.argtypes = [ctypes.c_int]
     so.kascade_status_str.restype = ctypes.c_char_p
     return so
@@ -92,6 +95,14 @@ lib = _load()
 
 def status_str(status: int) -> str:
     return lib.kascade_status_str(status).decode()
+
+
+def launch_count(shape: "Shape", op: int) -> int:
+    """Kernels that `op` launches for `shape` on the current device."""
+    n = lib.kascade_launch_count(ctypes.byref(shape), op)
+    if n < 0:
+        raise KascadeError(ERR_INVALID_ARG, "kascade_launch_count")
+    return n
 
 
 def _check(status: int, where: str):
