@@ -9,27 +9,25 @@
 //
 // Work item = (query tile, row block, batch x kv head): 128 MMA rows = 4
 // query heads x 32 queries (rows of absent heads are zero and never stored).
-// Persistent CTAs take items head by head, longest tile first.  Per CTA:
-//   warps 0..7  softmax, two warpgroups splitting the columns: one TMEM
-//               lane (= one query row) per thread of each group; reads S
-//               with tcgen05.ld, applies the causal mask by original key
-//               index, keeps the running max and sum, writes P (bf16) into
-//               TMEM as the A operand of the second product, and
-//               finally reads O, normalises and stores it.  The running max
-//               used for the exponent is raised (and O, l rescaled in TMEM)
-//               only when a row's max grows by more than 2^8, which keeps
-//               the result exact and P within bf16 range;
-//   warps 8..11 gather: 64 selected K and V rows per block, 16-byte
-//               cp.async into 128-byte-swizzled shared memory, a ring of
-//               kStages blocks, completion tracked per thread on the stage's
-//               mbarrier; one thread also issues the TMA loads of the item's
-//               Q tile (double-buffered);
-//   warp 12     single-thread tcgen05.mma issue (whichever product is
-//               ready first) and TMEM owner:
-//               S = Q K^T (M = 128, N = 64, into one of two TMEM buffers),
-//               O += P V (M = 128, N = d, P from TMEM, V as an MN-major
-//               shared-memory operand, into
-//               one of two TMEM output buffers, one per item in flight).
+// Persistent CTAs take items head by head, longest tile first.  Each CTA
+// runs two independent pipelines ("subs") on alternate items of its share,
+// so that one pipeline's softmax overlaps the other's products and gathers.
+// Per pipeline:
+//   4 softmax warps   one TMEM lane (= one query row) per thread: read S
+//                     with tcgen05.ld, mask causally by original key index,
+//                     keep the running max and sum, write P (bf16) into TMEM
+//                     as the A operand of the second product; finally read
+//                     O, normalise and store it.  The running max used for
+//                     the exponent is raised (and O, l rescaled in TMEM) only
+//                     when a row's max grows by more than 2^8, which keeps
+//                     the result exact and P within bf16 range;
+//   2 gather warps    64 selected K and V rows per block, 16-byte cp.async
+//                     into 128-byte-swizzled shared memory (kStages blocks),
+//                     completion tracked per thread on the stage's mbarrier;
+//                     one thread also TMA-loads the item's Q tile;
+//   1 MMA thread      tcgen05.mma by readiness: S = Q K^T (M = 128, N = 64)
+//                     and O += P V (M = 128, N = d, P from TMEM, V an MN-major
+//                     shared-memory operand).
 // All hand-offs are mbarriers; every wait is bounded and a timeout stops the
 // CTA's waits and records an error code in the workspace error word.
 #include "common.cuh"
@@ -41,15 +39,16 @@ namespace kascade {
 namespace {
 
 constexpr int kKB = 64;          // keys per block
-constexpr int kStages = 5;       // K/V ring; >= 3 keeps the MMA issue order deadlock-free
-constexpr int kThreads = 416;    // 8 softmax warps, 4 gather warps, 1 MMA warp
-constexpr int kGather0 = 256;    // first gather thread
-constexpr int kMmaWarp = 12;
+constexpr int kSubs = 2;         // independent pipelines per CTA
+constexpr int kStages = 2;       // K/V blocks in flight per pipeline
+constexpr int kGather = 64;      // gather threads per pipeline
+constexpr int kThreads = 448;    // 8 softmax warps, 4 gather warps, 2 MMA warps
 constexpr int kErrTimeout = 4;
 constexpr float kRescale = 8.0f; // log2 growth of a row max that forces a rescale
 constexpr int kNoKey = 0x7fffffff;
-// TMEM columns: S[2] (kKB each), O[2] (128 each), P[2] (kKB / 2 each, bf16 pairs)
-constexpr uint32_t kColS = 0, kColO = 128, kColP = 384;
+// TMEM columns of pipeline `sub` start at 256 sub: S (kKB), P (kKB / 2, bf16
+// pairs), O (128)
+constexpr uint32_t kColS = 0, kColP = 64, kColO = 128;
 
 template <int D>
 struct PAL {
@@ -57,25 +56,22 @@ struct PAL {
   static constexpr int QCB = 128 * 128;             // one 64-column block of the Q tile
   static constexpr int KB = kKB * D * 2;            // K (or V) of one block
   static constexpr int KVCB = kKB * 128;            // one 64-column block of K (or V)
-  static constexpr size_t q = 0;                     // [2] Q
-  static constexpr size_t kv = q + 2 * (size_t)QB;   // [S] K then V
-  static constexpr size_t bars = kv + (size_t)kStages * 2 * KB;
-  static constexpr int NBARS = 4 + 2 * kStages + 12 + 1;
-  static constexpr size_t xch = bars + NBARS * 8;     // [2][128] f32 row maxima / sums of the two softmax groups
-  static constexpr size_t tslot = xch + 2 * 128 * 4;
+  static constexpr size_t SUB = (size_t)QB + (size_t)kStages * 2 * KB;   // Q then the K/V stages
+  static constexpr size_t bars = kSubs * SUB;
+  static constexpr int NBARS = 10 + 2 * kStages;    // per pipeline
+  static constexpr size_t tslot = bars + (size_t)kSubs * NBARS * 8;
   static constexpr size_t stop = tslot + 8;
   static constexpr size_t total = stop + 8;
   static constexpr size_t alloc = total + 1024;      // slack for 1024-byte alignment
-  static_assert(kv % 1024 == 0 && KB % 1024 == 0, "swizzled tiles");
+  static_assert(SUB % 1024 == 0 && QB % 1024 == 0 && KB % 1024 == 0, "swizzled tiles");
   static_assert(bars % 8 == 0, "mbarrier alignment");
   static_assert(alloc <= 232448, "more than 227 KB of shared memory per block");
 };
 
-// barrier slots
-constexpr int bQFull = 0, bQEmpty = 2, bKVFull = 4, bKVEmpty = 4 + kStages, bSFull = 4 + 2 * kStages,
-              bSEmpty = bSFull + 2, bPFull = bSEmpty + 2, bPEmpty = bPFull + 2, bODone = bPEmpty + 2,
-              bOEmpty = bODone + 2, bDrain = bOEmpty + 2;
-static_assert(bDrain + 1 == PAL<128>::NBARS, "barrier count");
+// barrier slots of one pipeline
+constexpr int bQFull = 0, bQEmpty = 1, bSFull = 2, bSEmpty = 3, bPFull = 4, bPEmpty = 5, bODone = 6, bOEmpty = 7,
+              bDrain = 8, bKVFull = 10, bKVEmpty = 10 + kStages;
+static_assert(bKVEmpty + kStages == PAL<128>::NBARS, "barrier count");
 
 // One work item: which rows, which key list.
 struct Item {
@@ -113,7 +109,6 @@ __device__ __forceinline__ Item item_of(const AttnArgs& a, int it, int T, int RB
 
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
 
-
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const AttnArgs a, int RB) {
@@ -123,54 +118,59 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   char* sm = smem_raw + (base - raw);
-  const uint32_t q_s = base + (uint32_t)L::q, kv_s = base + (uint32_t)L::kv;
-  const uint32_t bar0 = base + (uint32_t)L::bars;
-  auto bar = [&](int slot) { return bar0 + 8u * (uint32_t)slot; };
   volatile int* stop = reinterpret_cast<volatile int*>(sm + L::stop);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // roles: warps 0-3 / 4-7 softmax of pipeline 0 / 1, warps 8-9 / 10-11
+  // gather, warps 12 / 13 MMA issue (warp 12 also owns TMEM)
+  const int sub = warp < 8 ? warp >> 2 : (warp < 12 ? (warp - 8) >> 1 : warp - 12);
+  const uint32_t q_s = base + (uint32_t)(sub * L::SUB), kv_s = q_s + (uint32_t)L::QB;
+  const uint32_t bar0 = base + (uint32_t)(L::bars + (size_t)sub * L::NBARS * 8);
+  auto bar = [&](int slot) { return bar0 + 8u * (uint32_t)slot; };
   const int G = a.G;
   const int T = (a.N + a.tile - 1) / a.tile;
   const int items = T * RB * a.B * a.Hkv;
   const bool causal = a.idx != nullptr || a.causal;
   const int heads_rb = min(4, G);   // query heads per row block
+  // this pipeline's items: the CTA's share, alternating between pipelines
+  const int it0 = blockIdx.x + sub * gridDim.x, istep = kSubs * gridDim.x;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(bQFull + i), 1);
-      mbar_init(bar(bQEmpty + i), 1);
-      mbar_init(bar(bSFull + i), 1);
-      mbar_init(bar(bSEmpty + i), 8);
-      mbar_init(bar(bPFull + i), 8);
-      mbar_init(bar(bPEmpty + i), 1);
-      mbar_init(bar(bODone + i), 1);
-      mbar_init(bar(bOEmpty + i), 8);
+    for (int p = 0; p < kSubs; ++p) {
+      const uint32_t b0 = base + (uint32_t)(L::bars + (size_t)p * L::NBARS * 8);
+      mbar_init(b0 + 8 * bQFull, 1);
+      mbar_init(b0 + 8 * bQEmpty, 1);
+      mbar_init(b0 + 8 * bSFull, 1);
+      mbar_init(b0 + 8 * bSEmpty, 4);
+      mbar_init(b0 + 8 * bPFull, 4);
+      mbar_init(b0 + 8 * bPEmpty, 1);
+      mbar_init(b0 + 8 * bODone, 1);
+      mbar_init(b0 + 8 * bOEmpty, 4);
+      mbar_init(b0 + 8 * bDrain, 1);
+      for (int s = 0; s < kStages; ++s) {
+        mbar_init(b0 + 8 * (bKVFull + s), kGather);
+        mbar_init(b0 + 8 * (bKVEmpty + s), 1);
+      }
     }
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar(bKVFull + s), 128);
-      mbar_init(bar(bKVEmpty + s), 1);
-    }
-    mbar_init(bar(bDrain), 1);
     *stop = 0;
     mbar_fence_init();
   }
-  // rows of absent heads (G < 4) stay zero in both Q buffers
-  for (int i = threadIdx.x; i < 2 * CB * (4 - heads_rb) * 32 * 8; i += kThreads) {
-    const int per_buf = CB * (4 - heads_rb) * 32 * 8;
-    const int qb = i / per_buf, rem0 = i - qb * per_buf;
+  // rows of absent heads (G < 4) stay zero in both pipelines' Q tiles
+  for (int i = threadIdx.x; i < kSubs * CB * (4 - heads_rb) * 32 * 8; i += kThreads) {
+    const int per_sub = CB * (4 - heads_rb) * 32 * 8;
+    const int p = i / per_sub, rem0 = i - p * per_sub;
     const int cb = rem0 / ((4 - heads_rb) * 32 * 8), rem = rem0 - cb * (4 - heads_rb) * 32 * 8;
     const int r = 32 * heads_rb + rem / 8, ch = rem % 8;
-    *reinterpret_cast<uint4*>(sm + L::q + (size_t)qb * L::QB + cb * L::QCB + r * 128 + ch * 16) =
-        make_uint4(0, 0, 0, 0);
+    *reinterpret_cast<uint4*>(sm + (size_t)p * L::SUB + cb * L::QCB + r * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
   }
   fence_async_smem();
-  if (warp == kMmaWarp) tc::tmem_alloc(base + (uint32_t)L::tslot, 512);
+  if (warp == 12) tc::tmem_alloc(base + (uint32_t)L::tslot, 512);
   pdl_wait();
   pdl_launch_dependents();
   tc::fence_before();
   __syncthreads();
   tc::fence_after();
-  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + L::tslot);
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + L::tslot) + (uint32_t)(256 * sub);
 
   // bounded wait; after a timeout every later wait is skipped so that all
   // loops run to their (finite) ends
@@ -182,15 +182,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   };
 
-  if (warp >= 8 && warp < kMmaWarp) {
+  if (warp >= 8 && warp < 12) {
     // ------------------------------------------------------------ gather
     // thread -> 16-byte chunk c of rows r0, r0 + RPP, ...: one warp
     // instruction copies whole 256-byte rows.  The key indices of the next
     // block are loaded one block ahead, and every thread arrives on the
     // stage's barrier asynchronously when its copies land, so the gather
     // only ever waits for a free stage.
-    constexpr int CH = D / 8, RPP = 128 / CH, KR = kKB / RPP;
-    const int pt = threadIdx.x - kGather0;
+    constexpr int CH = D / 8, RPP = kGather / CH, KR = kKB / RPP;
+    const int pt = threadIdx.x - 256 - kGather * sub;
     const int c = pt % CH, r0 = pt / CH;
     const int cb = c >> 3, cc = c & 7;
     auto load_keys = [&](const Item& I, int j, int (&kk)[KR]) {
@@ -203,31 +203,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     int cur[KR], nxt[KR];
     int pf_it = -1, pf_j = 0;   // block whose keys sit in cur
     int n = 0, qn = 0;
-    if (blockIdx.x < items) {
-      const Item I0 = item_of(a, blockIdx.x, T, RB);
+    if (it0 < items) {
+      const Item I0 = item_of(a, it0, T, RB);
       if (I0.nb > 0) {
         load_keys(I0, 0, cur);
-        pf_it = blockIdx.x;
+        pf_it = it0;
       }
     }
-    for (int it = blockIdx.x; it < items; it += gridDim.x, ++qn) {
+    for (int it = it0; it < items; it += istep, ++qn) {
       const Item I = item_of(a, it, T, RB);
-      const int it2 = it + gridDim.x;
+      const int it2 = it + istep;
       const Item I2 = item_of(a, it2 < items ? it2 : it, T, RB);
       const bool have2 = it2 < items && I2.nb > 0;
       if (pt == 0) {
-        const int qb = qn & 1;
-        if (qn >= 2) wait(bQEmpty + qb, (qn >> 1) - 1);
-        mbar_arrive_expect_tx(bar(bQFull + qb), (uint32_t)(CB * heads_rb * 32 * 128));
+        if (qn >= 1) wait(bQEmpty, qn - 1);
+        mbar_arrive_expect_tx(bar(bQFull), (uint32_t)(CB * heads_rb * 32 * 128));
         for (int b = 0; b < CB; ++b)
           for (int g = 0; g < heads_rb; ++g)
-            tc::tma_load_3d(q_s + qb * L::QB + b * L::QCB + g * 4096, &mq, b * 64, I.i0,
-                            I.b * a.Hq + I.hq0 + g, bar(bQFull + qb));
+            tc::tma_load_3d(q_s + b * L::QCB + g * 4096, &mq, b * 64, I.i0, I.b * a.Hq + I.hq0 + g, bar(bQFull));
       }
       const size_t bhoff = (size_t)(I.b * a.Hkv + I.h) * a.N * D;
       for (int j = 0; j < I.nb; ++j, ++n) {
         if (pf_it != it || pf_j != j) load_keys(I, j, cur);   // not prefetched (rare)
-        // keys of the following block
         int nx_it = -1, nx_j = 0;
         if (j + 1 < I.nb) {
           load_keys(I, j + 1, nxt);
@@ -259,69 +256,63 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     asm volatile("cp.async.wait_all;\n" ::: "memory");
     // no TMA copy may still be in flight when the CTA exits
-    if (pt == 0 && qn > 0 && !mbar_wait_bounded(bar(bQFull + ((qn - 1) & 1)), ((qn - 1) >> 1) & 1))
-      raise_error(a.err, kErrTimeout);
-  } else if (warp == kMmaWarp) {
+    if (pt == 0 && qn > 0 && !mbar_wait_bounded(bar(bQFull), (qn - 1) & 1)) raise_error(a.err, kErrTimeout);
+  } else if (warp >= 12) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
       const uint32_t id1 = tc::idesc_bf16_f32(128, kKB);
       const uint32_t id2 = tc::idesc_bf16_f32_bmn(128, D);
       int n = 0, qn = 0;
-      for (int it = blockIdx.x; it < items; it += gridDim.x, ++qn) {
+      for (int it = it0; it < items; it += istep, ++qn) {
         const Item I = item_of(a, it, T, RB);
-        const int qb = qn & 1, ob = qn & 1;
-        wait(bQFull + qb, qn >> 1);
+        wait(bQFull, qn);
         tc::fence_after();
-        auto mma1 = [&](int m) {   // S[m & 1] = Q K_m^T
-          const int s = m % kStages, sb = m & 1;
-          fence_async_smem();   // K / V arrived by cp.async
+        auto mma1 = [&](int m) {   // S = Q K_m^T
+          const int s = m % kStages;
           tc::fence_after();
-          const uint32_t d = tmem + kColS + (uint32_t)(sb * kKB);
           const uint32_t ks = kv_s + (uint32_t)(s * 2 * L::KB);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t qoff = (uint32_t)((kk >> 2) * L::QCB + (kk & 3) * 32);
             const uint32_t koff = (uint32_t)((kk >> 2) * L::KVCB + (kk & 3) * 32);
-            tc::mma_bf16(d, tc::smem_desc_sw128(q_s + qb * L::QB + qoff), tc::smem_desc_sw128(ks + koff), id1,
-                         kk > 0);
+            tc::mma_bf16(tmem + kColS, tc::smem_desc_sw128(q_s + qoff), tc::smem_desc_sw128(ks + koff), id1, kk > 0);
           }
-          tc::commit(bar(bSFull + sb));
+          tc::commit(bar(bSFull));
         };
-        auto mma2 = [&](int m, int j) {   // O[ob] += P[m & 1] V_m, P from TMEM
-          const int s = m % kStages, pb = m & 1;
+        auto mma2 = [&](int m, int j) {   // O += P V_m, P from TMEM
+          const int s = m % kStages;
           tc::fence_after();
-          const uint32_t d = tmem + kColO + (uint32_t)(ob * 128);
-          const uint32_t pa = tmem + kColP + (uint32_t)(pb * (kKB / 2));
           const uint32_t vs = kv_s + (uint32_t)(s * 2 * L::KB + L::KB);
 #pragma unroll
           for (int kk = 0; kk < kKB / 16; ++kk)
-            tc::mma_bf16_ts(d, pa + (uint32_t)(kk * 8), tc::smem_desc_sw128_mn(vs + kk * 2048, L::KVCB), id2,
-                            (j > 0 || kk > 0) ? 1u : 0u);
+            tc::mma_bf16_ts(tmem + kColO, tmem + kColP + (uint32_t)(kk * 8),
+                            tc::smem_desc_sw128_mn(vs + kk * 2048, L::KVCB), id2, (j > 0 || kk > 0) ? 1u : 0u);
           tc::commit(bar(bKVEmpty + s));
-          tc::commit(bar(bPEmpty + pb));
-          tc::commit(bar(bODone + ob));
+          tc::commit(bar(bPEmpty));
+          tc::commit(bar(bODone));
         };
-        // issue whichever product is ready: S of a later block (up to two
-        // ahead of P V) or P V of the oldest block whose P is published
+        // issue whichever product is ready: P V of the oldest published
+        // block, else S of the next block (at most one ahead: S and P are
+        // single buffers)
         int i1 = 0, i2 = 0;
         long long t_last = clock64();
         while (i2 < I.nb && !*stop) {
           bool did = false;
-          if (i1 < I.nb && i1 <= i2 + 2) {
-            const int m = n + i1;
-            if (mbar_test(bar(bKVFull + m % kStages), (uint32_t)((m / kStages) & 1)) &&
-                (m < 2 || mbar_test(bar(bSEmpty + (m & 1)), (uint32_t)(((m >> 1) - 1) & 1)))) {
-              mma1(m);
-              ++i1;
+          if (i2 < i1) {
+            const int m = n + i2;
+            if (mbar_test(bar(bPFull), (uint32_t)(m & 1)) &&
+                (i2 > 0 || qn < 1 || mbar_test(bar(bOEmpty), (uint32_t)((qn - 1) & 1)))) {
+              mma2(m, i2);
+              ++i2;
               did = true;
             }
           }
-          if (!did && i2 < i1) {
-            const int m = n + i2;
-            if (mbar_test(bar(bPFull + (m & 1)), (uint32_t)((m >> 1) & 1)) &&
-                (i2 > 0 || qn < 2 || mbar_test(bar(bOEmpty + ob), (uint32_t)(((qn >> 1) - 1) & 1)))) {
-              mma2(m, i2);
-              ++i2;
+          if (!did && i1 < I.nb && i1 <= i2 + 1) {
+            const int m = n + i1;
+            if (mbar_test(bar(bKVFull + m % kStages), (uint32_t)((m / kStages) & 1)) &&
+                (m < 1 || mbar_test(bar(bSEmpty), (uint32_t)((m - 1) & 1)))) {
+              mma1(m);
+              ++i1;
               did = true;
             }
           }
@@ -332,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             raise_error(a.err, kErrTimeout);
           }
         }
-        tc::commit(bar(bQEmpty + qb));
+        tc::commit(bar(bQEmpty));
         n += I.nb;
       }
       // every issued MMA completes before TMEM is released
@@ -341,21 +332,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax
-    // two warpgroups share every row: group wg takes S columns
-    // [32 wg, 32 wg + 32) of each block and O columns [wg D/2, (wg+1) D/2);
-    // they exchange row maxima (and at the end row sums) through shared
-    // memory at a named barrier
-    const int wg = warp >> 2;
     const int r = threadIdx.x & 127;                  // TMEM lane = MMA row
     const uint32_t lane_addr = (uint32_t)(32 * (warp & 3)) << 16;
     const float scale2 = kLog2e * rsqrtf((float)D);
-    float* xch = reinterpret_cast<float*>(sm + L::xch);   // [2 groups][128]
-    constexpr int OC = D / 2;                             // O columns per group
     int n = 0, qn = 0;
-    int ocnt[2] = {0, 0};                             // completed MMA2 groups per O buffer
-    for (int it = blockIdx.x; it < items; it += gridDim.x, ++qn) {
+    int ocnt = 0;                                     // completed MMA2 groups of this pipeline
+    for (int it = it0; it < items; it += istep, ++qn) {
       const Item I = item_of(a, it, T, RB);
-      const int ob = qn & 1;
       const int g = r >> 5, qi = r & 31;
       const int pos = I.i0 + qi;
       const bool valid = g < heads_rb && qi < I.rows_t;
@@ -368,7 +351,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       int last_next = I.nb > 0 ? last_key(0) : 0;
       for (int j = 0; j < I.nb; ++j) {
         const int m = n + j;
-        const int sb = m & 1, pb = m & 1;
         // the block needs a per-key check if it holds keys past the list
         // end or (causal) keys after the tile start
         const int pos0 = j * kKB;
@@ -376,34 +358,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int last = last_next;
         if (j + 1 < I.nb) last_next = last_key(j + 1);
         const bool check = tail || (causal && last > I.i0);
-        wait(bSFull + sb, m >> 1);
+        wait(bSFull, m);
         tc::fence_after();
-        float v[32];
-        tc::tmem_ld32(tmem + lane_addr + kColS + (uint32_t)(sb * kKB + 32 * wg), v);
+        float v[kKB];
+        tc::tmem_ld32(tmem + lane_addr + kColS, *reinterpret_cast<float(*)[32]>(v));
+        tc::tmem_ld32(tmem + lane_addr + kColS + 32, *reinterpret_cast<float(*)[32]>(v + 32));
         tc::fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(bSEmpty + sb));
+        if (lane == 0) mbar_arrive(bar(bSEmpty));
         if (check) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int q = pos0 + 32 * wg + c;
+          for (int c = 0; c < kKB; ++c) {
+            const int q = pos0 + c;
             const int key = q < I.list_len ? (I.list ? __ldg(I.list + q) : q) : kNoKey;
             if (key == kNoKey || (causal && key > pos)) v[c] = -INFINITY;
           }
         }
         float mx4[4] = {v[0], v[1], v[2], v[3]};
 #pragma unroll
-        for (int c = 4; c < 32; c += 4) {
+        for (int c = 4; c < kKB; c += 4) {
           mx4[0] = fmaxf(mx4[0], v[c]);
           mx4[1] = fmaxf(mx4[1], v[c + 1]);
           mx4[2] = fmaxf(mx4[2], v[c + 2]);
           mx4[3] = fmaxf(mx4[3], v[c + 3]);
         }
-        const float mine = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-        xch[wg * 128 + r] = mine;
-        asm volatile("bar.sync 1, 256;\n" ::: "memory");
-        const float mx2 = fmaxf(mine, xch[(wg ^ 1) * 128 + r]) * scale2;   // scale > 0 keeps the order
-        asm volatile("bar.sync 1, 256;\n" ::: "memory");   // xch is rewritten next
+        const float mx2 = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * scale2;   // scale > 0 keeps the order
         float m_new = m_used;
         bool resc = false;
         if (mx2 > m_used) {
@@ -415,15 +394,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (__any_sync(0xffffffffu, resc)) {
-          // rescale this group's half of O (and l) once the previous
-          // block's P V has landed
-          wait(bODone + ob, ocnt[ob] + j - 1);
+          // rescale O (and l) once the previous block's P V has landed
+          wait(bODone, ocnt + j - 1);
           tc::fence_after();
           const float alpha = resc ? exp2f(m_used - m_new) : 1.0f;
 #pragma unroll 1
-          for (int c32 = 0; c32 < OC / 32; ++c32) {
+          for (int c32 = 0; c32 < D / 32; ++c32) {
             float o[32];
-            const uint32_t ta = tmem + lane_addr + kColO + (uint32_t)(ob * 128 + wg * OC + c32 * 32);
+            const uint32_t ta = tmem + lane_addr + kColO + (uint32_t)(c32 * 32);
             tc::tmem_ld32(ta, o);
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] *= alpha;
@@ -432,17 +410,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           l *= alpha;
         }
         m_used = m_new;
-        // P = exp2(s * scale2 - m_used) in bf16: this group's 32 columns of
-        // row r of the block's A tile
-        uint32_t pk[16];
+        // P = exp2(s * scale2 - m_used) in bf16, row r of the block's A tile
+        uint32_t pk[kKB / 2];
         if (m_used == -INFINITY) {
 #pragma unroll
-          for (int c = 0; c < 16; ++c) pk[c] = 0u;
+          for (int c = 0; c < kKB / 2; ++c) pk[c] = 0u;
         } else {
           const float nm = -m_used;
           float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int c = 0; c < 32; c += 4) {
+          for (int c = 0; c < kKB; c += 4) {
             const float p0 = ex2_fast(fmaf(v[c], scale2, nm));
             const float p1 = ex2_fast(fmaf(v[c + 1], scale2, nm));
             const float p2 = ex2_fast(fmaf(v[c + 2], scale2, nm));
@@ -456,30 +433,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
         }
-        if (m >= 2) wait(bPEmpty + pb, (m >> 1) - 1);
-        // this group's 16 columns of P (bf16 pairs) in TMEM, row r
-        tc::tmem_st16(tmem + lane_addr + kColP + (uint32_t)(pb * (kKB / 2) + 16 * wg), pk);
+        if (m >= 1) wait(bPEmpty, m - 1);
+        tc::tmem_st16(tmem + lane_addr + kColP, *reinterpret_cast<uint32_t(*)[16]>(pk));
+        tc::tmem_st16(tmem + lane_addr + kColP + 16, *reinterpret_cast<uint32_t(*)[16]>(pk + 16));
         tc::fence_before();   // orders the P store and a TMEM rescale of O before the next P V
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(bPFull + pb));
+        if (lane == 0) mbar_arrive(bar(bPFull));
       }
-      // ---- output rows: O / l, bf16 (row sums of both groups)
-      xch[wg * 128 + r] = l;
-      asm volatile("bar.sync 1, 256;\n" ::: "memory");
-      const float lt = l + xch[(wg ^ 1) * 128 + r];
-      asm volatile("bar.sync 1, 256;\n" ::: "memory");   // xch is rewritten next
+      // ---- output rows: O / l, bf16
       if (I.nb > 0) {
-        wait(bODone + ob, ocnt[ob] + I.nb - 1);
+        wait(bODone, ocnt + I.nb - 1);
         tc::fence_after();
       }
-      ocnt[ob] += I.nb;
-      const float inv = lt > 0.f ? 1.0f / lt : 0.0f;
-      __nv_bfloat16* orow = a.o + ((size_t)(I.b * a.Hq + I.hq0 + g) * a.N + pos) * D + wg * OC;
+      ocnt += I.nb;
+      const float inv = l > 0.f ? 1.0f / l : 0.0f;
+      __nv_bfloat16* orow = a.o + ((size_t)(I.b * a.Hq + I.hq0 + g) * a.N + pos) * D;
 #pragma unroll 1
-      for (int c32 = 0; c32 < OC / 32; ++c32) {
+      for (int c32 = 0; c32 < D / 32; ++c32) {
         float o[32];
         if (I.nb > 0) {
-          tc::tmem_ld32(tmem + lane_addr + kColO + (uint32_t)(ob * 128 + wg * OC + c32 * 32), o);
+          tc::tmem_ld32(tmem + lane_addr + kColO + (uint32_t)(c32 * 32), o);
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = 0.f;
@@ -496,12 +469,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (valid && wg == 0 && a.lse)
-        a.lse[(size_t)(I.b * a.Hq + I.hq0 + g) * a.N + pos] =
-            lt > 0.f ? (m_used + log2f(lt)) * (float)kLn2 : -INFINITY;
+      if (valid && a.lse)
+        a.lse[(size_t)(I.b * a.Hq + I.hq0 + g) * a.N + pos] = l > 0.f ? (m_used + log2f(l)) * (float)kLn2 : -INFINITY;
       tc::fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(bOEmpty + ob));
+      if (lane == 0) mbar_arrive(bar(bOEmpty));
       n += I.nb;
     }
   }
@@ -509,9 +481,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ------------------------------------------------------------ teardown
   tc::fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == 12) {
     tc::fence_after();
-    tc::tmem_dealloc(tmem, 512);
+    tc::tmem_dealloc(*reinterpret_cast<volatile uint32_t*>(sm + L::tslot), 512);
   }
 }
 
@@ -527,7 +499,8 @@ cudaError_t launch_prefill_attn_tc(const AttnArgs& a, int num_sms, cudaStream_t 
   const int T = (a.N + a.tile - 1) / a.tile;
   const int RB = a.G <= 4 ? 1 : a.G / 4;
   const long items = (long)T * RB * a.B * a.Hkv;
-  const int grid = (int)(items < num_sms ? items : num_sms);
+  const long long ctas = (items + kSubs - 1) / kSubs;
+  const int grid = (int)(ctas < num_sms ? ctas : num_sms);
   const bool pdl = (a.flags & 1) != 0;
   if (a.D == 128) {
     cudaError_t e = cudaFuncSetAttribute(prefill_attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
