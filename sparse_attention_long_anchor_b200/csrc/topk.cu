@@ -26,11 +26,11 @@ namespace kascade {
 
 namespace {
 
-constexpr int kSelThreads = 1024;
+constexpr int kSelThreads = 256;
+constexpr int kSelCtasPerSM = 4;   // problems in flight per SM
 constexpr int kBins = 2048;
 constexpr float kBandDelta = 1.0f / 8192.0f;
 constexpr float kBandFloor = 0x1p-96f;   // below this fp32 exp2 underflow may hide mass
-constexpr int kMaxRows = 256;             // G * tile rows of one prefill problem
 constexpr int kMaxD = 128;
 
 struct SelShared {
@@ -46,12 +46,12 @@ struct SelShared {
   double b_val[kSelThreads];
 };
 
-// dynamic shared memory after SelShared (rounded up to 128 bytes so that the
-// 16-byte vector stores into the q tile are aligned): decode q rows as float
-// [8][D]; prefill q tile as bf16 [kMaxRows][D]; per-warp key row as double [32][D]
+// dynamic shared memory after SelShared (rounded up to 128 bytes): decode q
+// rows as float [8][D], then a per-warp key row as double [warps][D]
 constexpr size_t kSelHead = (sizeof(SelShared) + 127) / 128 * 128;
+constexpr size_t kSelQ = (size_t)8 * kMaxD * 4;
 __host__ __device__ constexpr size_t sel_dyn_bytes() {
-  return kSelHead + (size_t)kMaxRows * kMaxD * 2 + (size_t)(kSelThreads / 32) * kMaxD * 8;
+  return kSelHead + kSelQ + (size_t)(kSelThreads / 32) * kMaxD * 8;
 }
 
 template <int NT>
@@ -111,8 +111,7 @@ __device__ double refine_decode(const SelArgs& a, const Problem& p, int j, const
   return total / (double)a.G;
 }
 
-__device__ double refine_prefill(const SelArgs& a, const Problem& p, int j,
-                                 const __nv_bfloat16* qtile, double* kbuf, double c2) {
+__device__ double refine_prefill(const SelArgs& a, const Problem& p, int j, double* kbuf, double c2) {
   const int lane = threadIdx.x & 31;
   const __nv_bfloat16* krow = a.k + ((size_t)(p.b * a.Hkv + p.h) * a.N + j) * a.D;
   for (int e = lane; e < a.D; e += 32) kbuf[e] = (double)__bfloat162float(krow[e]);
@@ -123,10 +122,10 @@ __device__ double refine_prefill(const SelArgs& a, const Problem& p, int j,
     const int g = r / a.tile, il = r - g * a.tile;
     const int i = p.i0 + il;
     if (il >= p.rows || j > i) continue;
-    const __nv_bfloat16* qr = qtile + (size_t)r * a.D;
+    const __nv_bfloat16* qr = a.q + ((size_t)(p.b * a.Hq + p.h * a.G + g) * a.N + i) * a.D;
     double dot = 0.0;
     for (int e = 0; e < a.D; e += 2) {
-      const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162*>(qr + e);
+      const __nv_bfloat162 q2 = __ldg(reinterpret_cast<const __nv_bfloat162*>(qr + e));
       dot += (double)__low2float(q2) * kbuf[e] + (double)__high2float(q2) * kbuf[e + 1];
     }
     const size_t srow = (size_t)(p.b * a.Hq + p.h * a.G + g) * a.N + i;
@@ -152,8 +151,7 @@ __device__ void run_problem(const SelArgs& a, Problem& p, SelShared& sh, float* 
   }
 
   float* qf = reinterpret_cast<float*>(dyn);                      // decode
-  __nv_bfloat16* qtile = reinterpret_cast<__nv_bfloat16*>(dyn);   // prefill
-  double* kbuf = reinterpret_cast<double*>(dyn + (size_t)kMaxRows * kMaxD * 2) + warp * kMaxD;
+  double* kbuf = reinterpret_cast<double*>(dyn + kSelQ) + warp * kMaxD;
 
   const float* v = p.v;
   clear_hist(sh);
@@ -192,17 +190,6 @@ __device__ void run_problem(const SelArgs& a, Problem& p, SelShared& sh, float* 
     }
     v = vscr;
   } else {
-    // stage the tile's query rows (bf16) for the fp64 refinement
-    const int nrows = a.G * a.tile;
-    const int vec_per_row = a.D / 8;
-    for (int e = tid; e < nrows * vec_per_row; e += NT) {
-      const int r = e / vec_per_row, c8 = e - r * vec_per_row;
-      const int g = r / a.tile, il = r - g * a.tile;
-      uint4 val = make_uint4(0, 0, 0, 0);
-      if (il < p.rows)
-        val = *reinterpret_cast<const uint4*>(a.q + ((size_t)(p.b * a.Hq + p.h * a.G + g) * a.N + p.i0 + il) * a.D + c8 * 8);
-      *reinterpret_cast<uint4*>(qtile + (size_t)r * a.D + c8 * 8) = val;
-    }
     for (int j = tid; j < p.n; j += NT) atomicAdd(&sh.hist[__float_as_uint(v[j]) >> 21], 1u);
   }
   __syncthreads();
@@ -263,7 +250,7 @@ __device__ void run_problem(const SelArgs& a, Problem& p, SelShared& sh, float* 
   // fp64 pooled scores of the band members, one warp per member
   for (int i = warp; i < nb; i += NT / 32) {
     const int j = band_idx[i];
-    const double val = a.prefill ? refine_prefill(a, p, j, qtile, kbuf, c2)
+    const double val = a.prefill ? refine_prefill(a, p, j, kbuf, c2)
                                  : refine_decode(a, p, j, qf, sh, c2);
     if (lane == 0) band_val[i] = val;
   }
@@ -316,6 +303,22 @@ __device__ void run_problem(const SelArgs& a, Problem& p, SelShared& sh, float* 
   __syncthreads();
 
   // ascending compaction
+  if (need_tie == 0) {
+    // one scan: thread t owns the consecutive keys [t * kpt, (t + 1) * kpt)
+    const int kpt = (p.n + NT - 1) / NT;
+    const int j0 = min(p.n, tid * kpt), j1 = min(p.n, j0 + kpt);
+    auto flag_of = [&](int j) -> int {
+      const float x = v[j];
+      return x > hi || (x >= lo && state[j] == 1);
+    };
+    int c = 0;
+    for (int j = j0; j < j1; ++j) c += flag_of(j);
+    const int incl = block_inclusive_scan<NT>(c, sh.scan_buf, nullptr);
+    int w = incl - c;
+    for (int j = j0; j < j1; ++j)
+      if (flag_of(j)) p.out[w++] = j;
+    return;
+  }
   int written = 0, ties_taken = 0;
   for (int base = 0; base < p.n; base += NT) {
     const int j = base + tid;
@@ -344,7 +347,7 @@ __device__ void run_problem(const SelArgs& a, Problem& p, SelShared& sh, float* 
 }
 
 template <int NT>
-__global__ void __launch_bounds__(NT) select_kernel(const SelArgs a) {
+__global__ void __launch_bounds__(NT, kSelCtasPerSM) select_kernel(const SelArgs a) {
   pdl_wait();
   pdl_launch_dependents();
   extern __shared__ __align__(128) char smem_raw[];
@@ -406,7 +409,7 @@ size_t select_scratch_bytes_per_cta(int n_max) {
 
 int select_grid(bool prefill, int problems, int num_sms) {
   (void)prefill;
-  const int cap = num_sms;   // one 1024-thread CTA per SM
+  const int cap = num_sms * kSelCtasPerSM;
   return problems < cap ? problems : cap;
 }
 
