@@ -154,3 +154,27 @@ def test_decode_pdl_flags_give_identical_results():
     for other in outs[1:]:
         for x, y in zip(outs[0], other):
             assert torch.equal(x, y)
+
+
+def test_decode_long_context_takes_the_two_kernel_path():
+    """A context whose scores do not fit on chip (N = 131072, G = 4) runs the
+    scoring kernel plus the 8-CTA cluster select; the Llama-shaped anchor
+    (N = 32768) runs the fused single launch.  Both match the oracle."""
+    kc = _kc()
+    B, Hq, Hkv, d, N, frac = 1, 8, 2, 128, 131072, (10, 100)
+    s = kc.Shape.make(B, Hq, Hkv, d, 1, N, frac)
+    assert kc.launch_count(s, kc.OP_SELECT) == 2
+    assert kc.launch_count(kc.Shape.make(1, 32, 8, 128, 1, 32768, frac), kc.OP_SELECT) == 1
+    q, k, v = gen_inputs(dict(B=B, Hq=Hq, Hkv=Hkv, d=d, N=N), seed=31)
+    ws = kc.Workspace(s)
+    idx = kc.select(s, q, k, ws=ws)
+    o = kc.sparse_decode(s, q, k, v, idx, None, ws=ws)
+    torch.cuda.synchronize()
+    assert ws.error() == 0
+    kk = O.topk_count(N, *frac)
+    idx_g = idx.view(B, Hkv, kk).cpu().numpy()
+    qn, kn, vn = np64(q), np64(k), np64(v)
+    _, tally = decode_idx_check(qn, kn, idx_g, frac)
+    tally.assert_ok()
+    o_ref, _ = O.sparse_decode(qn, kn, vn, idx_g)
+    check_out(np64(o).reshape(B, Hq, d), o_ref, "long-context decode")
