@@ -15,10 +15,10 @@
 //   * select_decode_cluster_kernel (fallback for contexts too long to keep
 //     the scores on chip, or devices without 16-CTA clusters) reads the
 //     scores and per-split statistics written by the scoring kernel.
-// Both then run the same cluster Top-k: radix select on the fp32 bit
-// patterns with 8-bit digits, histograms summed over distributed shared
-// memory; the band of keys within delta (relative) of the k-th fp32 value is
-// re-scored in fp64 (exact bf16 products, fp64 sums and exp2) and settled by
+// Both then run the same cluster Top-k: radix select on the top 24 bits of
+// the fp32 bit patterns (three 8-bit digits), histograms summed over
+// distributed shared memory; the band of keys within delta (relative) of the
+// 2^-15-wide bin holding the k-th fp32 value is re-scored in fp64 (exact bf16 products, fp64 sums and exp2) and settled by
 // (value desc, index asc); counts are exchanged over DSMEM and each CTA
 // writes its selected keys, ascending, at its prefix offset.
 #include <cooperative_groups.h>
@@ -40,6 +40,7 @@ constexpr float kBandDelta = 1.0f / 8192.0f;
 constexpr float kBandFloor = 0x1p-96f;
 constexpr int kFallbackCS = 8;    // cluster size of the fallback kernel
 constexpr int kRoundKeys = 256;   // fused kernel: K rows per streamed round
+constexpr int kSlots = 2;         // fused kernel: rounds in flight
 constexpr int kErrTimeout = 5;
 
 struct CSh {
@@ -56,7 +57,7 @@ struct CSh {
   float wpool[8];         // fused: weight exp2(cmax - m2) / l of the stored terms
   float wmax[kWarpsC][8];
   double wsum[kWarpsC][8];
-  unsigned long long full[2];   // fused: K round barriers
+  unsigned long long full[kSlots];   // fused: K round barriers
   int b_idx[kSmallBand];
   double b_val[kSmallBand];
 };
@@ -133,10 +134,12 @@ __device__ void cluster_topk(cg::cluster_group& cluster, CSh& sh, const float* v
   clear_hist(sh, 1);
   for (int i = tid; i < cnt; i += kCNT) atomicAdd(&sh.hist[0][__float_as_uint(v[i]) >> 24], 1u);
 
-  // radix select over the cluster: digits [31:24] [23:16] [15:8] [7:0]
+  // radix select over the cluster on digits [31:24] [23:16] [15:8]: the K-th
+  // largest fp32 value lies in the bin [prefix, prefix | 0xff], 2^-15
+  // relative wide, which the band below covers
   int need = K;
   unsigned prefix = 0;
-  for (int pass = 0; pass < 4; ++pass) {
+  for (int pass = 0; pass < 3; ++pass) {
     const int shift = 24 - 8 * pass;
     const int buf = pass & 1;
     if (pass > 0) {
@@ -151,10 +154,11 @@ __device__ void cluster_topk(cg::cluster_group& cluster, CSh& sh, const float* v
     clear_hist(sh, buf ^ 1);   // the other buffer's readers have all passed this pass's barrier
   }
 
-  // band around the k-th fp32 value
-  const float tau = __uint_as_float(prefix);
-  const float lo = tau < kBandFloor ? 0.0f : tau * (1.0f - kBandDelta);
-  const float hi = fmaxf(tau * (1.0f + kBandDelta), kBandFloor);
+  // band around the bin holding the K-th fp32 value: fewer than K values lie
+  // above hi and at least K at or above lo
+  const float tau_lo = __uint_as_float(prefix), tau_hi = __uint_as_float(prefix | 0xffu);
+  const float lo = tau_lo < kBandFloor ? 0.0f : tau_lo * (1.0f - kBandDelta);
+  const float hi = fmaxf(tau_hi * (1.0f + kBandDelta), kBandFloor);
   if (tid == 0) {
     sh.nb = 0;
     sh.chi = 0;
@@ -427,9 +431,9 @@ __global__ void __cluster_dims__(kFallbackCS, 1, 1) __launch_bounds__(kCNT)
 template <int D>
 struct ASL {
   static constexpr size_t qf = kCHead;                               // [8][128] f32
-  static constexpr size_t ring = qf + 8 * 128 * 4;                    // [2][kRoundKeys][D] bf16
+  static constexpr size_t ring = qf + 8 * 128 * 4;                    // [kSlots][kRoundKeys][D] bf16
   static constexpr size_t RB = (size_t)kRoundKeys * D * 2;
-  static constexpr size_t sc = ring + 2 * RB;                         // [G][per + 4] f32 scores
+  static constexpr size_t sc = ring + kSlots * RB;                         // [G][per + 4] f32 scores
   static size_t bytes(int G, int per) { return sc + (size_t)G * (per + 4) * 4 + (size_t)per + 16; }
   static_assert(ring % 128 == 0, "bulk copy destination alignment");
 };
@@ -468,28 +472,25 @@ __global__ void __launch_bounds__(kCNT, 1) anchor_select_kernel(const SelArgs a,
     return;
   }
 
-  // ---- stream this CTA's K rows in rounds of kRoundKeys (two in flight)
+  // ---- stream this CTA's K rows in rounds of kRoundKeys (kSlots in flight)
   const uint32_t full0 = smem_u32(&sh.full[0]);
   const int nr = (cnt + kRoundKeys - 1) / kRoundKeys;
   if (tid == 0) {
-    mbar_init(full0, 1);
-    mbar_init(full0 + 8, 1);
+    for (int sl = 0; sl < kSlots; ++sl) mbar_init(full0 + 8u * sl, 1);
     mbar_fence_init();
   }
   __syncthreads();
   auto issue = [&](int r) {   // thread 0 only
     const int k0 = r * kRoundKeys, nk = min(kRoundKeys, cnt - k0);
     const uint32_t bytes = (uint32_t)nk * D * 2;
-    const uint32_t bar = full0 + 8u * (uint32_t)(r & 1);
-    const uint32_t dst = ring + (uint32_t)((r & 1) * L::RB);
+    const uint32_t bar = full0 + 8u * (uint32_t)(r % kSlots);
+    const uint32_t dst = ring + (uint32_t)((r % kSlots) * L::RB);
     const char* src = reinterpret_cast<const char*>(kb + (size_t)(j0 + k0) * D);
     mbar_arrive_expect_tx(bar, bytes);
     for (uint32_t off = 0; off < bytes; off += 16384u) bulk_g2s(dst + off, src + off, min(16384u, bytes - off), bar);
   };
-  if (tid == 0) {
-    if (nr > 0) issue(0);
-    if (nr > 1) issue(1);
-  }
+  if (tid == 0)
+    for (int r = 0; r < kSlots && r < nr; ++r) issue(r);
   // query rows: fp32 copy for the fp64 band, MMA B fragments in registers
   // (lane (g, c) holds dims [32 s + 8 c, +8) of head g; heads >= G zero)
   for (int e = tid; e < G * D; e += kCNT) {
@@ -504,9 +505,10 @@ __global__ void __launch_bounds__(kCNT, 1) anchor_select_kernel(const SelArgs a,
   const float scale2 = kLog2e * rsqrtf((float)D);
   float mx0 = -INFINITY, mx1 = -INFINITY;   // heads 2c, 2c+1
   for (int r = 0; r < nr; ++r) {
-    if (!mbar_wait_bounded(full0 + 8u * (uint32_t)(r & 1), (uint32_t)((r >> 1) & 1))) raise_error(a.err, kErrTimeout);
+    if (!mbar_wait_bounded(full0 + 8u * (uint32_t)(r % kSlots), (uint32_t)((r / kSlots) & 1)))
+      raise_error(a.err, kErrTimeout);
     const int k0 = r * kRoundKeys, nk = min(kRoundKeys, cnt - k0);
-    const uint32_t slot = ring + (uint32_t)((r & 1) * L::RB);
+    const uint32_t slot = ring + (uint32_t)((r % kSlots) * L::RB);
     if (16 * warp < nk) {
       // S^T for 16 keys: A = K rows g and g + 8 of the group (d-permuted
       // 16-byte loads), B = q^T; k-step 2s+t takes dims 32s + 8c + 4t + {0..3}
@@ -543,9 +545,9 @@ __global__ void __launch_bounds__(kCNT, 1) anchor_select_kernel(const SelArgs a,
       }
     }
     __syncthreads();   // every warp is done with this slot
-    if (tid == 0 && r + 2 < nr) {
+    if (tid == 0 && r + kSlots < nr) {
       asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-      issue(r + 2);
+      issue(r + kSlots);
     }
   }
 
@@ -571,16 +573,26 @@ __global__ void __launch_bounds__(kCNT, 1) anchor_select_kernel(const SelArgs a,
       for (int w = 0; w < kWarpsC; ++w) cm[hh] = fmaxf(cm[hh], sh.wmax[w][hh]);
     }
   }
+  // four keys per thread and head per step (rows are 16-byte aligned: SCS is
+  // a multiple of 4); lanes past cnt exponentiate slack entries of the row and
+  // leave them out of the sums
   float ps[8];
 #pragma unroll
   for (int hh = 0; hh < 8; ++hh) ps[hh] = 0.f;
-  for (int i = tid; i < cnt; i += kCNT) {
+  const int n4 = (cnt + 3) >> 2;
+  for (int j = tid; j < n4; j += kCNT) {
+    const int rem = cnt - 4 * j;
 #pragma unroll
     for (int hh = 0; hh < 8; ++hh)
       if (hh < G) {
-        const float e = ex2_fast(sc[hh * SCS + i] - cm[hh]);   // kept for the pooled scores
-        sc[hh * SCS + i] = e;
-        ps[hh] += e;
+        float4* p = reinterpret_cast<float4*>(sc + hh * SCS + 4 * j);
+        float4 x = *p;
+        x.x = ex2_fast(x.x - cm[hh]);   // kept for the pooled scores
+        x.y = ex2_fast(x.y - cm[hh]);
+        x.z = ex2_fast(x.z - cm[hh]);
+        x.w = ex2_fast(x.w - cm[hh]);
+        *p = x;
+        ps[hh] += rem > 3 ? (x.x + x.y) + (x.z + x.w) : (x.x + (rem > 1 ? x.y : 0.f)) + (rem > 2 ? x.z : 0.f);
       }
   }
 #pragma unroll
@@ -630,12 +642,19 @@ __global__ void __launch_bounds__(kCNT, 1) anchor_select_kernel(const SelArgs a,
   float wh[8];
 #pragma unroll
   for (int hh = 0; hh < 8; ++hh) wh[hh] = hh < G ? sh.wpool[hh] : 0.f;
-  for (int i = tid; i < cnt; i += kCNT) {
-    float acc = 0.f;
+  for (int j = tid; j < n4; j += kCNT) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int hh = 0; hh < 8; ++hh)
-      if (hh < G) acc += sc[hh * SCS + i] * wh[hh];
-    v[i] = acc * invG;
+      if (hh < G) {
+        const float4 x = *reinterpret_cast<const float4*>(sc + hh * SCS + 4 * j);
+        acc.x += x.x * wh[hh];
+        acc.y += x.y * wh[hh];
+        acc.z += x.z * wh[hh];
+        acc.w += x.w * wh[hh];
+      }
+    *reinterpret_cast<float4*>(v + 4 * j) =
+        make_float4(acc.x * invG, acc.y * invG, acc.z * invG, acc.w * invG);
   }
   __syncthreads();
   cluster_topk<CS>(cluster, sh, v, st, cnt, j0, rank, K, per, out, a.band_idx + bbase + (size_t)rank * per,
@@ -673,27 +692,44 @@ int fused_active_clusters(size_t smem) {
   return n;
 }
 
-// Cluster size of the fused kernel for this shape on the current device:
-// 16 when every (batch, kv head) cluster runs at once (one wave), else 8;
+// Cluster sizes the fused kernel is built for.  A cluster must sit inside
+// one GPC, so how many clusters of each size run at once depends on the
+// device's GPC layout rather than on the SM count alone (on a 148-SM B200:
+// 15 of 8 or 9 CTAs, 11 of 10, 7 of 11 to 16).
+constexpr int kFusedSizes[] = {16, 12, 10, 9, 8};
+constexpr int kNumFusedSizes = 5;
+
+// Cluster size of the fused kernel for this shape on the current device: the
+// fewest waves of (batch, kv head) clusters, then the most CTAs (K streaming
+// bandwidth grows with the SMs a problem spans; the Top-k is latency-bound);
 // 0 when the scores do not fit on chip.
 template <int D>
 int fused_cluster_size(const SelArgs& a) {
-  static int cached[64][2] = {{0}};   // max active clusters of 16 and of 8 (+1; 0 = unknown)
+  static int cached[64][kNumFusedSizes] = {{0}};   // max active clusters (+1; 0 = unknown)
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
   const size_t max_smem = 227 * 1024;
-  const size_t s16 = ASL<D>::bytes(a.G, fused_per(a.N, 16)), s8 = ASL<D>::bytes(a.G, fused_per(a.N, 8));
   if (!cached[dev][0]) {
     cached[dev][0] = 1 + fused_active_clusters<16, D>(max_smem);
-    cached[dev][1] = 1 + fused_active_clusters<8, D>(max_smem);
+    cached[dev][1] = 1 + fused_active_clusters<12, D>(max_smem);
+    cached[dev][2] = 1 + fused_active_clusters<10, D>(max_smem);
+    cached[dev][3] = 1 + fused_active_clusters<9, D>(max_smem);
+    cached[dev][4] = 1 + fused_active_clusters<8, D>(max_smem);
     cudaGetLastError();
   }
-  const int n16 = cached[dev][0] - 1, n8 = cached[dev][1] - 1;
-  const int problems = a.B * a.Hkv;
-  const bool ok16 = s16 <= max_smem && n16 > 0, ok8 = s8 <= max_smem && n8 > 0;
-  if (ok16 && (problems <= n16 || !ok8)) return 16;
-  if (ok8) return 8;
-  return ok16 ? 16 : 0;
+  const long long problems = (long long)a.B * a.Hkv;
+  int best = 0;
+  long long best_waves = 0;
+  for (int i = 0; i < kNumFusedSizes; ++i) {   // sizes in decreasing order
+    const int cs = kFusedSizes[i], n = cached[dev][i] - 1;
+    if (n <= 0 || ASL<D>::bytes(a.G, fused_per(a.N, cs)) > max_smem) continue;
+    const long long waves = (problems + n - 1) / n;
+    if (best == 0 || waves < best_waves) {
+      best = cs;
+      best_waves = waves;
+    }
+  }
+  return best;
 }
 
 template <int CS, int D>
@@ -720,8 +756,12 @@ bool select_decode_cluster_ok(int N) { return select_decode_cluster_keys(N) <= 1
 size_t select_decode_cluster_scratch(int B, int Hkv, int N) {
   // band entries for the fallback layout and both fused cluster sizes
   const size_t fb = (size_t)kFallbackCS * select_decode_cluster_keys(N);
-  const size_t f16 = (size_t)16 * fused_per(N, 16), f8 = (size_t)8 * fused_per(N, 8);
-  return (size_t)B * Hkv * (fb > f16 ? (fb > f8 ? fb : f8) : (f16 > f8 ? f16 : f8));
+  size_t m = fb;
+  for (int i = 0; i < kNumFusedSizes; ++i) {
+    const size_t f = (size_t)kFusedSizes[i] * fused_per(N, kFusedSizes[i]);
+    m = f > m ? f : m;
+  }
+  return (size_t)B * Hkv * m;
 }
 
 cudaError_t launch_select_decode_cluster(const SelArgs& a, cudaStream_t stream) {
@@ -741,13 +781,23 @@ bool anchor_select_fused_ok(const SelArgs& a) {
 
 cudaError_t launch_anchor_select_fused(const SelArgs& a, cudaStream_t stream) {
   if (a.D == 128) {
-    const int cs = fused_cluster_size<128>(a);
-    if (cs == 16) return launch_fused<16, 128>(a, stream);
-    if (cs == 8) return launch_fused<8, 128>(a, stream);
+    switch (fused_cluster_size<128>(a)) {
+      case 16: return launch_fused<16, 128>(a, stream);
+      case 12: return launch_fused<12, 128>(a, stream);
+      case 10: return launch_fused<10, 128>(a, stream);
+      case 9: return launch_fused<9, 128>(a, stream);
+      case 8: return launch_fused<8, 128>(a, stream);
+      default: break;
+    }
   } else {
-    const int cs = fused_cluster_size<64>(a);
-    if (cs == 16) return launch_fused<16, 64>(a, stream);
-    if (cs == 8) return launch_fused<8, 64>(a, stream);
+    switch (fused_cluster_size<64>(a)) {
+      case 16: return launch_fused<16, 64>(a, stream);
+      case 12: return launch_fused<12, 64>(a, stream);
+      case 10: return launch_fused<10, 64>(a, stream);
+      case 9: return launch_fused<9, 64>(a, stream);
+      case 8: return launch_fused<8, 64>(a, stream);
+      default: break;
+    }
   }
   return cudaErrorInvalidValue;
 }
