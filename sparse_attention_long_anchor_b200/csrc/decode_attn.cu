@@ -106,55 +106,6 @@ __device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
   return r;
 }
 
-__device__ __forceinline__ uint32_t mapa(uint32_t addr, int rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(addr), "r"(rank));
-  return r;
-}
-
-// asynchronous store into another CTA's shared memory, completing on that
-// CTA's mbarrier (both addresses in the shared::cluster window)
-__device__ __forceinline__ void st_async_v4(uint32_t raddr, float4 v, uint32_t rbar) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];\n" ::"r"(raddr),
-      "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(rbar)
-      : "memory");
-}
-__device__ __forceinline__ void st_async_v2(uint32_t raddr, float2 v, uint32_t rbar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];\n" ::"r"(raddr),
-               "f"(v.x), "f"(v.y), "r"(rbar)
-               : "memory");
-}
-
-__device__ __forceinline__ void cluster_arrive_release() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait_acquire() {
-  asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// bounded wait (about 2^32 SM clocks) for data other CTAs of the cluster
-// stored into this CTA
-__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint32_t bar, uint32_t parity) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (!mbar_try_wait_cluster(bar, parity)) {
-    if (clock64() - t0 > (1ll << 32)) return false;
-  }
-  return true;
-}
-
 // kRing = false: every warp owns at most two slices (per <= 16 * 2 * kWarps),
 // all issued up front; kRing = true: the slabs are refilled two slices ahead.
 template <int D, bool kRing>

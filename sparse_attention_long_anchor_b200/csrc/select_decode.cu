@@ -16,11 +16,12 @@
 //     the scores on chip, or devices without 16-CTA clusters) reads the
 //     scores and per-split statistics written by the scoring kernel.
 // Both then run the same cluster Top-k: radix select on the top 24 bits of
-// the fp32 bit patterns (three 8-bit digits), histograms summed over
-// distributed shared memory; the band of keys within delta (relative) of the
-// 2^-15-wide bin holding the k-th fp32 value is re-scored in fp64 (exact bf16 products, fp64 sums and exp2) and settled by
-// (value desc, index asc); counts are exchanged over DSMEM and each CTA
-// writes its selected keys, ascending, at its prefix offset.
+// the fp32 bit patterns (three 8-bit digits), histograms, counts and band
+// entries sent to every CTA of the cluster with one-sided stores into its
+// shared memory; the band of keys within delta (relative) of the 2^-15-wide
+// bin holding the k-th fp32 value is re-scored in fp64 (exact bf16
+// products, fp64 sums and exp2) and settled by (value desc, index asc); each
+// CTA writes its selected keys, ascending, at its prefix offset.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -42,6 +43,12 @@ constexpr int kFallbackCS = 8;    // cluster size of the fallback kernel
 constexpr int kRoundKeys = 256;   // fused kernel: K rows per streamed round
 constexpr int kSlots = 2;         // fused kernel: rounds in flight
 constexpr int kErrTimeout = 5;
+constexpr int kMaxCS = 16;        // largest cluster
+constexpr int kRadixPasses = 3;   // 8-bit digits [31:24] [23:16] [15:8]
+// exchange barriers: one per radix pass, counts, band entries, softmax stats
+constexpr int kBarCnt = kRadixPasses, kBarBand = kRadixPasses + 1, kBarStats = kRadixPasses + 2;
+constexpr int kNumXBars = kRadixPasses + 3;
+constexpr size_t kRxBytes(int cs) { return (size_t)kRadixPasses * cs * 256 * 4; }   // radix receive slots
 
 struct CSh {
   unsigned hist[2][kCBins];
@@ -52,17 +59,40 @@ struct CSh {
   float m2[8];
   double l[8];
   float inv_l[8];
-  float cmax[8];          // fused: this CTA's max score of each head (read by the cluster)
-  double csum[8];         // fused: this CTA's sum of exp2(s2 - cmax) of each head
   float wpool[8];         // fused: weight exp2(cmax - m2) / l of the stored terms
   float wmax[kWarpsC][8];
   double wsum[kWarpsC][8];
   unsigned long long full[kSlots];   // fused: K round barriers
-  int b_idx[kSmallBand];
+  unsigned long long xbar[kNumXBars];  // one-sided exchanges (see exchange_init)
+  // slot r of these arrays is written by CTA r of the cluster
+  int2 rx_cnt[kMaxCS];               // (count above the band, band size)
+  float rx_cmax[kMaxCS][8];          // fused: CTA r's max score of each head
+  double rx_csum[kMaxCS][8];         // fused: CTA r's sum of exp2(s2 - max) of each head
+  int b_idx[kSmallBand];             // the cluster's band, ordered by CTA rank
   double b_val[kSmallBand];
 };
 
 constexpr size_t kCHead = (sizeof(CSh) + 127) / 128 * 128;
+
+// Exchanges between the CTAs of a cluster are one-sided: each CTA stores its
+// share into every other CTA's shared memory with st.async, which completes
+// on the receiver's mbarrier, and the receiver waits on its own barrier only
+// (no cluster-wide barrier, no remote loads).  Thread 0 sets the barriers up
+// with the bytes of every fixed-size exchange; the band's size is added once
+// the counts are known.  The caller then arrives on the cluster barrier and
+// waits on it before its first store into another CTA, which orders the
+// initialisation before any remote completion.
+template <int CS>
+__device__ void exchange_init(CSh& sh, int stats_bytes_per_cta) {
+  const uint32_t xb = smem_u32(&sh.xbar[0]);
+  for (int i = 0; i < kNumXBars; ++i) mbar_init(xb + 8u * i, 1);
+  mbar_fence_init();
+  for (int p = 0; p < kRadixPasses; ++p) mbar_arrive_expect_tx(xb + 8u * p, (CS - 1) * kCBins * 4);
+  mbar_arrive_expect_tx(xb + 8u * kBarCnt, (CS - 1) * 8);
+  if (stats_bytes_per_cta > 0) mbar_arrive_expect_tx(xb + 8u * kBarStats, (CS - 1) * stats_bytes_per_cta);
+}
+
+__device__ __forceinline__ int peer_of(int rank, int l, int cs) { return rank + l < cs ? rank + l : rank + l - cs; }
 
 // Sum the cluster's histograms (buffer `buf`) and find the digit holding the
 // need-th largest element.  Every CTA computes the same (bin, above).
@@ -121,37 +151,57 @@ __device__ void cluster_exchange(cg::cluster_group& cluster, CSh& sh, int slot, 
 // Everything after the pooled scores: exact Top-K over the cluster of the
 // pooled values v[0, cnt) of this CTA (keys j0 + i), written ascending into
 // out[0, K).  sh.m2 / sh.l hold the softmax statistics of the G heads and
-// qf the fp32 query rows (for the fp64 band).  Band scratch: this CTA's
-// `per` entries at band_idx / band_val; the cluster's CS * per entries start
-// at band_idx0 / band_val0.
+// qf the fp32 query rows (for the fp64 band).  rx: kRxBytes(CS) of shared
+// memory at the same offset in every CTA, receiving the radix histograms.
+// Band scratch for degenerate (large) bands: this CTA's `per` entries at
+// band_idx / band_val.  The exchanges must have been set up (exchange_init,
+// cluster barrier) before the call.
 template <int CS>
-__device__ void cluster_topk(cg::cluster_group& cluster, CSh& sh, const float* v, uint8_t* st, int cnt, int j0,
-                             int rank, int K, int per, int32_t* out, int32_t* band_idx, double* band_val,
-                             const int32_t* band_idx0, const double* band_val0, const float* qf,
-                             const __nv_bfloat16* kb, int G, int D) {
+__device__ void cluster_topk(cg::cluster_group& cluster, CSh& sh, uint32_t* rx, const float* v, uint8_t* st, int cnt,
+                             int j0, int rank, int K, int32_t* out, int32_t* band_idx, double* band_val,
+                             const float* qf, const __nv_bfloat16* kb, int G, int D, int* err) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  clear_hist(sh, 0);
-  clear_hist(sh, 1);
-  for (int i = tid; i < cnt; i += kCNT) atomicAdd(&sh.hist[0][__float_as_uint(v[i]) >> 24], 1u);
+  const uint32_t xb = smem_u32(&sh.xbar[0]);
+  // this CTA's histogram slots start at zero (the others only ever receive)
+  for (int i = tid; i < kRadixPasses * kCBins; i += kCNT)
+    rx[((i / kCBins) * CS + rank) * kCBins + (i % kCBins)] = 0u;
+  __syncthreads();
 
   // radix select over the cluster on digits [31:24] [23:16] [15:8]: the K-th
   // largest fp32 value lies in the bin [prefix, prefix | 0xff], 2^-15
-  // relative wide, which the band below covers
+  // relative wide, which the band below covers.  Each pass: local histogram,
+  // sent to the other CTAs in 16-byte pieces, summed over the CS slots.
   int need = K;
   unsigned prefix = 0;
-  for (int pass = 0; pass < 3; ++pass) {
+  for (int pass = 0; pass < kRadixPasses; ++pass) {
     const int shift = 24 - 8 * pass;
-    const int buf = pass & 1;
-    if (pass > 0) {
-      for (int i = tid; i < cnt; i += kCNT) {
-        const unsigned x = __float_as_uint(v[i]);
-        if ((x >> (shift + 8)) == (prefix >> (shift + 8))) atomicAdd(&sh.hist[buf][(x >> shift) & 255u], 1u);
-      }
+    uint32_t* mine = rx + (pass * CS + rank) * kCBins;
+    for (int i = tid; i < cnt; i += kCNT) {
+      const unsigned x = __float_as_uint(v[i]);
+      if (pass == 0 || (x >> (shift + 8)) == (prefix >> (shift + 8))) atomicAdd(&mine[(x >> shift) & 255u], 1u);
     }
-    cluster_find_bin<CS>(cluster, sh, buf, need);
+    __syncthreads();
+    for (int t = tid; t < (CS - 1) * (kCBins / 4); t += kCNT) {
+      const int pr = peer_of(rank, 1 + t / (kCBins / 4), CS), ch = t % (kCBins / 4);
+      const uint32_t src = smem_u32(mine) + 16u * ch;
+      st_async_v4u(mapa(src, pr), reinterpret_cast<const uint4*>(mine)[ch], mapa(xb + 8u * pass, pr));
+    }
+    if (!mbar_wait_cluster_bounded(xb + 8u * pass, 0)) raise_error(err, kErrTimeout);
+    int local = 0, bin = -1;
+    if (tid < kCBins) {
+      bin = kCBins - 1 - tid;   // thread 0 holds the largest digit
+#pragma unroll
+      for (int r = 0; r < CS; ++r) local += (int)rx[(pass * CS + r) * kCBins + bin];
+    }
+    const int incl = block_inclusive_scan<kCNT>(local, sh.scan_buf, nullptr);
+    const int excl = incl - local;
+    if (tid < kCBins && excl < need && need <= incl) {
+      sh.bin = bin;
+      sh.above = excl;
+    }
+    __syncthreads();
     prefix |= (unsigned)sh.bin << shift;
     need -= sh.above;
-    clear_hist(sh, buf ^ 1);   // the other buffer's readers have all passed this pass's barrier
   }
 
   // band around the bin holding the K-th fp32 value: fewer than K values lie
@@ -179,23 +229,31 @@ __device__ void cluster_topk(cg::cluster_group& cluster, CSh& sh, const float* v
   __syncthreads();
   const int nb = sh.nb, chi = sh.chi;
   // one exchange of (count above the band, band size)
-  if (tid == 0) {
-    sh.xchg[0] = chi;
-    sh.xchg[1] = nb;
+  if (tid < CS) {
+    const unsigned long long pair = (unsigned long long)(unsigned)chi | ((unsigned long long)(unsigned)nb << 32);
+    if (tid == 0) {
+      sh.rx_cnt[rank] = make_int2(chi, nb);
+    } else {
+      const int pr = peer_of(rank, tid, CS);
+      st_async_u64(mapa(smem_u32(&sh.rx_cnt[rank]), pr), pair, mapa(xb + 8u * kBarCnt, pr));
+    }
   }
   __syncthreads();
-  cluster.sync();
+  if (!mbar_wait_cluster_bounded(xb + 8u * kBarCnt, 0)) raise_error(err, kErrTimeout);
   int chi_total = 0, chi_below = 0, nb_total = 0, nb_below = 0;
 #pragma unroll
   for (int r = 0; r < CS; ++r) {
-    const int x = *cluster.map_shared_rank(&sh.xchg[0], r);
-    const int y = *cluster.map_shared_rank(&sh.xchg[1], r);
-    chi_total += x;
-    nb_total += y;
-    chi_below += r < rank ? x : 0;
-    nb_below += r < rank ? y : 0;
+    const int2 xy = sh.rx_cnt[r];
+    chi_total += xy.x;
+    nb_total += xy.y;
+    chi_below += r < rank ? xy.x : 0;
+    nb_below += r < rank ? xy.y : 0;
   }
   const int need_band = K - chi_total;
+  // small bands (the usual case) are sent whole to every CTA: entry i of CTA
+  // r lands at position (entries of lower ranks) + i
+  const bool small = nb_total <= kSmallBand;
+  if (small && tid == 0) mbar_arrive_expect_tx(xb + 8u * kBarBand, (uint32_t)(nb_total - nb) * 12u);
 
   // fp64 pooled scores of this CTA's band members, one warp per member
   const double c2 = 1.4426950408889634 / sqrt((double)D);
@@ -215,34 +273,32 @@ __device__ void cluster_topk(cg::cluster_group& cluster, CSh& sh, const float* v
       for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
       total += exp2(dot * c2 - (double)sh.m2[g]) / sh.l[g];
     }
-    if (lane == 0) band_val[i] = total / (double)G;
+    const double val = total / (double)G;   // every lane holds it
+    if (!small) {
+      if (lane == 0) band_val[i] = val;
+    } else if (lane == 0) {
+      sh.b_idx[nb_below + i] = j;
+      sh.b_val[nb_below + i] = val;
+    } else if (lane < CS) {
+      const int pr = peer_of(rank, lane, CS);
+      const uint32_t bar = mapa(xb + 8u * kBarBand, pr);
+      st_async_u32(mapa(smem_u32(&sh.b_idx[nb_below + i]), pr), (uint32_t)j, bar);
+      st_async_u64(mapa(smem_u32(&sh.b_val[nb_below + i]), pr), (unsigned long long)__double_as_longlong(val), bar);
+    }
   }
-  __threadfence();
   __syncthreads();
-  cluster.sync();
 
   int tie_quota = 0, sel_below = 0;
   auto flag_of = [&](int i) -> int {
     const float x = v[i];
     return x > hi || (x >= lo && st[i] == 1);
   };
-  if (nb_total <= kSmallBand) {
-    // every CTA gathers the whole band (ordered by CTA rank) and ranks the
+  if (small) {
+    // every CTA holds the whole band (ordered by CTA rank) and ranks the
     // members of the lower CTAs and its own: its own are marked, the lower
     // ones give this CTA's output offset
-    for (int t = tid; t < nb_total; t += kCNT) {
-      int r = 0, off = t;
-      while (r < CS) {
-        const int nr = *cluster.map_shared_rank(&sh.xchg[1], r);
-        if (off < nr) break;
-        off -= nr;
-        ++r;
-      }
-      sh.b_idx[t] = __ldcg(band_idx0 + (size_t)r * per + off);
-      sh.b_val[t] = __ldcg(band_val0 + (size_t)r * per + off);
-    }
-    cluster_arrive();   // the last reads of other CTAs' shared memory
-    __syncthreads();
+    if (!mbar_wait_cluster_bounded(xb + 8u * kBarBand, 0)) raise_error(err, kErrTimeout);
+    cluster_arrive();   // nothing more is sent to other CTAs
     int low_sel = 0;
     for (int t = tid; t < nb_below + nb; t += kCNT) {
       const double mv = sh.b_val[t];
@@ -356,8 +412,8 @@ __device__ void cluster_topk(cg::cluster_group& cluster, CSh& sh, const float* v
 // ---------------------------------------------------------------- fallback
 
 __host__ __device__ constexpr size_t cluster_dyn_bytes(int keys_per_cta) {
-  // q rows fp32 [8][128], v[keys] fp32, state[keys] bytes
-  return kCHead + 8 * 128 * 4 + (size_t)keys_per_cta * 4 + (size_t)keys_per_cta;
+  // q rows fp32 [8][128], radix receive slots, v[keys] fp32, state[keys] bytes
+  return kCHead + 8 * 128 * 4 + kRxBytes(kFallbackCS) + (size_t)keys_per_cta * 4 + (size_t)keys_per_cta;
 }
 
 __global__ void __cluster_dims__(kFallbackCS, 1, 1) __launch_bounds__(kCNT)
@@ -367,7 +423,8 @@ __global__ void __cluster_dims__(kFallbackCS, 1, 1) __launch_bounds__(kCNT)
   extern __shared__ __align__(128) char smem_raw[];
   CSh& sh = *reinterpret_cast<CSh*>(smem_raw);
   float* qf = reinterpret_cast<float*>(smem_raw + kCHead);
-  float* v = qf + 8 * 128;
+  uint32_t* rx = reinterpret_cast<uint32_t*>(qf + 8 * 128);
+  float* v = reinterpret_cast<float*>(smem_raw + kCHead + 8 * 128 * 4 + kRxBytes(kFallbackCS));
   uint8_t* st = reinterpret_cast<uint8_t*>(v + keys_per_cta);
 
   cg::cluster_group cluster = cg::this_cluster();
@@ -387,6 +444,9 @@ __global__ void __cluster_dims__(kFallbackCS, 1, 1) __launch_bounds__(kCNT)
     for (int i = tid; i < cnt; i += kCNT) out[j0 + i] = j0 + i;
     return;
   }
+  if (tid == 0) exchange_init<kFallbackCS>(sh, 0);
+  __syncthreads();
+  cluster_arrive();
 
   // softmax statistics of the G query heads from the scoring kernel's splits
   for (int g = warp; g < G; g += kWarpsC) {
@@ -420,10 +480,11 @@ __global__ void __cluster_dims__(kFallbackCS, 1, 1) __launch_bounds__(kCNT)
     v[i] = acc * invG;
   }
   __syncthreads();
-  cluster_topk<kFallbackCS>(cluster, sh, v, st, cnt, j0, rank, K, keys_per_cta, out,
+  cluster_wait();   // every CTA's exchange barriers are initialised
+  cluster_topk<kFallbackCS>(cluster, sh, rx, v, st, cnt, j0, rank, K, out,
                             a.band_idx + bbase + (size_t)rank * keys_per_cta,
-                            a.band_val + bbase + (size_t)rank * keys_per_cta, a.band_idx + bbase,
-                            a.band_val + bbase, qf, a.k + (size_t)bh * N * D, G, D);
+                            a.band_val + bbase + (size_t)rank * keys_per_cta, qf, a.k + (size_t)bh * N * D, G, D,
+                            a.err);
 }
 
 // ------------------------------------------------------------ fused select
@@ -436,6 +497,7 @@ struct ASL {
   static constexpr size_t sc = ring + kSlots * RB;                         // [G][per + 4] f32 scores
   static size_t bytes(int G, int per) { return sc + (size_t)G * (per + 4) * 4 + (size_t)per + 16; }
   static_assert(ring % 128 == 0, "bulk copy destination alignment");
+  static_assert(kSlots * RB >= kRxBytes(kMaxCS), "the ring doubles as the radix receive buffer");
 };
 
 template <int CS, int D>
@@ -477,9 +539,10 @@ __global__ void __launch_bounds__(kCNT, 1) anchor_select_kernel(const SelArgs a,
   const int nr = (cnt + kRoundKeys - 1) / kRoundKeys;
   if (tid == 0) {
     for (int sl = 0; sl < kSlots; ++sl) mbar_init(full0 + 8u * sl, 1);
-    mbar_fence_init();
+    exchange_init<CS>(sh, G * 12);   // stats: one f32 max and one f64 sum per head
   }
   __syncthreads();
+  cluster_arrive();   // matched before the first exchange, long after every CTA got here
   auto issue = [&](int r) {   // thread 0 only
     const int k0 = r * kRoundKeys, nk = min(kRoundKeys, cnt - k0);
     const uint32_t bytes = (uint32_t)nk * D * 2;
@@ -611,14 +674,24 @@ __global__ void __launch_bounds__(kCNT, 1) anchor_select_kernel(const SelArgs a,
     for (int w = 0; w < kWarpsC; ++w) s += sh.wsum[w][tid];
 #pragma unroll
     for (int hh = 0; hh < 8; ++hh)
-      if (hh == tid) sh.cmax[hh] = cm[hh];
-    sh.csum[tid] = s;
+      if (hh == tid) sh.rx_cmax[rank][hh] = cm[hh];
+    sh.rx_csum[rank][tid] = s;
   }
-  cluster.sync();
+  __syncthreads();
+  cluster_wait();   // every CTA's exchange barriers are initialised
+  const uint32_t stats_bar = smem_u32(&sh.xbar[kBarStats]);
+  if (tid < (CS - 1) * G) {
+    const int hh = tid % G, pr = peer_of(rank, 1 + tid / G, CS);
+    const uint32_t bar = mapa(stats_bar, pr);
+    st_async_u32(mapa(smem_u32(&sh.rx_cmax[rank][hh]), pr), __float_as_uint(sh.rx_cmax[rank][hh]), bar);
+    st_async_u64(mapa(smem_u32(&sh.rx_csum[rank][hh]), pr),
+                 (unsigned long long)__double_as_longlong(sh.rx_csum[rank][hh]), bar);
+  }
+  if (!mbar_wait_cluster_bounded(stats_bar, 0)) raise_error(a.err, kErrTimeout);
   // warp hh (< G): lane r < CS takes CTA r's (max, sum) of head hh
   if (warp < G) {
-    const float mr = lane < CS ? *cluster.map_shared_rank(&sh.cmax[warp], lane) : -INFINITY;
-    const double sr = lane < CS ? *cluster.map_shared_rank(&sh.csum[warp], lane) : 0.0;
+    const float mr = lane < CS ? sh.rx_cmax[lane][warp] : -INFINITY;
+    const double sr = lane < CS ? sh.rx_csum[lane][warp] : 0.0;
     float m = mr;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -630,7 +703,7 @@ __global__ void __launch_bounds__(kCNT, 1) anchor_select_kernel(const SelArgs a,
       sh.l[warp] = l;
       sh.inv_l[warp] = (float)(1.0 / l);
       // pooled weight of this CTA's stored terms exp2(s - cm)
-      const float cmh = sh.cmax[warp];
+      const float cmh = sh.rx_cmax[rank][warp];
       sh.wpool[warp] = cmh == -INFINITY ? 0.f : (float)(exp2((double)cmh - (double)m) / l);
     }
   }
@@ -657,8 +730,10 @@ __global__ void __launch_bounds__(kCNT, 1) anchor_select_kernel(const SelArgs a,
         make_float4(acc.x * invG, acc.y * invG, acc.z * invG, acc.w * invG);
   }
   __syncthreads();
-  cluster_topk<CS>(cluster, sh, v, st, cnt, j0, rank, K, per, out, a.band_idx + bbase + (size_t)rank * per,
-                   a.band_val + bbase + (size_t)rank * per, a.band_idx + bbase, a.band_val + bbase, qf, kb, G, D);
+  // the ring is free: it receives the radix histograms
+  cluster_topk<CS>(cluster, sh, reinterpret_cast<uint32_t*>(smem_raw + L::ring), v, st, cnt, j0, rank, K, out,
+                   a.band_idx + bbase + (size_t)rank * per, a.band_val + bbase + (size_t)rank * per, qf, kb, G, D,
+                   a.err);
 }
 
 int fused_per(int N, int cs) {
