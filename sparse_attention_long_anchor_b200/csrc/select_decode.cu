@@ -94,6 +94,57 @@ __device__ void exchange_init(CSh& sh, int stats_bytes_per_cta) {
 
 __device__ __forceinline__ int peer_of(int rank, int l, int cs) { return rank + l < cs ? rank + l : rank + l - cs; }
 
+// Thread t < 256 holds c, the count of digit 255 - t; find the digit holding
+// the need-th largest element into (sh.bin, sh.above): a scan over the eight
+// warps that hold digits, two barriers.
+__device__ __forceinline__ void find_digit(CSh& sh, int c, int need) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int x = c;
+  if (warp < kCBins / 32) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) sh.scan_buf[warp] = x;
+  }
+  __syncthreads();
+  if (warp < kCBins / 32) {
+    int pre = 0;
+#pragma unroll
+    for (int w = 0; w < kCBins / 32 - 1; ++w) pre += w < warp ? sh.scan_buf[w] : 0;
+    const int incl = pre + x, excl = incl - c;
+    if (excl < need && need <= incl) {
+      sh.bin = kCBins - 1 - tid;
+      sh.above = excl;
+    }
+  }
+  __syncthreads();
+}
+
+// exclusive prefix over the CTA of one count per thread, and the total: one
+// barrier (the caller must not reuse sh.scan_buf before another barrier)
+__device__ __forceinline__ int cta_exclusive_scan(CSh& sh, int c, int* total) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int x = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh.scan_buf[warp] = x;
+  __syncthreads();
+  int pre = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < kWarpsC; ++w) {
+    const int t = sh.scan_buf[w];
+    pre += w < warp ? t : 0;
+    tot += t;
+  }
+  *total = tot;
+  return pre + x - c;
+}
+
 // Sum the cluster's histograms (buffer `buf`) and find the digit holding the
 // need-th largest element.  Every CTA computes the same (bin, above).
 template <int CS>
@@ -187,19 +238,12 @@ __device__ void cluster_topk(cg::cluster_group& cluster, CSh& sh, uint32_t* rx, 
       st_async_v4u(mapa(src, pr), reinterpret_cast<const uint4*>(mine)[ch], mapa(xb + 8u * pass, pr));
     }
     if (!mbar_wait_cluster_bounded(xb + 8u * pass, 0)) raise_error(err, kErrTimeout);
-    int local = 0, bin = -1;
-    if (tid < kCBins) {
-      bin = kCBins - 1 - tid;   // thread 0 holds the largest digit
+    int local = 0;
+    if (tid < kCBins) {   // thread 0 holds the largest digit
 #pragma unroll
-      for (int r = 0; r < CS; ++r) local += (int)rx[(pass * CS + r) * kCBins + bin];
+      for (int r = 0; r < CS; ++r) local += (int)rx[(pass * CS + r) * kCBins + (kCBins - 1 - tid)];
     }
-    const int incl = block_inclusive_scan<kCNT>(local, sh.scan_buf, nullptr);
-    const int excl = incl - local;
-    if (tid < kCBins && excl < need && need <= incl) {
-      sh.bin = bin;
-      sh.above = excl;
-    }
-    __syncthreads();
+    find_digit(sh, local, need);
     prefix |= (unsigned)sh.bin << shift;
     need -= sh.above;
   }
@@ -259,20 +303,35 @@ __device__ void cluster_topk(cg::cluster_group& cluster, CSh& sh, uint32_t* rx, 
   const double c2 = 1.4426950408889634 / sqrt((double)D);
   for (int i = warp; i < nb; i += kWarpsC) {
     const int j = band_idx[i];
-    const __nv_bfloat16* krow = kb + (size_t)j * D;
-    float kv[4];
-#pragma unroll
-    for (int t = 0; t < 4; ++t) kv[t] = lane + 32 * t < D ? __bfloat162float(krow[lane + 32 * t]) : 0.f;
-    double total = 0.0;
-    for (int g = 0; g < G; ++g) {
-      double dot = 0.0;
-#pragma unroll
-      for (int t = 0; t < 4; ++t)
-        if (lane + 32 * t < D) dot += (double)qf[g * D + lane + 32 * t] * (double)kv[t];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-      total += exp2(dot * c2 - (double)sh.m2[g]) / sh.l[g];
+    // lane holds dims [4 lane, 4 lane + 4) (d = 128) or [2 lane, 2 lane + 2)
+    // (d = 64); every head's dot product and reduction interleaved
+    float kv[4] = {0.f, 0.f, 0.f, 0.f};
+    const int dl = D / 32;
+    if (dl == 4) {
+      const uint2 r = *reinterpret_cast<const uint2*>(kb + (size_t)j * D + 4 * lane);
+      kv[0] = bf16_lo(r.x), kv[1] = bf16_hi(r.x), kv[2] = bf16_lo(r.y), kv[3] = bf16_hi(r.y);
+    } else {
+      const uint32_t r = *reinterpret_cast<const uint32_t*>(kb + (size_t)j * D + 2 * lane);
+      kv[0] = bf16_lo(r), kv[1] = bf16_hi(r);
     }
+    double dot[8];
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      dot[g] = 0.0;
+      if (g < G)
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          if (t < dl) dot[g] += (double)qf[g * D + dl * lane + t] * (double)kv[t];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int g = 0; g < 8; ++g)
+        if (g < G) dot[g] += __shfl_xor_sync(0xffffffffu, dot[g], o);
+    double total = 0.0;
+#pragma unroll
+    for (int g = 0; g < 8; ++g)
+      if (g < G) total += exp2(dot[g] * c2 - (double)sh.m2[g]) / sh.l[g];
     const double val = total / (double)G;   // every lane holds it
     if (!small) {
       if (lane == 0) band_val[i] = val;
@@ -297,8 +356,9 @@ __device__ void cluster_topk(cg::cluster_group& cluster, CSh& sh, uint32_t* rx, 
     // every CTA holds the whole band (ordered by CTA rank) and ranks the
     // members of the lower CTAs and its own: its own are marked, the lower
     // ones give this CTA's output offset
+    // every byte another CTA sends here has now arrived, and no CTA reads
+    // another's shared memory on this path: no closing cluster barrier
     if (!mbar_wait_cluster_bounded(xb + 8u * kBarBand, 0)) raise_error(err, kErrTimeout);
-    cluster_arrive();   // nothing more is sent to other CTAs
     int low_sel = 0;
     for (int t = tid; t < nb_below + nb; t += kCNT) {
       const double mv = sh.b_val[t];
@@ -377,8 +437,8 @@ __device__ void cluster_topk(cg::cluster_group& cluster, CSh& sh, uint32_t* rx, 
     const int b0 = min(cnt, tid * kpt), b1 = min(cnt, b0 + kpt);
     int c = 0;
     for (int i = b0; i < b1; ++i) c += flag_of(i);
-    const int incl = block_inclusive_scan<kCNT>(c, sh.scan_buf, nullptr);
-    int w = sel_below + incl - c;
+    int unused;
+    int w = sel_below + cta_exclusive_scan(sh, c, &unused);
     for (int i = b0; i < b1; ++i)
       if (flag_of(i)) out[w++] = j0 + i;
   } else {
@@ -405,8 +465,8 @@ __device__ void cluster_topk(cg::cluster_group& cluster, CSh& sh, uint32_t* rx, 
       written += total;
     }
   }
-  // no CTA may leave while another can still read its shared memory
-  cluster_wait();
+  // large bands: no CTA may leave while another can still read its shared memory
+  if (!small) cluster_wait();
 }
 
 // ---------------------------------------------------------------- fallback
