@@ -304,7 +304,8 @@ __device__ void cluster_topk(cg::cluster_group& cluster, CSh& sh, uint32_t* rx, 
   for (int i = warp; i < nb; i += kWarpsC) {
     const int j = band_idx[i];
     // lane holds dims [4 lane, 4 lane + 4) (d = 128) or [2 lane, 2 lane + 2)
-    // (d = 64); every head's dot product and reduction interleaved
+    // (d = 64).  The head loop stays rolled: this runs once per launch,
+    // mostly from a cold instruction cache, where code size is the cost.
     float kv[4] = {0.f, 0.f, 0.f, 0.f};
     const int dl = D / 32;
     if (dl == 4) {
@@ -314,24 +315,17 @@ __device__ void cluster_topk(cg::cluster_group& cluster, CSh& sh, uint32_t* rx, 
       const uint32_t r = *reinterpret_cast<const uint32_t*>(kb + (size_t)j * D + 2 * lane);
       kv[0] = bf16_lo(r), kv[1] = bf16_hi(r);
     }
-    double dot[8];
-#pragma unroll
-    for (int g = 0; g < 8; ++g) {
-      dot[g] = 0.0;
-      if (g < G)
-#pragma unroll
-        for (int t = 0; t < 4; ++t)
-          if (t < dl) dot[g] += (double)qf[g * D + dl * lane + t] * (double)kv[t];
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-      for (int g = 0; g < 8; ++g)
-        if (g < G) dot[g] += __shfl_xor_sync(0xffffffffu, dot[g], o);
     double total = 0.0;
+#pragma unroll 1
+    for (int g = 0; g < G; ++g) {
+      double dot = 0.0;
 #pragma unroll
-    for (int g = 0; g < 8; ++g)
-      if (g < G) total += exp2(dot[g] * c2 - (double)sh.m2[g]) / sh.l[g];
+      for (int t = 0; t < 4; ++t)
+        if (t < dl) dot += (double)qf[g * D + dl * lane + t] * (double)kv[t];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+      total += exp2(dot * c2 - (double)sh.m2[g]) / sh.l[g];
+    }
     const double val = total / (double)G;   // every lane holds it
     if (!small) {
       if (lane == 0) band_val[i] = val;
