@@ -224,6 +224,7 @@ __device__ void cluster_topk(cg::cluster_group& cluster, CSh& sh, uint32_t* rx, 
   // sent to the other CTAs in 16-byte pieces, summed over the CS slots.
   int need = K;
   unsigned prefix = 0;
+#pragma unroll 1   // one copy of the pass: passes 2 and 3 run from the instruction cache pass 1 filled
   for (int pass = 0; pass < kRadixPasses; ++pass) {
     const int shift = 24 - 8 * pass;
     uint32_t* mine = rx + (pass * CS + rank) * kCBins;
@@ -749,16 +750,17 @@ __global__ void __launch_bounds__(kCNT, 1) anchor_select_kernel(const SelArgs a,
     float m = mr;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    double l = mr != -INFINITY ? sr * exp2((double)mr - (double)m) : 0.0;
+    const double e = mr != -INFINITY ? exp2((double)mr - (double)m) : 0.0;   // CTA r's terms rescaled
+    const double e_own = __shfl_sync(0xffffffffu, e, rank);
+    double l = sr * e;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
     if (lane == 0) {
+      const double inv = 1.0 / l;
       sh.m2[warp] = m;
       sh.l[warp] = l;
-      sh.inv_l[warp] = (float)(1.0 / l);
-      // pooled weight of this CTA's stored terms exp2(s - cm)
-      const float cmh = sh.rx_cmax[rank][warp];
-      sh.wpool[warp] = cmh == -INFINITY ? 0.f : (float)(exp2((double)cmh - (double)m) / l);
+      sh.inv_l[warp] = (float)inv;
+      sh.wpool[warp] = (float)(e_own * inv);   // pooled weight of this CTA's stored terms exp2(s - cm)
     }
   }
   __syncthreads();
