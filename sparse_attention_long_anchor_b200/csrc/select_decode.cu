@@ -682,54 +682,43 @@ __global__ void __launch_bounds__(kCNT, 1) anchor_select_kernel(const SelArgs a,
     sh.wmax[warp][2 * c + 1] = mx1;
   }
   __syncthreads();
-  float cm[8];
+  if (tid < G) {   // this CTA's max of each head, in its own exchange slot
+    float m = -INFINITY;
 #pragma unroll
-  for (int hh = 0; hh < 8; ++hh) {
-    cm[hh] = -INFINITY;
-    if (hh < G) {
-#pragma unroll
-      for (int w = 0; w < kWarpsC; ++w) cm[hh] = fmaxf(cm[hh], sh.wmax[w][hh]);
-    }
+    for (int w = 0; w < kWarpsC; ++w) m = fmaxf(m, sh.wmax[w][tid]);
+    sh.rx_cmax[rank][tid] = m;
   }
-  // four keys per thread and head per step (rows are 16-byte aligned: SCS is
-  // a multiple of 4); lanes past cnt exponentiate slack entries of the row and
-  // leave them out of the sums
-  float ps[8];
-#pragma unroll
-  for (int hh = 0; hh < 8; ++hh) ps[hh] = 0.f;
+  __syncthreads();
+  // exp2(s - max) in place, four keys per thread per step (rows are 16-byte
+  // aligned: SCS is a multiple of 4); lanes past cnt exponentiate slack
+  // entries of the row and leave them out of the sums.  The head loop stays
+  // rolled: this code runs once per launch from a cold instruction cache.
   const int n4 = (cnt + 3) >> 2;
-  for (int j = tid; j < n4; j += kCNT) {
-    const int rem = cnt - 4 * j;
-#pragma unroll
-    for (int hh = 0; hh < 8; ++hh)
-      if (hh < G) {
-        float4* p = reinterpret_cast<float4*>(sc + hh * SCS + 4 * j);
-        float4 x = *p;
-        x.x = ex2_fast(x.x - cm[hh]);   // kept for the pooled scores
-        x.y = ex2_fast(x.y - cm[hh]);
-        x.z = ex2_fast(x.z - cm[hh]);
-        x.w = ex2_fast(x.w - cm[hh]);
-        *p = x;
-        ps[hh] += rem > 3 ? (x.x + x.y) + (x.z + x.w) : (x.x + (rem > 1 ? x.y : 0.f)) + (rem > 2 ? x.z : 0.f);
-      }
-  }
-#pragma unroll
-  for (int hh = 0; hh < 8; ++hh) {
-    if (hh < G) {
-      double d = ps[hh];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-      if (lane == 0) sh.wsum[warp][hh] = d;
+#pragma unroll 1
+  for (int hh = 0; hh < G; ++hh) {
+    const float cmh = sh.rx_cmax[rank][hh];
+    float ps = 0.f;
+    for (int j = tid; j < n4; j += kCNT) {
+      const int rem = cnt - 4 * j;
+      float4* p = reinterpret_cast<float4*>(sc + hh * SCS + 4 * j);
+      float4 x = *p;
+      x.x = ex2_fast(x.x - cmh);   // kept for the pooled scores
+      x.y = ex2_fast(x.y - cmh);
+      x.z = ex2_fast(x.z - cmh);
+      x.w = ex2_fast(x.w - cmh);
+      *p = x;
+      ps += rem > 3 ? (x.x + x.y) + (x.z + x.w) : (x.x + (rem > 1 ? x.y : 0.f)) + (rem > 2 ? x.z : 0.f);
     }
+    double d = ps;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+    if (lane == 0) sh.wsum[warp][hh] = d;
   }
   __syncthreads();
   if (tid < G) {
     double s = 0.0;
 #pragma unroll
     for (int w = 0; w < kWarpsC; ++w) s += sh.wsum[w][tid];
-#pragma unroll
-    for (int hh = 0; hh < 8; ++hh)
-      if (hh == tid) sh.rx_cmax[rank][hh] = cm[hh];
     sh.rx_csum[rank][tid] = s;
   }
   __syncthreads();
@@ -768,20 +757,17 @@ __global__ void __launch_bounds__(kCNT, 1) anchor_select_kernel(const SelArgs a,
   // ---- pooled scores, in place of head 0's scores
   float* v = sc;
   const float invG = 1.0f / (float)G;
-  float wh[8];
-#pragma unroll
-  for (int hh = 0; hh < 8; ++hh) wh[hh] = hh < G ? sh.wpool[hh] : 0.f;
   for (int j = tid; j < n4; j += kCNT) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int hh = 0; hh < 8; ++hh)
-      if (hh < G) {
-        const float4 x = *reinterpret_cast<const float4*>(sc + hh * SCS + 4 * j);
-        acc.x += x.x * wh[hh];
-        acc.y += x.y * wh[hh];
-        acc.z += x.z * wh[hh];
-        acc.w += x.w * wh[hh];
-      }
+#pragma unroll 1
+    for (int hh = 0; hh < G; ++hh) {
+      const float wh = sh.wpool[hh];
+      const float4 x = *reinterpret_cast<const float4*>(sc + hh * SCS + 4 * j);
+      acc.x += x.x * wh;
+      acc.y += x.y * wh;
+      acc.z += x.z * wh;
+      acc.w += x.w * wh;
+    }
     *reinterpret_cast<float4*>(v + 4 * j) =
         make_float4(acc.x * invG, acc.y * invG, acc.z * invG, acc.w * invG);
   }
