@@ -24,6 +24,7 @@
 // CTA writes its selected keys, ascending, at its prefix offset.
 #include <cooperative_groups.h>
 
+#include "cluster_choice.h"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -816,10 +817,9 @@ int fused_active_clusters(size_t smem) {
 constexpr int kFusedSizes[] = {16, 12, 10, 9, 8};
 constexpr int kNumFusedSizes = 5;
 
-// Cluster size of the fused kernel for this shape on the current device: the
-// fewest waves of (batch, kv head) clusters, then the most CTAs (K streaming
-// bandwidth grows with the SMs a problem spans; the Top-k is latency-bound);
-// 0 when the scores do not fit on chip.
+// Cluster size of the fused kernel for this shape on the current device
+// (choose_cluster_size: fewest waves, then the most CTAs); 0 when the scores
+// do not fit on chip.
 template <int D>
 int fused_cluster_size(const SelArgs& a) {
   static int cached[64][kNumFusedSizes] = {{0}};   // max active clusters (+1; 0 = unknown)
@@ -834,19 +834,13 @@ int fused_cluster_size(const SelArgs& a) {
     cached[dev][4] = 1 + fused_active_clusters<8, D>(max_smem);
     cudaGetLastError();
   }
-  const long long problems = (long long)a.B * a.Hkv;
-  int best = 0;
-  long long best_waves = 0;
-  for (int i = 0; i < kNumFusedSizes; ++i) {   // sizes in decreasing order
-    const int cs = kFusedSizes[i], n = cached[dev][i] - 1;
-    if (n <= 0 || ASL<D>::bytes(a.G, fused_per(a.N, cs)) > max_smem) continue;
-    const long long waves = (problems + n - 1) / n;
-    if (best == 0 || waves < best_waves) {
-      best = cs;
-      best_waves = waves;
-    }
+  int active[kNumFusedSizes];
+  bool fits[kNumFusedSizes];
+  for (int i = 0; i < kNumFusedSizes; ++i) {
+    active[i] = cached[dev][i] - 1;
+    fits[i] = ASL<D>::bytes(a.G, fused_per(a.N, kFusedSizes[i])) <= max_smem;
   }
-  return best;
+  return choose_cluster_size((long long)a.B * a.Hkv, kFusedSizes, active, fits, kNumFusedSizes);
 }
 
 template <int CS, int D>

@@ -1,0 +1,74 @@
+"""Host-side rules of the CUDA library that need no GPU, compiled from the
+library's own headers with the host C++ compiler.
+
+choose_cluster_size (csrc/cluster_choice.h) picks the cluster size of the fused
+decode select: the fewest waves of (batch, kv head) clusters, then the largest
+size.  The active-cluster counts below are the ones the occupancy query
+reports on a 148-SM B200 at one CTA per SM (15 clusters of 8 or 9 CTAs, 11 of
+10, 7 of 12 or 16)."""
+import os
+import shutil
+import subprocess
+
+import pytest
+
+CSRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                    "sparse_attention_long_anchor_b200", "csrc")
+
+SIZES = [16, 12, 10, 9, 8]
+B200_ACTIVE = [7, 7, 11, 15, 15]
+
+CASES = [
+    # (problems, active, fits, expected)
+    *[(p, B200_ACTIVE, [1] * 5, 16) for p in range(1, 8)],
+    (8, B200_ACTIVE, [1] * 5, 10),      # the Llama-shaped layer: 8 kv heads
+    (11, B200_ACTIVE, [1] * 5, 10),
+    (12, B200_ACTIVE, [1] * 5, 9),
+    (15, B200_ACTIVE, [1] * 5, 9),
+    (16, B200_ACTIVE, [1] * 5, 10),     # two waves at 10, 9 or 8: the largest
+    (22, B200_ACTIVE, [1] * 5, 10),
+    (23, B200_ACTIVE, [1] * 5, 9),
+    (64, B200_ACTIVE, [1] * 5, 9),      # batch 8: five waves of 9
+    (4, B200_ACTIVE, [0, 1, 1, 1, 1], 12),   # 16-CTA shared memory does not fit
+    (4, [0, 0, 11, 15, 15], [1] * 5, 10),     # no large clusters on the device
+    (4, B200_ACTIVE, [0, 0, 0, 0, 1], 8),
+    (4, [0] * 5, [1] * 5, 0),                 # nothing runs: no fused kernel
+    (4, B200_ACTIVE, [0] * 5, 0),
+]
+
+
+def _program() -> str:
+    lines = ['#include <cstdio>', '#include "cluster_choice.h"', "int main() {",
+             "  const int sizes[5] = {%s};" % ", ".join(map(str, SIZES))]
+    for i, (p, act, fits, _) in enumerate(CASES):
+        lines.append("  { const int a[5] = {%s}; const bool f[5] = {%s};"
+                     % (", ".join(map(str, act)), ", ".join("true" if x else "false" for x in fits)))
+        lines.append('    std::printf("%%d\\n", kascade::choose_cluster_size(%dLL, sizes, a, f, 5)); }' % p)
+    lines += ["  return 0;", "}"]
+    return "\n".join(lines) + "\n"
+
+
+@pytest.fixture(scope="module")
+def chosen(tmp_path_factory):
+    cxx = shutil.which("g++") or shutil.which("c++")
+    if cxx is None:
+        pytest.skip("no host C++ compiler")
+    d = tmp_path_factory.mktemp("host_rules")
+    src, exe = d / "t.cpp", d / "t"
+    src.write_text(_program())
+    subprocess.run([cxx, "-std=c++17", "-O1", "-I", CSRC, str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    return [int(x) for x in out]
+
+
+@pytest.mark.parametrize("case", range(len(CASES)))
+def test_cluster_size_rule(chosen, case):
+    problems, active, fits, expected = CASES[case]
+    assert chosen[case] == expected, (problems, active, fits)
+
+
+def test_rule_never_picks_a_size_that_cannot_run(chosen):
+    for (problems, active, fits, _), got in zip(CASES, chosen):
+        if got:
+            i = SIZES.index(got)
+            assert active[i] > 0 and fits[i]
