@@ -11,10 +11,12 @@
 //     MMAs (keys as the MMA rows, the <= 8 query heads of the group as its
 //     columns), keeps the scores in shared memory and takes the softmax
 //     statistics of every head over the cluster through distributed shared
-//     memory: one launch, no score round trip through global memory;
+//     memory: one launch, no score round trip through global memory.
+//     The cluster size (16, 12, 10, 9 or 8 CTAs) is chosen per device and
+//     shape by choose_cluster_size;
 //   * select_decode_cluster_kernel (fallback for contexts too long to keep
-//     the scores on chip, or devices without 16-CTA clusters) reads the
-//     scores and per-split statistics written by the scoring kernel.
+//     the scores on chip at any of those sizes) reads the scores and
+//     per-split statistics written by the scoring kernel.
 // Both then run the same cluster Top-k: radix select on the top 24 bits of
 // the fp32 bit patterns (three 8-bit digits), histograms, counts and band
 // entries sent to every CTA of the cluster with one-sided stores into its
