@@ -250,8 +250,18 @@ def decode_layer(kc, st, l, which="all"):
         if which in ("all", "attn"):
             kc.sparse_decode(shape, q, k, v, idx[l], None, o=outs[l], ws=ws)
     elif which in ("all", "attn"):
-        stable = shape.with_flags(kc.FLAG_PDL | kc.FLAG_INPUTS_STABLE)
-        kc.sparse_decode(stable, q, k, v, idx[anchor], hms[l], o=outs[l], ws=ws)
+        kc.sparse_decode(_stable_shape(kc, shape), q, k, v, idx[anchor], hms[l], o=outs[l], ws=ws)
+
+
+_STABLE = {}
+
+
+def _stable_shape(kc, shape):
+    """The reuse layers' shape (early gathers), built once per stack shape."""
+    hit = _STABLE.get(id(shape))
+    if hit is None or hit[0] is not shape:
+        hit = _STABLE[id(shape)] = (shape, shape.with_flags(kc.FLAG_PDL | kc.FLAG_INPUTS_STABLE))
+    return hit[1]
 
 
 def build_prefill(kc, synth, torch, dev):

@@ -5,6 +5,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+#include <vector>
+
 namespace kascade {
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -315,6 +318,41 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }  // namespace kascade
 
 namespace kascade {
+
+// Set a kernel's dynamic shared-memory limit (and, for clusters above 8
+// CTAs, the non-portable cluster size) once per device: the attributes stay
+// with the function in the device's context, so repeating the driver calls
+// on every launch only adds host latency.  The limit is raised when a launch
+// needs more than any earlier one on the device.  (A device reset clears the
+// attributes; the cache assumes none happens while the library is in use.)
+inline cudaError_t ensure_func_attrs(const void* fn, size_t smem, bool nonportable_cluster) {
+  struct Entry {
+    const void* fn;
+    int dev;
+    long long smem;
+    bool nonportable;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  size_t i = 0;
+  while (i < done.size() && !(done[i].fn == fn && done[i].dev == dev)) ++i;
+  if (i == done.size()) done.push_back({fn, dev, -1, false});
+  if ((long long)smem > done[i].smem) {
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    done[i].smem = (long long)smem;
+  }
+  if (nonportable_cluster && !done[i].nonportable) {
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    done[i].nonportable = true;
+  }
+  return cudaSuccess;
+}
 
 // Host-side launch with optional programmatic dependent launch and a
 // runtime cluster size (1 = none).

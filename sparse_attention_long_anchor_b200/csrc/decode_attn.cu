@@ -439,13 +439,9 @@ int cluster_size_for_device() {
 
 template <int D, bool kRing>
 cudaError_t launch_cs(const AttnArgs& a, int cs, int per, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<D, kRing>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)Lay<D>::total);
+  const cudaError_t e =
+      ensure_func_attrs(reinterpret_cast<const void*>(decode_attn_kernel<D, kRing>), Lay<D>::total, cs > 8);
   if (e != cudaSuccess) return e;
-  if (cs > 8) {
-    e = cudaFuncSetAttribute(decode_attn_kernel<D, kRing>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-  }
   return launch_ex(decode_attn_kernel<D, kRing>, dim3(cs, a.B * a.Hkv), dim3(kThreads), Lay<D>::total, stream,
                    (a.flags & 1) != 0, cs, a, per);
 }

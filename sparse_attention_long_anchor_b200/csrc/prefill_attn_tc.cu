@@ -503,14 +503,14 @@ cudaError_t launch_prefill_attn_tc(const AttnArgs& a, int num_sms, cudaStream_t 
   const int grid = (int)(ctas < num_sms ? ctas : num_sms);
   const bool pdl = (a.flags & 1) != 0;
   if (a.D == 128) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)PAL<128>::alloc);
+    const cudaError_t e =
+        ensure_func_attrs(reinterpret_cast<const void*>(prefill_attn_tc_kernel<128>), PAL<128>::alloc, false);
     if (e != cudaSuccess) return e;
     return launch_ex(prefill_attn_tc_kernel<128>, dim3(grid), dim3(kThreads), PAL<128>::alloc, stream, pdl, 1, mq,
                      a, RB);
   }
-  cudaError_t e = cudaFuncSetAttribute(prefill_attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)PAL<64>::alloc);
+  const cudaError_t e =
+      ensure_func_attrs(reinterpret_cast<const void*>(prefill_attn_tc_kernel<64>), PAL<64>::alloc, false);
   if (e != cudaSuccess) return e;
   return launch_ex(prefill_attn_tc_kernel<64>, dim3(grid), dim3(kThreads), PAL<64>::alloc, stream, pdl, 1, mq, a,
                    RB);

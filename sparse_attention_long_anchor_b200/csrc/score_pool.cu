@@ -243,11 +243,13 @@ cudaError_t launch_score_pool(const ScorePoolArgs& a, cudaStream_t stream) {
   dim3 grid(T, a.B * a.Hkv);
   if (a.D == 128) {
     const size_t sm = score_pool_smem<128>();
-    cudaFuncSetAttribute(score_pool_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    const cudaError_t e = ensure_func_attrs(reinterpret_cast<const void*>(score_pool_kernel<128>), sm, false);
+    if (e != cudaSuccess) return e;
     return launch_ex(score_pool_kernel<128>, grid, dim3(kSpWarps * 32), sm, stream, (a.flags & 1) != 0, 1, a);
   } else {
     const size_t sm = score_pool_smem<64>();
-    cudaFuncSetAttribute(score_pool_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    const cudaError_t e = ensure_func_attrs(reinterpret_cast<const void*>(score_pool_kernel<64>), sm, false);
+    if (e != cudaSuccess) return e;
     return launch_ex(score_pool_kernel<64>, grid, dim3(kSpWarps * 32), sm, stream, (a.flags & 1) != 0, 1, a);
   }
   return cudaGetLastError();

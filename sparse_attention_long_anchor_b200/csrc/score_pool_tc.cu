@@ -368,14 +368,14 @@ cudaError_t launch_score_pool_tc(const ScorePoolArgs& a, int* err, int num_sms, 
   const int grid = (int)(items < num_sms ? items : num_sms);
   const bool pdl = (a.flags & 1) != 0;
   if (a.D == 128) {
-    cudaError_t e = cudaFuncSetAttribute(score_pool_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)SPL<128>::alloc);
+    const cudaError_t e =
+        ensure_func_attrs(reinterpret_cast<const void*>(score_pool_tc_kernel<128>), SPL<128>::alloc, false);
     if (e != cudaSuccess) return e;
     return launch_ex(score_pool_tc_kernel<128>, dim3(grid), dim3(kThreads), SPL<128>::alloc, stream, pdl, 1, mq, mk,
                      a, err);
   }
-  cudaError_t e = cudaFuncSetAttribute(score_pool_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)SPL<64>::alloc);
+  const cudaError_t e =
+      ensure_func_attrs(reinterpret_cast<const void*>(score_pool_tc_kernel<64>), SPL<64>::alloc, false);
   if (e != cudaSuccess) return e;
   return launch_ex(score_pool_tc_kernel<64>, dim3(grid), dim3(kThreads), SPL<64>::alloc, stream, pdl, 1, mq, mk, a,
                    err);

@@ -849,13 +849,8 @@ template <int CS, int D>
 cudaError_t launch_fused(const SelArgs& a, cudaStream_t stream) {
   const int per = fused_per(a.N, CS);
   const size_t smem = ASL<D>::bytes(a.G, per);
-  cudaError_t e = cudaFuncSetAttribute(anchor_select_kernel<CS, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  const cudaError_t e = ensure_func_attrs(reinterpret_cast<const void*>(anchor_select_kernel<CS, D>), smem, CS > 8);
   if (e != cudaSuccess) return e;
-  if (CS > 8) {
-    e = cudaFuncSetAttribute(anchor_select_kernel<CS, D>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-  }
   return launch_ex(anchor_select_kernel<CS, D>, dim3(CS, a.B * a.Hkv), dim3(kCNT), smem, stream,
                    (a.flags & 1) != 0, CS, a, per);
 }
@@ -880,8 +875,7 @@ size_t select_decode_cluster_scratch(int B, int Hkv, int N) {
 cudaError_t launch_select_decode_cluster(const SelArgs& a, cudaStream_t stream) {
   const int per = select_decode_cluster_keys(a.N);
   const size_t smem = cluster_dyn_bytes(per);
-  cudaError_t e = cudaFuncSetAttribute(select_decode_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  const cudaError_t e = ensure_func_attrs(reinterpret_cast<const void*>(select_decode_cluster_kernel), smem, false);
   if (e != cudaSuccess) return e;
   dim3 grid(kFallbackCS, a.B * a.Hkv);
   return launch_ex(select_decode_cluster_kernel, grid, dim3(kCNT), smem, stream, (a.flags & 1) != 0, 1, a, per);

@@ -254,12 +254,14 @@ cudaError_t launch_prefill_attn(const AttnArgs& a, cudaStream_t stream) {
   dim3 grid(T * row_blocks, a.B * a.Hkv);
   if (a.D == 128) {
     const size_t sm = prefill_smem<128>();
-    cudaFuncSetAttribute(prefill_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    const cudaError_t e = ensure_func_attrs(reinterpret_cast<const void*>(prefill_attn_kernel<128>), sm, false);
+    if (e != cudaSuccess) return e;
     return launch_ex(prefill_attn_kernel<128>, grid, dim3(kPreWarps * 32), sm, stream, (a.flags & 1) != 0, 1, a,
                      row_blocks);
   } else {
     const size_t sm = prefill_smem<64>();
-    cudaFuncSetAttribute(prefill_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    const cudaError_t e = ensure_func_attrs(reinterpret_cast<const void*>(prefill_attn_kernel<64>), sm, false);
+    if (e != cudaSuccess) return e;
     return launch_ex(prefill_attn_kernel<64>, grid, dim3(kPreWarps * 32), sm, stream, (a.flags & 1) != 0, 1, a,
                      row_blocks);
   }

@@ -415,8 +415,7 @@ int select_grid(bool prefill, int problems, int num_sms) {
 
 cudaError_t launch_select(const SelArgs& a, cudaStream_t stream) {
   const size_t smem = sel_dyn_bytes();
-  cudaError_t e = cudaFuncSetAttribute(select_kernel<kSelThreads>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const cudaError_t e = ensure_func_attrs(reinterpret_cast<const void*>(select_kernel<kSelThreads>), smem, false);
   if (e != cudaSuccess) return e;
   return launch_ex(select_kernel<kSelThreads>, dim3(a.grid), dim3(kSelThreads), smem, stream, (a.flags & 1) != 0, 1, a);
 }

@@ -118,8 +118,15 @@ def _ptr(t):
     return t.data_ptr()
 
 
+# the raw handle of the current stream without building a Stream object
+# (a per-call host cost of the eager API); the public call where absent
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(stream):
     if stream is None:
+        if _raw_stream is not None:
+            return _raw_stream(torch.cuda.current_device())
         return torch.cuda.current_stream().cuda_stream
     if isinstance(stream, int):
         return stream
