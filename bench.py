@@ -432,21 +432,24 @@ def run_kascade(args, rank, world, local):
         }
         launches += len(pcfg.anchors) * (kc.launch_count(pre[3], kc.OP_SELECT) + 1) + (pcfg.n_layers - len(pcfg.anchors))
 
-    # ---- end to end through the public API: pinned host q -> device, step, outputs -> host
+    # ---- end to end through the public API: the step's queries (every layer's
+    # q, one pinned host buffer) copied in, the layers run, the step's outputs
+    # copied back; one copy each way
     cfg, plan, layers, shape, ws, idx, hms, outs = dec
-    host_q = [layers[l][0].cpu().pin_memory() for l in range(n_dec)]
-    host_o = [torch.empty_like(h).pin_memory() for h in host_q]
-    dev_q = [layers[l][0] for l in range(n_dec)]
-    h2d = sum(h.numel() * h.element_size() for h in host_q)
-    d2h = sum(h.numel() * h.element_size() for h in host_o)
+    q_all = torch.stack([layers[l][0] for l in range(n_dec)])
+    o_all = torch.empty_like(q_all)
+    host_q = q_all.cpu().pin_memory()
+    host_o = torch.empty_like(host_q).pin_memory()
+    e2e_dec = (cfg, plan, [(q_all[l], layers[l][1], layers[l][2]) for l in range(n_dec)], shape, ws, idx, hms,
+               {l: o_all[l] for l in range(n_dec)})
+    h2d = host_q.numel() * host_q.element_size()
+    d2h = host_o.numel() * host_o.element_size()
 
     def e2e_step():
+        q_all.copy_(host_q, non_blocking=True)
         for l in range(n_dec):
-            dev_q[l].copy_(host_q[l], non_blocking=True)
-        for l in range(n_dec):
-            decode_layer(kc, dec, l)
-        for l in range(n_dec):
-            host_o[l].copy_(outs[l], non_blocking=True)
+            decode_layer(kc, e2e_dec, l)
+        host_o.copy_(o_all, non_blocking=True)
 
     for _ in range(args.warmup):
         e2e_step()
@@ -481,7 +484,8 @@ def run_kascade(args, rank, world, local):
         "roofline": roofline, "components": components, "prefill": prefill_obj,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_ms * 1e3 / (n_dec * world), "unit": "us/layer-step", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "path": "eager Python API calls per layer, pinned host q in, o out"},
+                "d2h_bytes_per_step": d2h,
+                "path": "eager Python API calls per layer; the step's q (all layers) in and o out, one pinned copy each"},
         "gpu_launches": launches * args.steps,
         "clocks": clk,
     }
