@@ -54,11 +54,11 @@ constexpr int kNumXBars = kRadixPasses + 3;
 constexpr size_t kRxBytes(int cs) { return (size_t)kRadixPasses * cs * 256 * 4; }   // radix receive slots
 
 struct CSh {
-  unsigned hist[2][kCBins];
+  unsigned hist[2][kCBins];   // large-band path: fp64 radix histograms, read by the cluster
   int scan_buf[kCNT / 32 + 1];
   int bin, above;
   int nb, chi;
-  int xchg[4];            // published to the cluster: c_hi, nb, ties, selected
+  int xchg[4];            // large-band path, read by the cluster: slots 2 (ties) and 3 (selected)
   float m2[8];
   double l[8];
   float inv_l[8];
@@ -148,8 +148,10 @@ __device__ __forceinline__ int cta_exclusive_scan(CSh& sh, int c, int* total) {
   return pre + x - c;
 }
 
-// Sum the cluster's histograms (buffer `buf`) and find the digit holding the
-// need-th largest element.  Every CTA computes the same (bin, above).
+// Large-band path only (degenerate inputs): sum the cluster's histograms
+// (buffer `buf`) over cluster barriers and remote loads, and find the digit
+// holding the need-th largest element.  Every CTA computes the same
+// (bin, above).
 template <int CS>
 __device__ void cluster_find_bin(cg::cluster_group& cluster, CSh& sh, int buf, int need) {
   __syncthreads();
@@ -184,7 +186,8 @@ __device__ __forceinline__ void clear_hist(CSh& sh, int buf) {
 __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.aligned;\n" ::: "memory"); }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;\n" ::: "memory"); }
 
-// exchange one int per CTA: returns the total and the sum over lower ranks
+// large-band path: exchange one int per CTA over a cluster barrier; returns
+// the total and the sum over lower ranks
 template <int CS>
 __device__ void cluster_exchange(cg::cluster_group& cluster, CSh& sh, int slot, int mine, int rank, int* total,
                                  int* below) {
