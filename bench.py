@@ -37,6 +37,7 @@ if ROOT not in sys.path:
 METRIC = "sparse decode µs/layer-step & prefill ms/layer at 32K-128K ctx; % HBM/TC roofline"
 DECODE_CFG = "decode_llama8b_n32k"
 PREFILL_CFG = "prefill_qwen8b_n32k"
+BATCHED_DECODE_CFG = "decode_llama8b_b8_n64k"
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -323,6 +324,43 @@ def decode_bytes(cfg):
     return kk, reuse, anchor_score
 
 
+def batched_decode_component(kc, synth, torch, dev, reps, pk):
+    """Anchor select and sparse decode of the batched 64K decode stack (B=8,
+    N=65536, 10 %), where a reuse layer gathers 216 MB: the bandwidth-bound
+    regime of the sparse decode.  Layers 0 (anchor), 1 and 2 (reuse) are
+    built; the timed graph alternates the two reuse layers, so the 432 MB
+    they gather together exceed L2."""
+    cfg = synth.CONFIGS[BATCHED_DECODE_CFG]
+    plan, layers = synth.make_stack(cfg, device=dev, layers=[0, 1, 2])
+    frac = (cfg.frac_num, cfg.frac_den)
+    shape = kc.Shape.make(cfg.batch, cfg.hq, cfg.hkv, cfg.d, 1, cfg.n_ctx, frac, flags=kc.FLAG_PDL)
+    stable = shape.with_flags(kc.FLAG_PDL | kc.FLAG_INPUTS_STABLE)
+    ws = kc.Workspace(shape, device=dev)
+    idx = torch.empty(kc.index_count(shape), dtype=torch.int32, device=dev)
+    q0, k0, _ = layers[0]
+    hms = {l: torch.tensor(plan[l][2], dtype=torch.int32, device=dev) for l in (1, 2)}
+    outs = {l: torch.empty_like(layers[l][0]) for l in (1, 2)}
+    kc.select(shape, q0, k0, idx, ws=ws)
+    torch.cuda.synchronize()
+
+    def reuse(l):
+        q, k, v = layers[l]
+        kc.sparse_decode(stable, q, k, v, idx, hms[l], o=outs[l], ws=ws)
+
+    g_sel = capture(torch, lambda: kc.select(shape, q0, k0, idx, ws=ws))
+    g_att = capture(torch, lambda: [reuse(1 + (i & 1)) for i in range(8)])
+    sel_us = time_graph(torch, g_sel, reps) * 1e3
+    att_us = time_graph(torch, g_att, reps) * 1e3 / 8
+    _, reuse_bytes, score_bytes = decode_bytes(cfg)
+    gbs = reuse_bytes / (att_us * 1e-6) / 1e9
+    err = ws.error()
+    del g_sel, g_att
+    return {"workload": BATCHED_DECODE_CFG, "sparse_decode_us": att_us, "algorithmic_bytes": reuse_bytes,
+            "sparse_decode_GBps": gbs, "frac_of_hbm": gbs / pk["hbm_gbs"],
+            "anchor_select_us": sel_us, "anchor_select_GBps_on_K": score_bytes / (sel_us * 1e-6) / 1e9,
+            "device_error_word": err}
+
+
 def prefill_flops(cfg):
     """Executed flops of the two-pass exact scoring of one anchor layer and
     gathered bytes / flops of one sparse prefill layer."""
@@ -404,6 +442,8 @@ def run_kascade(args, rank, world, local):
                   "anchor_select_us_per_anchor": sel_ms * 1e3 / n_anchor,
                   "anchor_scoring_bytes": anchor_score_bytes,
                   "anchor_select_GBps_on_K": anchor_score_bytes / (sel_ms * 1e-3 / n_anchor) / 1e9}
+    if args.batched_decode:
+        components["batched_decode"] = batched_decode_component(kc, synth, torch, dev, reps, pk)
     # kernels per step, as the library reports them for these shapes on this device
     launches = n_anchor * (kc.launch_count(dec[3], kc.OP_SELECT) + 1) + (n_dec - n_anchor)
 
@@ -502,6 +542,8 @@ def main():
     ap.add_argument("--impl", choices=("kascade", "reference"), default="kascade")
     ap.add_argument("--decode-only", action="store_true", help="skip the prefill stack")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batched-decode", action="store_true",
+                    help="also time the batched 64K decode (B=8) select and sparse decode, outside the step")
     args = ap.parse_args()
     rank, world, local = dist_setup()
     try:
