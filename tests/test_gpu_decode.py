@@ -5,7 +5,7 @@ import pytest
 import torch
 
 import oracle as O
-from parity import Tally, check_lse, check_out, decode_idx_check, gen_inputs, np64
+from parity import check_lse, check_out, decode_idx_check, gen_inputs, np64
 
 pytestmark = pytest.mark.gpu
 

@@ -7,7 +7,6 @@ measured times.  These run here with world size 2 on the host."""
 import os
 import socket
 
-import pytest
 import torch.multiprocessing as mp
 
 
