@@ -39,18 +39,31 @@ def _stale() -> bool:
     return any(os.path.getmtime(p) > t for p in deps)
 
 
+def _finish(proc) -> None:
+    if proc.wait() != 0:
+        raise subprocess.CalledProcessError(proc.returncode, proc.args)
+
+
 def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     if not force and not _stale():
         return LIB
     os.makedirs(BUILD, exist_ok=True)
-    objs = []
+    jobs = []
     for src in sources():
         obj = os.path.join(BUILD, os.path.basename(src) + ".o")
-        cmd = [nvcc(), *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
+        jobs.append(([nvcc(), *ARCH, *FLAGS, *extra, "-c", src, "-o", obj], obj))
+    # one nvcc per translation unit, run side by side
+    width = max(1, min(len(jobs), os.cpu_count() or 1))
+    running = []
+    for cmd, _ in jobs:
         if verbose:
             print(" ".join(cmd), flush=True)
-        subprocess.run(cmd, check=True)
-        objs.append(obj)
+        running.append(subprocess.Popen(cmd))
+        if len(running) >= width:
+            _finish(running.pop(0))
+    for p in running:
+        _finish(p)
+    objs = [obj for _, obj in jobs]
     tmp = LIB + ".tmp"
     cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-Xlinker", "--exclude-libs=ALL"]
     subprocess.run(cmd, check=True)

@@ -31,6 +31,7 @@
 
 #include <type_traits>
 
+#include "cluster_choice.h"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -295,6 +296,74 @@ __global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const AttnArgs
     }
   };
 
+  // Both of a warp's slices as one 32-key block: four independent QK^T
+  // accumulator chains, one online-softmax update, then both PV products, so
+  // the two slices' latency chains overlap.
+  auto step2 = [&](int s0, int s1) {
+    float sa0[4] = {0.f, 0.f, 0.f, 0.f}, sb0[4] = {0.f, 0.f, 0.f, 0.f};
+    float sa1[4] = {0.f, 0.f, 0.f, 0.f}, sb1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int q = 0; q < KS; ++q) {
+      const uint2 qlo = *reinterpret_cast<const uint2*>(qrow + 64 * q);
+      const uint2 qhi = *reinterpret_cast<const uint2*>(qrow + 64 * q + 8);
+      const int pch = (4 * q + c) ^ ((g & 1) << 2);
+      const uint4 m0 = lds_v4(kslot + g * L::ROWB + pch * 16);
+      const uint4 m1 = lds_v4(kslot + (8 + g) * L::ROWB + pch * 16);
+      const uint4 k0 = kr[0][q], k1 = kr[1][q];
+      const uint32_t a0[4] = {k0.x, k1.x, k0.y, k1.y}, a1[4] = {k0.z, k1.z, k0.w, k1.w};
+      const uint32_t d0[4] = {m0.x, m1.x, m0.y, m1.y}, d1[4] = {m0.z, m1.z, m0.w, m1.w};
+      mma_bf16_16816(q & 1 ? sb0 : sa0, a0, qlo.x, qlo.y);
+      mma_bf16_16816(q & 1 ? sb1 : sa1, d0, qlo.x, qlo.y);
+      mma_bf16_16816(q & 1 ? sb0 : sa0, a1, qhi.x, qhi.y);
+      mma_bf16_16816(q & 1 ? sb1 : sa1, d1, qhi.x, qhi.y);
+    }
+    const int kb0 = c0 + s0 * 16, kb1 = c0 + s1 * 16;
+    const bool v0l = kb0 + g < c1, v0h = kb0 + 8 + g < c1, v1l = kb1 + g < c1, v1h = kb1 + 8 + g < c1;
+    float sv[8];
+    sv[0] = v0l ? (sa0[0] + sb0[0]) * scale2 : -INFINITY;
+    sv[1] = v0l ? (sa0[1] + sb0[1]) * scale2 : -INFINITY;
+    sv[2] = v0h ? (sa0[2] + sb0[2]) * scale2 : -INFINITY;
+    sv[3] = v0h ? (sa0[3] + sb0[3]) * scale2 : -INFINITY;
+    sv[4] = v1l ? (sa1[0] + sb1[0]) * scale2 : -INFINITY;
+    sv[5] = v1l ? (sa1[1] + sb1[1]) * scale2 : -INFINITY;
+    sv[6] = v1h ? (sa1[2] + sb1[2]) * scale2 : -INFINITY;
+    sv[7] = v1h ? (sa1[3] + sb1[3]) * scale2 : -INFINITY;
+    float mx0 = fmaxf(fmaxf(sv[0], sv[2]), fmaxf(sv[4], sv[6]));
+    float mx1 = fmaxf(fmaxf(sv[1], sv[3]), fmaxf(sv[5], sv[7]));
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+    const float al0 = scale_from(m_run[0], mn0), al1 = scale_from(m_run[1], mn1);
+    float p[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) p[i] = exp2f(sv[i] - (i & 1 ? mn1 : mn0));
+    l_run[0] = l_run[0] * al0 + ((p[0] + p[2]) + (p[4] + p[6]));
+    l_run[1] = l_run[1] * al1 + ((p[1] + p[3]) + (p[5] + p[7]));
+    m_run[0] = mn0;
+    m_run[1] = mn1;
+    const uint32_t b00 = movmatrix_trans(pack_bf16(p[0], p[1])), b01 = movmatrix_trans(pack_bf16(p[2], p[3]));
+    const uint32_t b10 = movmatrix_trans(pack_bf16(p[4], p[5])), b11 = movmatrix_trans(pack_bf16(p[6], p[7]));
+    const int vrow = ((lane >> 4) << 3) + (lane & 7);
+    const int vch = (lane >> 3) & 1;
+#pragma unroll
+    for (int i = 0; i < D / 16; ++i) {
+      uint32_t r0[4], r1[4];
+      const uint32_t off = vrow * L::ROWB + (((2 * i + vch) ^ (lane & 7)) * 16);
+      ldmatrix_x4_trans(r0, wbase + off);
+      ldmatrix_x4_trans(r1, wbase + L::SLAB + off);
+      float t[4] = {oacc[i][0] * al0, oacc[i][1] * al1, oacc[i][2] * al0, oacc[i][3] * al1};
+      mma_bf16_16816(t, r0, b00, b01);
+      mma_bf16_16816(t, r1, b10, b11);
+      oacc[i][0] = t[0];
+      oacc[i][1] = t[1];
+      oacc[i][2] = t[2];
+      oacc[i][3] = t[3];
+    }
+  };
+
   if constexpr (kRing) {
     int it = 0;
     for (int s = warp; s < n_slices; s += kWarps, ++it) {
@@ -316,8 +385,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const AttnArgs
   } else {
     cp_async_wait<0>();
     __syncwarp();
-    if (warp < n_slices) step(warp, 0, std::false_type{});
-    if (warp + kWarps < n_slices) step(warp + kWarps, 1, std::true_type{});
+    if (warp + kWarps < n_slices) step2(warp, warp + kWarps);
+    else if (warp < n_slices) step(warp, 0, std::false_type{});
   }
   cp_async_wait<0>();
 #pragma unroll
@@ -414,27 +483,40 @@ cudaLaunchConfig_t make_cfg(int cs, int bh, cudaStream_t stream, cudaLaunchAttri
   return cfg;
 }
 
-// 16-CTA clusters when the device can co-schedule them, else 8
+// Cluster sizes of the sparse decode, largest first.  One cluster per
+// (batch, kv head) problem: at batch 1 the largest cluster spreads the
+// gathers widest (the kernel is latency-bound there); with many problems the
+// fewest waves matter (choose_cluster_size).
+constexpr int kDecSizes[] = {16, 8, 4};
+constexpr int kNumDecSizes = 3;
+
 template <int D, bool kRing>
-int cluster_size_for_device() {
-  static int cached[64] = {0};
+int decode_cluster_size(long long problems) {
+  static int cached[64][kNumDecSizes] = {{0}};   // max active clusters + 1 (0 = unknown)
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 8;
-  if (cached[dev]) return cached[dev];
-  int cs = 8;
-  if (cudaFuncSetAttribute(decode_attn_kernel<D, kRing>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)Lay<D>::total) == cudaSuccess &&
-      cudaFuncSetAttribute(decode_attn_kernel<D, kRing>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+  if (!cached[dev][0]) {
+    for (int i = 0; i < kNumDecSizes; ++i) {
+      const int cs = kDecSizes[i];
+      int n = 0;
+      if (ensure_func_attrs(reinterpret_cast<const void*>(decode_attn_kernel<D, kRing>), Lay<D>::total, cs > 8) ==
           cudaSuccess) {
-    cudaLaunchAttribute attr[1];
-    cudaLaunchConfig_t cfg = make_cfg<D, kRing>(kMaxCS, 1, nullptr, attr);
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, decode_attn_kernel<D, kRing>, &cfg) == cudaSuccess && n > 0)
-      cs = kMaxCS;
+        cudaLaunchAttribute attr[1];
+        cudaLaunchConfig_t cfg = make_cfg<D, kRing>(cs, 1, nullptr, attr);
+        if (cudaOccupancyMaxActiveClusters(&n, decode_attn_kernel<D, kRing>, &cfg) != cudaSuccess) n = 0;
+      }
+      cached[dev][i] = 1 + n;
+    }
+    cudaGetLastError();
   }
-  cudaGetLastError();
-  cached[dev] = cs;
-  return cs;
+  int active[kNumDecSizes];
+  bool fits[kNumDecSizes];
+  for (int i = 0; i < kNumDecSizes; ++i) {
+    active[i] = cached[dev][i] - 1;
+    fits[i] = true;
+  }
+  const int cs = choose_cluster_size(problems, kDecSizes, active, fits, kNumDecSizes);
+  return cs > 0 ? cs : 8;
 }
 
 template <int D, bool kRing>
@@ -450,7 +532,7 @@ template <int D>
 cudaError_t launch(const AttnArgs& a, cudaStream_t stream) {
   // both variants share the shared-memory size and cluster shape, so one
   // occupancy answer serves both
-  const int cs = cluster_size_for_device<D, false>();
+  const int cs = decode_cluster_size<D, false>((long long)a.B * a.Hkv);
   const int list_len = a.idx ? topk_count(a.N, a.num, a.den) : a.N;
   int per = (list_len + cs - 1) / cs;
   per = (per + 15) / 16 * 16;
