@@ -18,7 +18,7 @@ Inference", the Kascade README):
   / ``k=10`` arguments ("Kernel Benchmarks", "Python API") give the budget as a
   percentage of the context.
 
-Readings of what the page leaves open (each one is listed in the design doc):
+Readings of what the page leaves open:
 
 * scores are q.k / sqrt(d) with no bias (standard scaled dot product);
 * query head qh belongs to kv head qh // G (contiguous GQA groups);
@@ -52,6 +52,9 @@ __all__ = [
     "select_topk", "anchor_select_decode", "anchor_select_prefill_tile",
     "sparse_attend", "sparse_decode", "sparse_prefill_tile", "dense_attention",
     "check_index_set",
+    "MODES", "selection_heads", "pooled_decode_heads", "pooled_prefill_tile_heads",
+    "anchor_select_decode_mode", "anchor_select_prefill_tile_mode", "sparse_decode_mode",
+    "sparse_prefill_tile_mode",
 ]
 
 
@@ -285,3 +288,144 @@ def check_index_set(pooled: np.ndarray, k: int, got, rel: float = 1e-6) -> str:
     if np.all(np.abs(pooled[others] - tau_k) <= rel * tau_k):
         return "near_tie"
     return "fail"
+
+
+# ---------------------------------------------------------------------------
+# head-selection variants
+#
+# The README's Reproducibility section runs two more selection strategies
+# beside the default post_softmax_pooled_prefill_topk: oracle_topk (Figure 1,
+# sparsity "per Layer per Head") and post_softmax_all_heads_pooled_oracle_topk
+# (Figure 3).  The Abstract calls head-aware selection critical, which is the
+# contrast these variants show.  Readings (the page names the strategies and
+# nothing more):
+#
+# * "gqa"  (default): one problem per kv head h pools the post-softmax
+#   probabilities of its G query heads, as everything above;
+# * "head" (oracle_topk): one problem per query head qh, no pooling across
+#   heads; in prefill the tile-level constraint still holds, so the problem
+#   pools the rows of query tile t of that one head;
+# * "all"  (all heads pooled): one problem per batch row (and tile) pools
+#   every query head of every kv head, each scored against its own kv head's
+#   keys; all heads then share the one index set ("head-unaware").
+# A reuse layer in "head" mode maps query heads to anchor query heads
+# (head_map over [0, Hq)); in "all" mode every head reads the batch's single
+# list.
+
+MODES = ("gqa", "head", "all")
+
+
+def selection_heads(hq: int, hkv: int, mode: str) -> list[list[int]]:
+    """The query heads each selection problem of one batch row pools, in
+    problem order (gqa: Hkv problems, head: Hq, all: 1)."""
+    g_size = hq // hkv
+    if mode == "gqa":
+        return [list(range(h * g_size, (h + 1) * g_size)) for h in range(hkv)]
+    if mode == "head":
+        return [[qh] for qh in range(hq)]
+    if mode == "all":
+        return [list(range(hq))]
+    raise ValueError(mode)
+
+
+def pooled_decode_heads(q: np.ndarray, k: np.ndarray, b: int, heads) -> np.ndarray:
+    """P[j] = mean over the listed query heads qh of
+    softmax_j(q_qh . k_{qh // G, j} / sqrt(d)), j < N (decode)."""
+    hq, hkv, n_ctx = q.shape[1], k.shape[1], k.shape[2]
+    g_size = hq // hkv
+    total = np.zeros(n_ctx, dtype=F64)
+    for qh in heads:
+        s = scores(q[b, qh, 0:1, :], k[b, qh // g_size])
+        total += masked_softmax(s, np.ones_like(s, dtype=bool))[0]
+    return total / len(heads)
+
+
+def pooled_prefill_tile_heads(q: np.ndarray, k: np.ndarray, b: int, heads, t: int,
+                              tile: int) -> np.ndarray:
+    """Pooled post-softmax scores of query tile t over the listed query
+    heads: candidates j < e_t, row i sees j <= i, each head scored against
+    its own kv head's keys, sum over heads and rows divided by
+    len(heads) * rows_t."""
+    hq, hkv, n_ctx = q.shape[1], k.shape[1], k.shape[2]
+    g_size = hq // hkv
+    i0 = t * tile
+    i1 = min(i0 + tile, n_ctx)
+    e_t = i1
+    pos = np.arange(i0, i1)
+    visible = np.arange(e_t)[None, :] <= pos[:, None]
+    total = np.zeros(e_t, dtype=F64)
+    for qh in heads:
+        s = scores(q[b, qh, i0:i1, :], k[b, qh // g_size, :e_t, :])
+        total += masked_softmax(s, visible).sum(axis=0)
+    return total / (len(heads) * (i1 - i0))
+
+
+def anchor_select_decode_mode(q: np.ndarray, k: np.ndarray, frac_num: int, frac_den: int, mode: str):
+    """Anchor decode selection in a head-selection mode: idx
+    [B, problems, kk] (ascending) and pooled [B, problems, N]."""
+    bsz, n_ctx = k.shape[0], k.shape[2]
+    groups = selection_heads(q.shape[1], k.shape[1], mode)
+    kk = topk_count(n_ctx, frac_num, frac_den)
+    idx = np.zeros((bsz, len(groups), kk), dtype=np.int64)
+    pooled = np.zeros((bsz, len(groups), n_ctx), dtype=F64)
+    for b in range(bsz):
+        for p, heads in enumerate(groups):
+            pooled[b, p] = pooled_decode_heads(q, k, b, heads)
+            idx[b, p] = select_topk(pooled[b, p], kk)
+    return idx, pooled
+
+
+def anchor_select_prefill_tile_mode(q, k, b, p, t, tile, frac_num, frac_den, mode):
+    """Anchor prefill in a head-selection mode, problem p of batch row b and
+    tile t: (ascending idx of k_t keys, pooled)."""
+    heads = selection_heads(q.shape[1], k.shape[1], mode)[p]
+    pooled = pooled_prefill_tile_heads(q, k, b, heads, t, tile)
+    return select_topk(pooled, topk_count(pooled.shape[0], frac_num, frac_den)), pooled
+
+
+def _list_of_head(qh: int, hq: int, hkv: int, mode: str, head_map) -> int:
+    """Which anchor list query head qh reads in a reuse (or anchor) layer."""
+    g_size = hq // hkv
+    if mode == "all":
+        return 0
+    own = qh if mode == "head" else qh // g_size
+    return own if head_map is None else int(head_map[own])
+
+
+def sparse_decode_mode(q, k, v, idx, mode, head_map=None):
+    """Decode attention in a head-selection mode: query head qh attends over
+    list idx[b, L(qh)] of its own kv head's keys, L(qh) = head_map[qh // G]
+    (gqa), head_map[qh] (head) or 0 (all); head_map None = identity."""
+    bsz, hq, _, d = q.shape
+    hkv = k.shape[1]
+    g_size = hq // hkv
+    o = np.zeros((bsz, hq, d), dtype=F64)
+    lse = np.zeros((bsz, hq), dtype=F64)
+    for b in range(bsz):
+        for qh in range(hq):
+            sel = np.asarray(idx[b, _list_of_head(qh, hq, hkv, mode, head_map)], dtype=np.int64)
+            h = qh // g_size
+            vis = np.ones((1, sel.shape[0]), dtype=bool)
+            ob, lb = sparse_attend(q[b, qh, 0:1, :], k[b, h, sel], v[b, h, sel], vis)
+            o[b, qh], lse[b, qh] = ob[0], lb[0]
+    return o, lse
+
+
+def sparse_prefill_tile_mode(q, k, v, lists, b, t, tile, mode, head_map=None):
+    """Prefill attention of query tile t in a head-selection mode: query
+    head qh's rows i attend over the keys j <= i of list
+    lists[L(qh)] (L as in sparse_decode_mode; lists[p] is tile t's list of
+    problem p of batch row b).  Returns o [Hq, rows_t, d], lse [Hq, rows_t]."""
+    hq, hkv, n_ctx = q.shape[1], k.shape[1], k.shape[2]
+    g_size = hq // hkv
+    i0 = t * tile
+    i1 = min(i0 + tile, n_ctx)
+    pos = np.arange(i0, i1)
+    o = np.zeros((hq, i1 - i0, q.shape[-1]), dtype=F64)
+    lse = np.zeros((hq, i1 - i0), dtype=F64)
+    for qh in range(hq):
+        sel = np.asarray(lists[_list_of_head(qh, hq, hkv, mode, head_map)], dtype=np.int64)
+        h = qh // g_size
+        vis = sel[None, :] <= pos[:, None]
+        o[qh], lse[qh] = sparse_attend(q[b, qh, i0:i1, :], k[b, h, sel], v[b, h, sel], vis)
+    return o, lse
