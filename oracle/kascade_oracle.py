@@ -54,7 +54,7 @@ __all__ = [
     "check_index_set",
     "MODES", "selection_heads", "pooled_decode_heads", "pooled_prefill_tile_heads",
     "anchor_select_decode_mode", "anchor_select_prefill_tile_mode", "sparse_decode_mode",
-    "sparse_prefill_tile_mode",
+    "sparse_prefill_tile_mode", "refine_select_decode",
 ]
 
 
@@ -429,3 +429,40 @@ def sparse_prefill_tile_mode(q, k, v, lists, b, t, tile, mode, head_map=None):
         vis = sel[None, :] <= pos[:, None]
         o[qh], lse[qh] = sparse_attend(q[b, qh, i0:i1, :], k[b, h, sel], v[b, h, sel], vis)
     return o, lse
+
+
+# ---------------------------------------------------------------------------
+# proposal-refine reuse (decode)
+#
+# The Prism Attention page (abstract; the captions of Figures 2 and 3 and of
+# Table 9) replaces rigid reuse with a coarse-to-fine step: a proposal layer
+# builds an expanded pool of rho * kappa candidate indices, and each refined
+# layer picks its own top-kappa from the pool of its nearest preceding
+# proposal layer.  Readings (the page's algorithm listing is not in the text):
+# the pool is the proposal layer's own exact Top-(rho kappa) selection, i.e.
+# anchor_select_decode with that budget; a refined layer scores only the
+# pool's keys, so its post-softmax probabilities are taken over the pool; they
+# are pooled over the GQA group as in an anchor layer (head-aware, Kascade
+# README Abstract), and the kappa largest win, lowest index on ties, listed
+# ascending.  kv head h of the refined layer reads pool head_map[h].
+
+
+def refine_select_decode(q: np.ndarray, k: np.ndarray, pool, kappa: int, head_map=None):
+    """Refined layer: idx [B, Hkv, kappa] (ascending key indices) and the
+    pooled scores [B, Hkv, pool_len] of the pool's keys, in pool order."""
+    bsz, hq = q.shape[0], q.shape[1]
+    hkv = k.shape[1]
+    g_size = hq // hkv
+    pool = np.asarray(pool, dtype=np.int64)
+    n = pool.shape[-1]
+    hm = np.arange(hkv) if head_map is None else np.asarray(head_map)
+    idx = np.zeros((bsz, hkv, kappa), dtype=np.int64)
+    pooled = np.zeros((bsz, hkv, n), dtype=F64)
+    for b in range(bsz):
+        for h in range(hkv):
+            cand = pool[b, hm[h]]
+            s = scores(q[b, h * g_size:(h + 1) * g_size, 0, :], k[b, h, cand])
+            pooled[b, h] = masked_softmax(s, np.ones_like(s, dtype=bool)).mean(axis=0)
+            pos = select_topk(pooled[b, h], kappa)
+            idx[b, h] = cand[pos]
+    return idx, pooled

@@ -2,7 +2,10 @@
 oracle_topk strategy; all heads pooled, the head-unaware strategy): exact
 closed forms for Q = 0, linearity of the post-softmax mean across the three
 poolings, per-head selection by raw score (softmax is monotone), the
-special cases where two modes coincide, and frac = 1 against torch's SDPA."""
+special cases where two modes coincide, and frac = 1 against torch's SDPA.
+Also the proposal-refine selection: the whole context as the pool gives the
+anchor selection, a pool of kappa keys is returned as is, Q = 0 takes the
+lowest pool entries, and brute force over a small pool (softmax by torch)."""
 from fractions import Fraction
 
 import numpy as np
@@ -164,3 +167,53 @@ def test_frac_one_modes_equal_sdpa(mode):
         lists = [O.anchor_select_prefill_tile_mode(qp, kp, 0, p, t, 32, 1, 1, mode)[0] for p in range(n_prob)]
         op, _ = O.sparse_prefill_tile_mode(qp, kp, vp, lists, 0, t, 32, mode)
         assert np.allclose(op, refp[0, :, 32 * t:min(32 * t + 32, N)], rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- proposal-refine reuse
+
+
+def test_refine_over_the_whole_context_is_the_anchor_selection():
+    B, Hq, Hkv, N, d = 2, 8, 2, 90, 16
+    q, k, _ = _qkv(B, Hq, Hkv, 1, N, d)
+    kk = O.topk_count(N, 10, 100)
+    pool = np.tile(np.arange(N), (B, Hkv, 1))
+    idx, pooled = O.refine_select_decode(q, k, pool, kk)
+    want, wp = O.anchor_select_decode(q, k, 10, 100)
+    assert (idx == want).all() and np.allclose(pooled, wp, rtol=1e-14, atol=0)
+
+
+def test_refine_with_a_pool_of_kappa_returns_the_pool():
+    B, Hq, Hkv, N, d = 1, 4, 2, 50, 8
+    q, k, _ = _qkv(B, Hq, Hkv, 1, N, d)
+    pool = np.stack([[np.sort(RNG.choice(N, 7, replace=False)) for _ in range(Hkv)] for _ in range(B)])
+    idx, _ = O.refine_select_decode(q, k, pool, 7)
+    assert (idx == pool).all()
+
+
+def test_refine_q_zero_takes_the_lowest_pool_entries():
+    """Q = 0: uniform over the pool, so ties everywhere and the kappa lowest
+    key indices of the pool win."""
+    B, Hq, Hkv, N, d = 1, 4, 2, 64, 8
+    q = np.zeros((B, Hq, 1, d))
+    k = RNG.standard_normal((B, Hkv, N, d))
+    pool = np.stack([[np.sort(RNG.choice(N, 20, replace=False)) for _ in range(Hkv)] for _ in range(B)])
+    idx, pooled = O.refine_select_decode(q, k, pool, 5, head_map=[1, 0])
+    assert np.allclose(pooled, 1.0 / 20, rtol=0, atol=1e-15)
+    assert (idx[0, 0] == pool[0, 1, :5]).all() and (idx[0, 1] == pool[0, 0, :5]).all()
+
+
+def test_refine_brute_force_pool_mass():
+    """The refined set maximises the pooled mass (softmax over the pool) over
+    all kappa-subsets of a small pool; ties go to lower key indices."""
+    import itertools
+    B, Hq, Hkv, N, d = 1, 4, 1, 40, 4
+    for trial in range(5):
+        q, k, _ = _qkv(B, Hq, Hkv, 1, N, d)
+        cand = np.sort(RNG.choice(N, 10, replace=False))
+        # pooled over the pool, computed independently with torch
+        qt = torch.from_numpy(q[0, :, 0])
+        kt = torch.from_numpy(k[0, 0, cand])
+        p = torch.softmax(qt @ kt.T / np.sqrt(d), dim=-1).mean(0).numpy()
+        best = max(itertools.combinations(range(10), 3), key=lambda sub: (round(sum(p[list(sub)]), 15), [-i for i in sub]))
+        idx, _ = O.refine_select_decode(q, k, cand[None, None, :], 3)
+        assert idx[0, 0].tolist() == cand[list(best)].tolist()
