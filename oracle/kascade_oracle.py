@@ -54,7 +54,7 @@ __all__ = [
     "check_index_set",
     "MODES", "selection_heads", "pooled_decode_heads", "pooled_prefill_tile_heads",
     "anchor_select_decode_mode", "anchor_select_prefill_tile_mode", "sparse_decode_mode",
-    "sparse_prefill_tile_mode", "refine_select_decode",
+    "sparse_prefill_tile_mode", "refine_select_decode", "index_overlap", "plan_anchors",
 ]
 
 
@@ -466,3 +466,55 @@ def refine_select_decode(q: np.ndarray, k: np.ndarray, pool, kappa: int, head_ma
             pos = select_topk(pooled[b, h], kappa)
             idx[b, h] = cand[pos]
     return idx, pooled
+
+
+# ---------------------------------------------------------------------------
+# anchor-layer selection
+#
+# README, Abstract: the anchor layers are chosen by a dynamic program that
+# maximises cross-layer similarity over a development set ("--run_type
+# select_layers", Reproducibility, Figure 4).  Readings: the similarity of a
+# layer l to an earlier layer a is the overlap of their Top-k index sets,
+# |S_a and S_l| / k, averaged over batch rows, lists and tiles (a layer's
+# similarity to itself is 1); a plan of M anchors always contains layer 0
+# (the first layer has nothing to reuse) and every other layer reuses its
+# nearest preceding anchor; the objective is the sum over layers of the
+# similarity to the anchor it reuses.  Among equal objectives the plan with
+# the lexicographically smallest anchor list wins.
+
+
+def index_overlap(a, b) -> int:
+    """|A and B| for two index lists."""
+    return int(np.intersect1d(np.asarray(a), np.asarray(b)).size)
+
+
+def plan_anchors(sim, n_anchors: int):
+    """Best plan for a similarity matrix sim[a][l] (a <= l used): returns
+    (anchors ascending, objective).  The recursion: best(m, j) is the best
+    objective of layers j.. when layer j is an anchor and m more anchors
+    follow it; with none, layers j.. reuse j; otherwise the next anchor i is
+    chosen (smallest i among equal objectives)."""
+    sim = np.asarray(sim, dtype=F64)
+    n = sim.shape[0]
+    if not 1 <= n_anchors <= n:
+        raise ValueError("need 1 <= anchors <= layers")
+    memo = {}
+
+    def best(m, j):
+        key = (m, j)
+        if key in memo:
+            return memo[key]
+        if m == 0:
+            res = (float(sim[j, j:].sum()), (j,))
+        else:
+            res = None
+            for i in range(j + 1, n - m + 1):
+                val, plan = best(m - 1, i)
+                tot = float(sim[j, j:i].sum()) + val
+                if res is None or tot > res[0]:
+                    res = (tot, (j,) + plan)
+        memo[key] = res
+        return res
+
+    val, plan = best(n_anchors - 1, 0)
+    return list(plan), val

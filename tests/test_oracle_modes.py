@@ -217,3 +217,55 @@ def test_refine_brute_force_pool_mass():
         best = max(itertools.combinations(range(10), 3), key=lambda sub: (round(sum(p[list(sub)]), 15), [-i for i in sub]))
         idx, _ = O.refine_select_decode(q, k, cand[None, None, :], 3)
         assert idx[0, 0].tolist() == cand[list(best)].tolist()
+
+
+# ---------------------------------------------------------------- anchor-layer selection
+
+
+def _brute_plan(sim, m):
+    """Exhaustive: every anchor set containing layer 0; each layer reuses its
+    nearest preceding anchor; best total, lexicographically smallest set on
+    ties."""
+    import itertools
+    n = sim.shape[0]
+    best = None
+    for rest in itertools.combinations(range(1, n), m - 1):
+        anchors = (0,) + rest
+        tot = 0.0
+        for l in range(n):
+            a = max(x for x in anchors if x <= l)
+            tot += sim[a, l]
+        if best is None or tot > best[1] + 1e-12 or (abs(tot - best[1]) <= 1e-12 and anchors < best[0]):
+            best = (anchors, tot)
+    return list(best[0]), best[1]
+
+
+@pytest.mark.parametrize("n,m", [(6, 1), (6, 2), (7, 3), (8, 4), (9, 9), (10, 3)])
+def test_plan_anchors_brute_force(n, m):
+    for trial in range(4):
+        sim = np.triu(RNG.random((n, n)))
+        np.fill_diagonal(sim, 1.0)
+        got = O.plan_anchors(sim, m)
+        want = _brute_plan(sim, m)
+        assert got[0] == want[0] and abs(got[1] - want[1]) < 1e-12
+
+
+def test_plan_anchors_closed_forms():
+    # identical layers: any plan scores n; the smallest anchor set wins
+    sim = np.ones((5, 5))
+    assert O.plan_anchors(sim, 3) == ([0, 1, 2], 5.0)
+    # two blocks of mutually similar layers: the second block's first layer
+    sim = np.zeros((6, 6))
+    sim[:3, :3] = 1.0
+    sim[3:, 3:] = 1.0
+    assert O.plan_anchors(sim, 2) == ([0, 3], 6.0)
+    # every layer its own anchor
+    assert O.plan_anchors(np.eye(4), 4) == ([0, 1, 2, 3], 4.0)
+    with pytest.raises(ValueError):
+        O.plan_anchors(np.eye(3), 0)
+
+
+def test_index_overlap_counts():
+    assert O.index_overlap([1, 3, 5, 7], [0, 3, 4, 7, 9]) == 2
+    assert O.index_overlap([], [1, 2]) == 0
+    assert O.index_overlap(np.arange(10), np.arange(5, 20)) == 5
