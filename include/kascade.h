@@ -13,24 +13,28 @@
  *
  * Conventions shared by every call
  * --------------------------------
- * Tensors are dense, row-major, bf16 unless stated:
+ * Tensors are dense, row-major, bf16 (or the shape's KASCADE_DTYPE_*):
  *   q   [B, Hq,  L, d]   L = q_len (1 in decode, N in prefill)
  *   k,v [B, Hkv, N, d]   one contiguous [N, d] slab per (batch, kv head)
- *   o   [B, Hq,  L, d]   bf16 output
+ *   o   [B, Hq,  L, d]   output, the input type
  *   lse [B, Hq,  L]      fp32 natural-log softmax denominator of the scaled
  *                        scores (may be NULL); -inf for a row that sees no key
  * Query head qh belongs to kv head qh / G, G = Hq / Hkv.  Scores are
  * q.k / sqrt(d).
  *
- * Index sets (int32, ascending within each list):
- *   decode  idx [B, Hkv, K]          K = ceil(frac * N)
- *   prefill idx [B, Hkv, S]          S = sum_t k_t, k_t = ceil(frac * e_t),
+ * Index sets (int32, ascending within each list), L lists per batch row
+ * (L = Hkv in the default GQA mode; see KASCADE_SELECT_*):
+ *   decode  idx [B, L, K]            K = ceil(frac * N)
+ *   prefill idx [B, L, S]            S = sum_t k_t, k_t = ceil(frac * e_t),
  *                                    e_t = min(32 (t+1), N); the list of tile t
  *                                    starts at offsets[t] (kascade_index_offsets)
  *
  * Ownership: the caller owns every buffer (device memory for tensors, index
  * lists and the workspace; host memory for kascade_shape and offsets).  The
- * library never allocates or frees memory and keeps no state between calls.
+ * library never allocates or frees memory and keeps no state between calls,
+ * with one exception: kascade_select_decode_static (below) runs on a fixed
+ * __device__ array inside the library image, which every GPU that loads the
+ * library holds and which keeps the last such call's contents.
  * All device work is enqueued on `stream` (a cudaStream_t; NULL = legacy
  * default stream) and is asynchronous: results are ready when the stream is.
  *
@@ -38,12 +42,13 @@
  * least kascade_workspace_bytes(shape, op) bytes, 256-byte aligned.  Its
  * first int is the device error word: kernels never trap or wait without
  * bound, and a bounded wait that gives up stores a non-zero code there
- * (read it with kascade_workspace_error).  Zero the workspace once before
- * first use (kascade_workspace_init); nothing else depends on its initial
- * contents.  The attention calls need only this 256-byte header (their
- * partial results stay on chip) and accept ws = NULL, in which case no error
- * word is kept.  One workspace sized for the largest op serves every call of
- * a shape; calls that may run concurrently must not share a workspace.
+ * (read it with kascade_workspace_error; codes KASCADE_DEVERR_* below).
+ * Zero the workspace once before first use (kascade_workspace_init);
+ * nothing else depends on its initial contents.  The attention calls need
+ * only this 256-byte header (their partial results stay on chip) and accept
+ * ws = NULL, in which case no error word is kept.  One workspace sized for
+ * the largest op serves every call of a shape; calls that may run
+ * concurrently must not share a workspace.
  *
  * Errors: every call returns KASCADE_OK (0) or a status below; argument
  * errors are detected on the host before anything is launched.  No kernel
@@ -68,16 +73,29 @@ extern "C" {
 
 #define KASCADE_OK 0
 #define KASCADE_ERR_INVALID_ARG 1  /* null pointer, bad dims, Hq % Hkv != 0, frac outside (0,1] */
-#define KASCADE_ERR_UNSUPPORTED 2  /* d not 64/128, tile != 32, G > 8, q_len not 1 or N, misaligned pointer */
+#define KASCADE_ERR_UNSUPPORTED 2  /* d not 64/128, tile != 32, G > 8, q_len not 1 or N, misaligned pointer,
+                                      dtype not built, all-heads mode with Hq > 64 */
 #define KASCADE_ERR_WORKSPACE 3    /* ws NULL, misaligned or smaller than kascade_workspace_bytes() */
 #define KASCADE_ERR_CUDA 4         /* a CUDA launch or device query failed */
 #define KASCADE_ERR_TOO_LARGE 5    /* the shape needs more scratch than a fixed library buffer holds */
+
+/* Codes a kernel stores in the device error word when one of its bounded
+ * waits (about 2^32 SM clocks, a few seconds) gives up.  The kernel records
+ * the code, carries on without the missing data and finishes; the call's
+ * outputs are then not valid.  The word keeps the last code written until it
+ * is cleared. */
+#define KASCADE_DEVERR_NONE 0
+#define KASCADE_DEVERR_SCORE_POOL 2      /* prefill scoring: a TMA or MMA stage never completed */
+#define KASCADE_DEVERR_DECODE_MERGE 3    /* sparse decode: a peer CTA's partial never arrived */
+#define KASCADE_DEVERR_PREFILL_ATTN 4    /* sparse prefill: a gather or MMA stage never completed */
+#define KASCADE_DEVERR_DECODE_SELECT 5   /* decode selection: a cluster exchange never completed */
 
 /* Operations for kascade_workspace_bytes(). */
 #define KASCADE_OP_SELECT 0
 #define KASCADE_OP_SPARSE_DECODE 1
 #define KASCADE_OP_SPARSE_PREFILL 2
 #define KASCADE_OP_DENSE 3
+#define KASCADE_OP_REFINE 4   /* kascade_refine_select, any pool length up to N */
 
 typedef struct kascade_shape {
   int32_t batch;        /* B  >= 1 */
@@ -90,7 +108,37 @@ typedef struct kascade_shape {
   int32_t topk_num;     /* frac = topk_num / topk_den, 0 < frac <= 1, */
   int32_t topk_den;     /*   e.g. 10/100 for the README's Top-k of 10 % */
   int32_t flags;        /* KASCADE_FLAG_* bits, 0 for plain stream ordering */
+  int32_t select_mode;  /* KASCADE_SELECT_*: which query heads a selection pools */
+  int32_t dtype;        /* KASCADE_DTYPE_*: element type of q, k, v and o */
 } kascade_shape;
+
+/* Head-selection modes (README, Reproducibility: the default strategy
+ * post_softmax_pooled_prefill_topk beside oracle_topk, Figure 1, and
+ * post_softmax_all_heads_pooled_oracle_topk, Figure 3; the Abstract calls
+ * head-aware selection critical for accuracy).  The mode fixes the index
+ * lists per batch row, L, and what head_map maps:
+ *   GQA       L = Hkv: list h pools the G query heads of kv head h (default);
+ *             head_map [Hkv] maps kv heads to anchor kv heads.
+ *   PER_HEAD  L = Hq: list qh is query head qh's own selection (no pooling
+ *             across heads; in prefill still pooled over the 32-row tile);
+ *             head_map [Hq] maps query heads to anchor query heads.
+ *   ALL_HEADS L = 1: one list per batch row pools every query head, each
+ *             scored against its own kv head (head-unaware); every head of
+ *             every layer reads it and head_map is ignored.  Hq <= 64.
+ * Index buffers are [B, L, K] (decode) or [B, L, sum_t k_t] (prefill). */
+#define KASCADE_SELECT_GQA 0
+#define KASCADE_SELECT_PER_HEAD 1
+#define KASCADE_SELECT_ALL_HEADS 2
+
+/* Element types of q, k, v and o (lse is always fp32).  BF16 runs the
+ * tensor-core kernels.  FP32 and FP16 run a CUDA-core path: selection scores
+ * with fp64 products, attention in fp32, results rounded once to the output
+ * type (fp32 outputs within 1e-4 of exact attention over the selected keys);
+ * built for correctness, not for the bf16 path's speed.  (The README's own
+ * kernels take fp16 only, Running Evaluations.) */
+#define KASCADE_DTYPE_BF16 0
+#define KASCADE_DTYPE_F32 1
+#define KASCADE_DTYPE_F16 2
 
 /* Launch the call's kernels with programmatic dependent launch: a kernel may
  * begin (set-up only) while the previous kernel on the stream finishes; it
@@ -107,6 +155,13 @@ typedef struct kascade_shape {
  * stream wrote any of those inputs (e.g. the anchor layer's own call right
  * after kascade_select). */
 #define KASCADE_FLAG_INPUTS_STABLE 2
+/* Test only, for checking failure reporting: the prefill scoring kernel of
+ * kascade_select announces each CTA's first query-tile load but never issues
+ * it.  The waits on that load give up after their bound (a few seconds),
+ * the kernel finishes without further waiting, the workspace error word
+ * reads KASCADE_DEVERR_SCORE_POOL and the call's outputs are not valid.  No
+ * other call reads the flag. */
+#define KASCADE_FLAG_TEST_DROP_LOAD (1 << 30)
 
 /* Bytes of workspace that `op` needs for `shape` (0 on an invalid shape). */
 KASCADE_API size_t kascade_workspace_bytes(const kascade_shape* shape, int op);
@@ -120,8 +175,9 @@ KASCADE_API size_t kascade_workspace_bytes(const kascade_shape* shape, int op);
  * The pages describe no such call; it exists for callers that size graphs. */
 KASCADE_API int kascade_launch_count(const kascade_shape* shape, int op);
 
-/* Number of int32 entries of the index buffer: B * Hkv * K (decode) or
- * B * Hkv * sum_t k_t (prefill).  Returns -1 on an invalid shape. */
+/* Number of int32 entries of the index buffer: B * L * K (decode) or
+ * B * L * sum_t k_t (prefill), L the lists per batch row of the shape's
+ * select_mode.  Returns -1 on an invalid shape. */
 KASCADE_API int64_t kascade_index_count(const kascade_shape* shape);
 
 /* Host-side: writes T+1 int64 tile offsets (T = ceil(N/32)) of one
@@ -137,10 +193,11 @@ KASCADE_API int kascade_workspace_init(void* ws, size_t ws_bytes, void* stream);
  * Anchor-layer selection (README Abstract: "exact Top-k indices ... in a
  * small set of anchor layers"; strategy post_softmax_pooled_prefill_topk).
  *
- * For every (b, kv head h) in decode, or (b, h, query tile t) in prefill:
- * softmax over the visible keys of every query row of h's G query heads,
- * mean of those probabilities over the rows (masked entries count as 0),
- * then the k (= ceil(frac * e)) keys with the largest pooled value among the
+ * For every (b, list l) in decode, or (b, l, query tile t) in prefill:
+ * softmax over the visible keys of every query row of the list's query heads
+ * (the G heads of kv head l by default; see KASCADE_SELECT_*), mean of those
+ * probabilities over the rows (masked entries count as 0), then the
+ * k (= ceil(frac * e)) keys with the largest pooled value among the
  * candidates [0, e), equal values going to the lower index, written in
  * ascending order to `idx` (layout above).  Selection is exact: near the
  * k-th value the pooled scores are recomputed in fp64.
@@ -151,16 +208,48 @@ KASCADE_API int kascade_select(const kascade_shape* shape, const void* q, const 
                    int32_t* idx, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Proposal-refine selection of a decode layer (Prism Attention page,
+ * abstract and the caption of Table 9: a proposal layer builds a pool of
+ * rho * kappa candidate indices and each refined layer picks its own top
+ * kappa from the pool of its nearest preceding proposal layer; an
+ * alternative to rigid reuse of one index set).
+ *
+ * kv head h scores only the keys of pool list head_map[h] (its own K rows
+ * at those positions), takes the post-softmax probabilities of each of its
+ * G query heads over the pool, pools them (mean over the G heads) and
+ * writes the k = ceil(frac * N) keys with the largest pooled value, lower
+ * index on ties, ascending, to idx [B, Hkv, k]; exact, with the same fp64
+ * band as kascade_select.
+ *   pool      device int32 [B, Hkv, pool_len], ascending key indices in
+ *             [0, N), e.g. written by kascade_select for the proposal layer
+ *             with a budget rho times this shape's (not checked on the
+ *             device)
+ *   pool_len  k <= pool_len <= N, else KASCADE_ERR_INVALID_ARG
+ *   head_map  device int32 [Hkv], entries in [0, Hkv) (an out-of-range
+ *             entry reads list 0); NULL = identity
+ *   ws        kascade_workspace_bytes(shape, KASCADE_OP_REFINE) bytes
+ * Requires q_len == 1 and the GQA selection mode (KASCADE_ERR_UNSUPPORTED
+ * otherwise); bf16 or fp32 inputs.  The refined layer then attends with
+ * kascade_sparse_decode over idx (head_map NULL).
+ */
+KASCADE_API int kascade_refine_select(const kascade_shape* shape, const void* q, const void* k,
+                                      const int32_t* pool, int32_t pool_len, const int32_t* head_map,
+                                      int32_t* idx, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Sparse decode attention of an anchor or reuse layer (README Abstract:
  * reuse layers attend over the anchor's indices; selection and reuse are
  * head-aware).  kv head h attends over the list idx[b, head_map[h]] (the
  * anchor layer's decode index buffer) and for each of its G query heads
  * writes o = softmax(q . k_S / sqrt(d)) v_S.
- *   head_map  device int32 [Hkv], entries in [0, Hkv); NULL = identity
- *             (an anchor layer attending over its own sets).  The host
- *             cannot read it, so the kernel guards it: a kv head whose entry
- *             is out of range attends over an empty list (o = 0, lse = -inf).
- *   idx       device int32 [B, Hkv, K] as written by kascade_select
+ *   head_map  device int32 [Hkv] with entries in [0, Hkv) (GQA mode), or
+ *             [Hq] with entries in [0, Hq) (per-head mode, query head qh
+ *             reads list head_map[qh]); ignored in the all-heads mode; NULL =
+ *             identity (an anchor layer attending over its own sets).  The
+ *             host cannot read it, so the kernel guards it: a head whose
+ *             entry is out of range attends over an empty list (o = 0,
+ *             lse = -inf).
+ *   idx       device int32 [B, L, K] as written by kascade_select
  *   o, lse    device outputs (lse may be NULL)
  * Requires q_len == 1.  Index values must lie in [0, N) (not checked on the
  * device; kascade_select only writes such values).
@@ -209,10 +298,43 @@ KASCADE_API int kascade_select_decode_static(const kascade_shape* shape, const v
 /* Size in bytes of the fixed scratch array of kascade_select_decode_static. */
 KASCADE_API size_t kascade_select_decode_static_max_bytes(void);
 
+/* The device error word of kascade_select_decode_static on the current
+ * device: the first int of its fixed array, which plays the role the
+ * workspace's first int plays for kascade_select.  Synchronises `stream`,
+ * stores the word (KASCADE_DEVERR_*) in *error_out and, if `clear` is
+ * non-zero, resets it.  Every static call on the device shares this word. */
+KASCADE_API int kascade_select_decode_static_error(int* error_out, int clear, void* stream);
+
 /* Synchronises `stream`, copies the device error word (the first int of
- * `ws`) to *error_out (0 = no failure; 1 = a bounded wait timed out) and, if
- * `clear` is non-zero, resets it. */
+ * `ws`) to *error_out (KASCADE_DEVERR_NONE = no failure, else the code of
+ * the kernel whose bounded wait gave up) and, if `clear` is non-zero,
+ * resets it. */
 KASCADE_API int kascade_workspace_error(const void* ws, int* error_out, int clear, void* stream);
+
+/*
+ * Anchor-layer selection (README, Abstract: the anchor layers are chosen by
+ * a dynamic program that maximises cross-layer similarity over a
+ * development set; Reproducibility, Figure 4, select_layers).
+ *
+ * kascade_index_overlap: for two index buffers a and b of one shape (layout
+ * above, ascending lists, e.g. two layers' kascade_select outputs), writes
+ * counts[p] = sum over the tiles of |a_t and b_t| for every (batch row,
+ * list) p, B * L int64 values (device memory), on `stream`.  Divided by the
+ * list length, this is the index-set overlap of the two layers.
+ *
+ * kascade_plan_anchors (host): sim is a row-major [n_layers][n_layers] host
+ * array, sim[a][l] the similarity of layer l to an earlier layer a (only
+ * a <= l is read; sim[l][l] is what an anchor scores for itself, e.g. 1).
+ * Writes the n_anchors anchor layers, ascending and always starting at layer
+ * 0, that maximise the sum over layers of sim[anchor(l)][l], anchor(l) the
+ * nearest anchor at or before l (every other layer reuses it), and the
+ * maximum to *objective (may be NULL).  Among equal sums the plan with the
+ * smallest anchor list (lexicographically) wins.  O(n_anchors * n_layers^2).
+ */
+KASCADE_API int kascade_index_overlap(const kascade_shape* shape, const int32_t* a, const int32_t* b,
+                                      int64_t* counts, void* stream);
+KASCADE_API int kascade_plan_anchors(const double* sim, int32_t n_layers, int32_t n_anchors, int32_t* anchors,
+                                     double* objective);
 
 /* Static string for a status code. */
 KASCADE_API const char* kascade_status_str(int status);

@@ -31,11 +31,30 @@ int check_shape(const kascade_shape* s) {
   if (s->topk_den > (1 << 20)) return KASCADE_ERR_UNSUPPORTED;
   if (s->q_len != 1 && s->q_len != s->kv_len) return KASCADE_ERR_UNSUPPORTED;
   if (s->q_len != 1 && s->tile != 32) return KASCADE_ERR_UNSUPPORTED;
-  if (s->flags & ~(KASCADE_FLAG_PDL | KASCADE_FLAG_INPUTS_STABLE)) return KASCADE_ERR_INVALID_ARG;
+  if (s->flags & ~(KASCADE_FLAG_PDL | KASCADE_FLAG_INPUTS_STABLE | KASCADE_FLAG_TEST_DROP_LOAD))
+    return KASCADE_ERR_INVALID_ARG;
+  if (s->select_mode < KASCADE_SELECT_GQA || s->select_mode > KASCADE_SELECT_ALL_HEADS) return KASCADE_ERR_INVALID_ARG;
+  if (s->select_mode == KASCADE_SELECT_ALL_HEADS && s->num_q_heads > 64) return KASCADE_ERR_UNSUPPORTED;
+  if (s->dtype != KASCADE_DTYPE_BF16 && s->dtype != KASCADE_DTYPE_F32 && s->dtype != KASCADE_DTYPE_F16)
+    return KASCADE_ERR_UNSUPPORTED;
   return KASCADE_OK;
 }
 
+// Problems per batch row (= index lists per row) and query heads per
+// problem of the selection (see kv_slab_of).
+int n_lists(const kascade_shape* s) {
+  switch (s->select_mode) {
+    case KASCADE_SELECT_PER_HEAD: return s->num_q_heads;
+    case KASCADE_SELECT_ALL_HEADS: return 1;
+    default: return s->num_kv_heads;
+  }
+}
+int sel_heads(const kascade_shape* s) { return s->num_q_heads / n_lists(s); }
+
 bool is_decode(const kascade_shape* s) { return s->q_len == 1; }
+// fp32 and fp16 inputs run the CUDA-core path (is_f32: either of them)
+bool is_f32(const kascade_shape* s) { return s->dtype == KASCADE_DTYPE_F32 || s->dtype == KASCADE_DTYPE_F16; }
+bool is_f16(const kascade_shape* s) { return s->dtype == KASCADE_DTYPE_F16; }
 int n_tiles(const kascade_shape* s) { return (s->kv_len + 31) / 32; }
 
 int64_t prefill_row_len(const kascade_shape* s) {
@@ -66,6 +85,7 @@ struct SelectPlan {
   float* row_m2;
   double* row_l;
   float* pooled;
+  float* pooled_all;
   float* v_scratch;
   int32_t* band_idx;
   double* band_val;
@@ -90,27 +110,51 @@ SelectPlan plan_select(const kascade_shape* s, void* ws) {
     p.s2 = cv.take<float>(B * Hq * N);
     p.m_part = cv.take<float>(B * Hq * p.splits);
     p.l_part = cv.take<double>(B * Hq * p.splits);
-    if (select_decode_cluster_ok(s->kv_len)) {
+    if (s->select_mode != KASCADE_SELECT_ALL_HEADS && !is_f32(s) && select_decode_cluster_ok(s->kv_len)) {
       p.cluster = true;
-      const size_t entries = select_decode_cluster_scratch(s->batch, s->num_kv_heads, s->kv_len);
+      const size_t entries = select_decode_cluster_scratch(s->batch, n_lists(s), s->kv_len);
       p.band_idx = cv.take<int32_t>(entries);
       p.band_val = cv.take<double>(entries);
       p.bytes = cv.off;
       return p;
     }
-    p.grid = select_grid(false, (int)(B * Hkv), kPlanSMs);
+    p.grid = select_grid(false, (int)(B * n_lists(s)), kPlanSMs);
     p.v_scratch = cv.take<float>((size_t)p.grid * n_max);
   } else {
     p.row_m2 = cv.take<float>(B * Hq * N);
     p.row_l = cv.take<double>(B * Hq * N);
-    p.pooled = cv.take<float>(B * Hkv * (size_t)pooled_row_len(s));
-    const int64_t problems = (int64_t)B * Hkv * n_tiles(s);
+    // scoring writes one pooled row per kv head (per query head in the
+    // per-head mode); the all-heads mode adds their mean per batch row
+    const size_t score_rows = s->select_mode == KASCADE_SELECT_PER_HEAD ? Hq : Hkv;
+    p.pooled = cv.take<float>(B * score_rows * (size_t)pooled_row_len(s));
+    p.pooled_all = s->select_mode == KASCADE_SELECT_ALL_HEADS ? cv.take<float>(B * (size_t)pooled_row_len(s)) : nullptr;
+    const int64_t problems = (int64_t)B * n_lists(s) * n_tiles(s);
     p.grid = select_grid(true, (int)(problems < (1 << 30) ? problems : (1 << 30)), kPlanSMs);
     p.v_scratch = nullptr;
   }
   p.band_idx = cv.take<int32_t>((size_t)p.grid * n_max);
   p.band_val = cv.take<double>((size_t)p.grid * n_max);
   p.state = cv.take<uint8_t>((size_t)p.grid * n_max);
+  p.bytes = cv.off;
+  return p;
+}
+
+// Proposal-refine selection (decode): scores of the pool's keys, split
+// statistics, and the one-CTA-per-problem Top-k over the pool.
+SelectPlan plan_refine(const kascade_shape* s, int pool_len, void* ws) {
+  SelectPlan p{};
+  Carver cv{static_cast<char*>(ws)};
+  cv.take<char>(kHeader);
+  const size_t B = s->batch, Hq = s->num_q_heads, Hkv = s->num_kv_heads, n = pool_len;
+  p.splits = (pool_len + decode_score_keys_per_split() - 1) / decode_score_keys_per_split();
+  p.s2 = cv.take<float>(B * Hq * n);
+  p.m_part = cv.take<float>(B * Hq * p.splits);
+  p.l_part = cv.take<double>(B * Hq * p.splits);
+  p.grid = select_grid(false, (int)(B * Hkv), kPlanSMs);
+  p.v_scratch = cv.take<float>((size_t)p.grid * n);
+  p.band_idx = cv.take<int32_t>((size_t)p.grid * n);
+  p.band_val = cv.take<double>((size_t)p.grid * n);
+  p.state = cv.take<uint8_t>((size_t)p.grid * n);
   p.bytes = cv.off;
   return p;
 }
@@ -168,6 +212,16 @@ AttnArgs attn_args(const kascade_shape* s, const void* q, const void* k, const v
   a.num = s->topk_num;
   a.den = s->topk_den;
   a.flags = s->flags;
+  a.Gkv = a.G;
+  a.Hp = a.Hkv;
+  a.n_lists = n_lists(s);
+  a.one_list = false;
+  if (idx && s->select_mode == KASCADE_SELECT_PER_HEAD) {   // one problem per query head
+    a.Hp = a.Hq;
+    a.G = 1;
+  } else if (idx && s->select_mode == KASCADE_SELECT_ALL_HEADS) {
+    a.one_list = true;   // every kv head reads the row's single list
+  }
   return a;
 }
 
@@ -187,6 +241,8 @@ size_t kascade_workspace_bytes(const kascade_shape* s, int op) {
     case KASCADE_OP_SPARSE_PREFILL:
     case KASCADE_OP_DENSE:
       return kHeader;   // only the error word: partial results stay on chip
+    case KASCADE_OP_REFINE:   // covers every pool length up to N
+      return is_decode(s) ? plan_refine(s, s->kv_len, nullptr).bytes : 0;
     default:
       return 0;
   }
@@ -194,7 +250,7 @@ size_t kascade_workspace_bytes(const kascade_shape* s, int op) {
 
 int64_t kascade_index_count(const kascade_shape* s) {
   if (check_shape(s)) return -1;
-  const int64_t BH = (int64_t)s->batch * s->num_kv_heads;
+  const int64_t BH = (int64_t)s->batch * n_lists(s);
   if (is_decode(s)) return BH * topk_count(s->kv_len, s->topk_num, s->topk_den);
   return BH * prefill_row_len(s);
 }
@@ -218,13 +274,15 @@ int kascade_launch_count(const kascade_shape* s, int op) {
   if (check_shape(s)) return -1;
   if (op == KASCADE_OP_SPARSE_DECODE || op == KASCADE_OP_SPARSE_PREFILL || op == KASCADE_OP_DENSE) return 1;
   if (op != KASCADE_OP_SELECT) return -1;
-  if (!is_decode(s)) return 2;
-  if (!select_decode_cluster_ok(s->kv_len)) return 2;
+  if (!is_decode(s)) return s->select_mode == KASCADE_SELECT_ALL_HEADS ? 3 : 2;
+  if (s->select_mode == KASCADE_SELECT_ALL_HEADS || is_f32(s) || !select_decode_cluster_ok(s->kv_len)) return 2;
   SelArgs a{};
   a.B = s->batch;
   a.Hq = s->num_q_heads;
   a.Hkv = s->num_kv_heads;
-  a.G = a.Hq / a.Hkv;
+  a.Hp = n_lists(s);
+  a.G = sel_heads(s);
+  a.Gkv = a.Hq / a.Hkv;
   a.D = s->head_dim;
   a.N = s->kv_len;
   return anchor_select_fused_ok(a) ? 1 : 2;
@@ -252,7 +310,9 @@ int kascade_select(const kascade_shape* s, const void* q, const void* k, int32_t
   a.B = s->batch;
   a.Hq = s->num_q_heads;
   a.Hkv = s->num_kv_heads;
-  a.G = a.Hq / a.Hkv;
+  a.Hp = n_lists(s);
+  a.G = sel_heads(s);
+  a.Gkv = a.Hq / a.Hkv;
   a.D = s->head_dim;
   a.N = s->kv_len;
   a.tile = 32;
@@ -269,6 +329,8 @@ int kascade_select(const kascade_shape* s, const void* q, const void* k, int32_t
   a.idx = idx;
   a.flags = s->flags & KASCADE_FLAG_PDL;
   a.err = err_word(ws, ws_bytes);
+  a.in_type = s->dtype;
+  const int test_flags = s->flags & KASCADE_FLAG_TEST_DROP_LOAD;
   if (is_decode(s)) {
     if (pl.cluster && anchor_select_fused_ok(a)) return cuda_status(launch_anchor_select_fused(a, st));
     DecodeScoreArgs d{};
@@ -281,10 +343,10 @@ int kascade_select(const kascade_shape* s, const void* q, const void* k, int32_t
     d.B = a.B;
     d.Hq = a.Hq;
     d.Hkv = a.Hkv;
-    d.G = a.G;
+    d.G = a.Gkv;   // scoring runs per kv head over its query heads
     d.D = a.D;
     d.N = a.N;
-    rc = cuda_status(launch_decode_score(d, st));
+    rc = cuda_status(is_f32(s) ? launch_decode_score_f32(d, is_f16(s), st) : launch_decode_score(d, st));
     if (rc) return rc;
     a.s2 = pl.s2;
     a.m_part = pl.m_part;
@@ -293,7 +355,7 @@ int kascade_select(const kascade_shape* s, const void* q, const void* k, int32_t
     if (pl.cluster) return cuda_status(launch_select_decode_cluster(a, st));
   } else {
     ScorePoolArgs sp{};
-    sp.flags = a.flags;
+    sp.flags = a.flags | test_flags;
     sp.q = a.q;
     sp.k = a.k;
     sp.row_m2 = pl.row_m2;
@@ -302,17 +364,97 @@ int kascade_select(const kascade_shape* s, const void* q, const void* k, int32_t
     sp.B = a.B;
     sp.Hq = a.Hq;
     sp.Hkv = a.Hkv;
-    sp.G = a.G;
+    sp.G = a.Gkv;   // scoring runs per kv head over its query heads
     sp.D = a.D;
     sp.N = a.N;
     sp.tile = 32;
-    rc = cuda_status(score_pool_tc_supported(sp) ? launch_score_pool_tc(sp, err_word(ws, ws_bytes), device_sms(), st)
-                                                 : launch_score_pool(sp, st));
+    sp.per_head = s->select_mode == KASCADE_SELECT_PER_HEAD;
+    rc = cuda_status(is_f32(s) ? launch_score_pool_f32(sp, is_f16(s), st)
+                     : score_pool_tc_supported(sp) ? launch_score_pool_tc(sp, err_word(ws, ws_bytes), device_sms(), st)
+                                                   : launch_score_pool(sp, st));
     if (rc) return rc;
     a.pooled = pl.pooled;
+    if (s->select_mode == KASCADE_SELECT_ALL_HEADS) {
+      rc = cuda_status(launch_pool_mean(pl.pooled, pl.pooled_all, a.B, a.Hkv, pooled_row_len(s), a.flags, st));
+      if (rc) return rc;
+      a.pooled = pl.pooled_all;
+    }
     a.row_m2 = pl.row_m2;
     a.row_l = pl.row_l;
   }
+  return cuda_status(launch_select(a, st));
+}
+
+int kascade_refine_select(const kascade_shape* s, const void* q, const void* k, const int32_t* pool,
+                          int32_t pool_len, const int32_t* head_map, int32_t* idx, void* ws, size_t ws_bytes,
+                          void* stream) {
+  int rc = check_shape(s);
+  if (rc) return rc;
+  if (!is_decode(s) || s->select_mode != KASCADE_SELECT_GQA) return KASCADE_ERR_UNSUPPORTED;
+  if (!q || !k || !pool || !idx) return KASCADE_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(idx, 4) || !aligned(pool, 4) ||
+      (head_map && !aligned(head_map, 4)))
+    return KASCADE_ERR_UNSUPPORTED;
+  const int kk = topk_count(s->kv_len, s->topk_num, s->topk_den);
+  if (pool_len < kk || pool_len > s->kv_len) return KASCADE_ERR_INVALID_ARG;
+  SelectPlan pl = plan_refine(s, pool_len, nullptr);
+  rc = check_ws(ws, ws_bytes, pl.bytes);
+  if (rc) return rc;
+  pl = plan_refine(s, pool_len, ws);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int flags = s->flags & KASCADE_FLAG_PDL;
+  DecodeScoreArgs d{};
+  d.flags = flags;
+  d.q = static_cast<const __nv_bfloat16*>(q);
+  d.k = static_cast<const __nv_bfloat16*>(k);
+  d.s2 = pl.s2;
+  d.m_part = pl.m_part;
+  d.l_part = pl.l_part;
+  d.B = s->batch;
+  d.Hq = s->num_q_heads;
+  d.Hkv = s->num_kv_heads;
+  d.G = d.Hq / d.Hkv;
+  d.D = s->head_dim;
+  d.N = pool_len;
+  d.cand = pool;
+  d.cand_map = head_map;
+  d.cand_lists = s->num_kv_heads;
+  d.n_ctx = s->kv_len;
+  rc = cuda_status(is_f32(s) ? launch_decode_score_f32(d, is_f16(s), st) : launch_decode_score(d, st));
+  if (rc) return rc;
+  SelArgs a{};
+  a.prefill = false;
+  a.B = d.B;
+  a.Hq = d.Hq;
+  a.Hkv = d.Hkv;
+  a.Hp = d.Hkv;
+  a.G = d.G;
+  a.Gkv = d.G;
+  a.D = d.D;
+  a.N = pool_len;
+  a.n_ctx = s->kv_len;
+  a.cand = pool;
+  a.cand_map = head_map;
+  a.cand_lists = s->num_kv_heads;
+  a.tile = 32;
+  a.num = s->topk_num;
+  a.den = s->topk_den;
+  a.q = d.q;
+  a.k = d.k;
+  a.s2 = pl.s2;
+  a.m_part = pl.m_part;
+  a.l_part = pl.l_part;
+  a.splits = pl.splits;
+  a.v_scratch = pl.v_scratch;
+  a.band_idx = pl.band_idx;
+  a.band_val = pl.band_val;
+  a.state = pl.state;
+  a.n_max = pool_len;
+  a.grid = pl.grid;
+  a.idx = idx;
+  a.flags = flags;
+  a.err = err_word(ws, ws_bytes);
+  a.in_type = s->dtype;
   return cuda_status(launch_select(a, st));
 }
 
@@ -329,6 +471,7 @@ int kascade_sparse_decode(const kascade_shape* s, const void* q, const void* k, 
     return KASCADE_ERR_UNSUPPORTED;
   AttnArgs a = attn_args(s, q, k, v, idx, head_map, o, lse);
   a.err = err_word(ws, ws_bytes);
+  if (is_f32(s)) return cuda_status(launch_sparse_decode_f32(a, is_f16(s), static_cast<cudaStream_t>(stream)));
   return cuda_status(launch_decode_attn(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -346,6 +489,7 @@ int kascade_sparse_prefill(const kascade_shape* s, const void* q, const void* k,
     return KASCADE_ERR_UNSUPPORTED;
   AttnArgs a = attn_args(s, q, k, v, idx, head_map, o, lse);
   a.err = err_word(ws, ws_bytes);
+  if (is_f32(s)) return cuda_status(launch_sparse_prefill_f32(a, is_f16(s), static_cast<cudaStream_t>(stream)));
   return cuda_status(launch_prefill(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -360,8 +504,12 @@ int kascade_dense_ref(const kascade_shape* s, const void* q, const void* k, cons
   AttnArgs a = attn_args(s, q, k, v, nullptr, nullptr, o, lse);
   a.err = err_word(ws, ws_bytes);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (is_decode(s)) return cuda_status(launch_decode_attn(a, st));
+  if (is_decode(s)) {
+    if (is_f32(s)) return cuda_status(launch_sparse_decode_f32(a, is_f16(s), st));
+    return cuda_status(launch_decode_attn(a, st));
+  }
   a.causal = causal != 0;
+  if (is_f32(s)) return cuda_status(launch_sparse_prefill_f32(a, is_f16(s), st));
   return cuda_status(launch_prefill(a, st));
 }
 

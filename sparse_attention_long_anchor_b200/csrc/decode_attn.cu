@@ -44,7 +44,7 @@ namespace {
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kMaxCS = 16;
-constexpr int kIdxStage = 512;      // index entries staged in shared memory
+constexpr int kIdxStage = 2048;     // index entries staged in shared memory (a 4-CTA cluster's share of 64K at 10 %)
 constexpr int kErrMergeTimeout = 3; // device error word: a merge wait gave up
 
 template <int D>
@@ -69,6 +69,8 @@ struct Lay {
   static constexpr size_t head = wts + kMaxCS * 8 * 4;     // [8] (m, l) of the whole list
   static_assert(head + 8 * 8 <= qs, "post-loop scratch must fit in the slabs");
   static_assert(recv_o % 16 == 0 && recv_ml % 8 == 0 && bar % 8 == 0, "alignment");
+  // two CTAs per SM: 228 KB per SM less 1 KB reserved per CTA
+  static_assert(total <= (228 * 1024 - 2 * 1024) / 2, "two CTAs per SM");
 };
 
 __device__ __forceinline__ float scale_from(float m_old, float m_new) {
@@ -91,22 +93,6 @@ __device__ __forceinline__ void merge_weights(int n, const float2* ml, float* w,
   if (lane == 0) *out = make_float2(M, ls);
 }
 
-// 8x8 b16 transpose across the warp: lane (g, c) passes row g, columns
-// 2c and 2c+1, and receives row 2c and 2c+1 of column g
-__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
-  uint32_t r;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(r) : "r"(x));
-  return r;
-}
-
-__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
-  uint4 r;
-  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];\n"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "r"(addr));
-  return r;
-}
-
 // kRing = false: every warp owns at most two slices (per <= 16 * 2 * kWarps),
 // all issued up front; kRing = true: the slabs are refilled two slices ahead.
 template <int D, bool kRing>
@@ -125,8 +111,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const AttnArgs
   cg::cluster_group cluster = cg::this_cluster();
   const int CS = (int)cluster.num_blocks();
   const int rank = (int)cluster.block_rank();
-  const int bh = blockIdx.y;
-  const int b = bh / a.Hkv, h = bh - b * a.Hkv;
+  const int bh = blockIdx.y;   // problem: batch row b, problem h of the row
+  const int b = bh / a.Hp, h = bh - b * a.Hp;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, c = lane & 3;
   const int G = a.G;
@@ -143,19 +129,20 @@ __global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const AttnArgs
   cluster_arrive_release();   // the matching wait comes before the first push
 
   // an out-of-range head_map entry reads as an empty list (output 0, lse -inf)
-  const int hm_raw = a.head_map ? a.head_map[h] : h;
-  const bool hm_ok = hm_raw >= 0 && hm_raw < a.Hkv;
+  const int hm_raw = a.one_list ? 0 : (a.head_map ? a.head_map[h] : h);
+  const bool hm_ok = hm_raw >= 0 && hm_raw < a.n_lists;
   const int hm = hm_ok ? hm_raw : 0;
   const int list_full = a.idx ? topk_count(a.N, a.num, a.den) : a.N;
   const int list_len = hm_ok ? list_full : 0;
-  const int32_t* list = a.idx ? a.idx + (size_t)(b * a.Hkv + hm) * list_full : nullptr;
+  const int32_t* list = a.idx ? a.idx + (size_t)(b * a.n_lists + hm) * list_full : nullptr;
   const int c0 = min(list_len, rank * per);
   const int c1 = min(list_len, c0 + per);
   const int n_slices = (c1 - c0 + 15) / 16;
   int* idx_s = reinterpret_cast<int*>(smem + L::idx);
   const bool staged = list != nullptr && (c1 - c0) <= kIdxStage;
-  const __nv_bfloat16* kb = a.k + (size_t)bh * a.N * D;
-  const __nv_bfloat16* vb = a.v + (size_t)bh * a.N * D;
+  const size_t slab = (size_t)kv_slab_of(b, h * G, a.Hkv, a.Gkv);
+  const __nv_bfloat16* kb = a.k + slab * a.N * D;
+  const __nv_bfloat16* vb = a.v + slab * a.N * D;
 
   if (staged)
     for (int i = threadIdx.x; i < c1 - c0; i += kThreads) idx_s[i] = __ldg(list + c0 + i);
@@ -524,7 +511,7 @@ cudaError_t launch_cs(const AttnArgs& a, int cs, int per, cudaStream_t stream) {
   const cudaError_t e =
       ensure_func_attrs(reinterpret_cast<const void*>(decode_attn_kernel<D, kRing>), Lay<D>::total, cs > 8);
   if (e != cudaSuccess) return e;
-  return launch_ex(decode_attn_kernel<D, kRing>, dim3(cs, a.B * a.Hkv), dim3(kThreads), Lay<D>::total, stream,
+  return launch_ex(decode_attn_kernel<D, kRing>, dim3(cs, a.B * a.Hp), dim3(kThreads), Lay<D>::total, stream,
                    (a.flags & 1) != 0, cs, a, per);
 }
 
@@ -532,7 +519,7 @@ template <int D>
 cudaError_t launch(const AttnArgs& a, cudaStream_t stream) {
   // both variants share the shared-memory size and cluster shape, so one
   // occupancy answer serves both
-  const int cs = decode_cluster_size<D, false>((long long)a.B * a.Hkv);
+  const int cs = decode_cluster_size<D, false>((long long)a.B * a.Hp);
   const int list_len = a.idx ? topk_count(a.N, a.num, a.den) : a.N;
   int per = (list_len + cs - 1) / cs;
   per = (per + 15) / 16 * 16;

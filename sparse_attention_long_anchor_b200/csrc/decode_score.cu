@@ -27,7 +27,8 @@ __global__ void __launch_bounds__(kScoreWarps * 32)
     decode_score_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                         float* __restrict__ s2, float* __restrict__ m_part,
                         double* __restrict__ l_part, int N, int Hq, int Hkv, int G, int splits,
-                        float scale2) {
+                        float scale2, const int32_t* __restrict__ cand, const int32_t* __restrict__ cand_map,
+                        int cand_lists, int n_ctx) {
   pdl_wait();
   pdl_launch_dependents();
   constexpr int CH = D / 32;
@@ -48,7 +49,14 @@ __global__ void __launch_bounds__(kScoreWarps * 32)
     for (int s = 0; s < CH; ++s) qf[s] = make_uint4(0, 0, 0, 0);
   }
 
-  const __nv_bfloat16* kbase = k + (size_t)bh * N * D;
+  const __nv_bfloat16* kbase = k + (size_t)bh * n_ctx * D;
+  // scored position r is key r, or key clist[r] of the candidate list
+  const int32_t* clist = nullptr;
+  if (cand) {
+    int hm = cand_map ? cand_map[h] : h;
+    if (hm < 0 || hm >= cand_lists) hm = 0;
+    clist = cand + (size_t)(b * cand_lists + hm) * N;
+  }
   const int j0 = split * KEYS;
   const int j1 = min(N, j0 + KEYS);
 
@@ -57,10 +65,12 @@ __global__ void __launch_bounds__(kScoreWarps * 32)
   auto load_group = [&](int it) {
     const int r0 = j0 + (it * kScoreWarps + warp) * 16 + g;
     const int r1 = r0 + 8;
+    const int k0 = r0 < j1 ? (clist ? __ldg(clist + r0) : r0) : 0;
+    const int k1 = r1 < j1 ? (clist ? __ldg(clist + r1) : r1) : 0;
 #pragma unroll
     for (int s = 0; s < CH; ++s) {
-      ra[s] = r0 < j1 ? ldg_nc_v4(kbase + (size_t)r0 * D + 32 * s + 8 * c) : make_uint4(0, 0, 0, 0);
-      rb[s] = r1 < j1 ? ldg_nc_v4(kbase + (size_t)r1 * D + 32 * s + 8 * c) : make_uint4(0, 0, 0, 0);
+      ra[s] = r0 < j1 ? ldg_nc_v4(kbase + (size_t)k0 * D + 32 * s + 8 * c) : make_uint4(0, 0, 0, 0);
+      rb[s] = r1 < j1 ? ldg_nc_v4(kbase + (size_t)k1 * D + 32 * s + 8 * c) : make_uint4(0, 0, 0, 0);
     }
   };
 
@@ -168,11 +178,14 @@ cudaError_t launch_decode_score(const DecodeScoreArgs& a, cudaStream_t stream) {
   dim3 grid(splits, a.B * a.Hkv);
   const float scale2 = kLog2e / sqrtf((float)a.D);
   const bool pdl = (a.flags & 1) != 0;
+  const int n_ctx = a.cand ? a.n_ctx : a.N;
   if (a.D == 128)
     return launch_ex(decode_score_kernel<128>, grid, dim3(kScoreWarps * 32), 0, stream, pdl, 1, a.q, a.k, a.s2,
-                     a.m_part, a.l_part, a.N, a.Hq, a.Hkv, a.G, splits, scale2);
+                     a.m_part, a.l_part, a.N, a.Hq, a.Hkv, a.G, splits, scale2, a.cand, a.cand_map, a.cand_lists,
+                     n_ctx);
   return launch_ex(decode_score_kernel<64>, grid, dim3(kScoreWarps * 32), 0, stream, pdl, 1, a.q, a.k, a.s2,
-                   a.m_part, a.l_part, a.N, a.Hq, a.Hkv, a.G, splits, scale2);
+                   a.m_part, a.l_part, a.N, a.Hq, a.Hkv, a.G, splits, scale2, a.cand, a.cand_map, a.cand_lists,
+                   n_ctx);
 }
 
 }  // namespace kascade

@@ -7,6 +7,14 @@
 
 namespace kascade {
 
+// Problems.  A selection or attention call is split into problems per batch
+// row: problem p serves query heads [p G, p G + G) and reads the keys and
+// values of kv head (p G) / Gkv (Gkv = Hq / Hkv).  GQA pooling (the default):
+// Hp = Hkv problems of G = Gkv heads.  Per query head: Hp = Hq problems of
+// G = 1 head.  All heads pooled (selection only): Hp = 1 problem of G = Hq
+// heads, whose heads read different kv heads.
+__host__ __device__ inline int kv_slab_of(int b, int qh, int Hkv, int Gkv) { return b * Hkv + qh / Gkv; }
+
 struct DecodeScoreArgs {
   const __nv_bfloat16* q;  // [B, Hq, 1, D]
   const __nv_bfloat16* k;  // [B, Hkv, N, D]
@@ -15,6 +23,13 @@ struct DecodeScoreArgs {
   double* l_part;          // [B, Hq, splits]
   int B, Hq, Hkv, G, D, N;
   int flags;
+  // proposal-refine: score only the keys of a candidate list per (b, kv
+  // head): list head_map[h] (NULL = h) of `cand` [B, cand_lists, N]; N is
+  // then the list length and n_ctx the rows of each K slab
+  const int32_t* cand;
+  const int32_t* cand_map;
+  int cand_lists;
+  int n_ctx;
 };
 int decode_score_keys_per_split();
 cudaError_t launch_decode_score(const DecodeScoreArgs& a, cudaStream_t stream);
@@ -23,6 +38,16 @@ cudaError_t launch_decode_score(const DecodeScoreArgs& a, cudaStream_t stream);
 struct SelArgs {
   bool prefill;
   int B, Hq, Hkv, G, D, N, tile, num, den;
+  int Hp;                  // problems per batch row (index lists per row)
+  int Gkv;                 // query heads per kv head
+  int in_type;             // element type of q and k: 0 bf16, 1 fp32, 2 fp16 (pointers reinterpreted)
+  // decode proposal-refine: the N candidates of problem (b, h) are the keys
+  // cand[(b * cand_lists + cand_map[h]) * N + j] (cand_map NULL = h); K slabs
+  // hold n_ctx rows and the output keeps topk_count(n_ctx) keys
+  const int32_t* cand;
+  const int32_t* cand_map;
+  int cand_lists;
+  int n_ctx;
   const __nv_bfloat16* q;  // [B, Hq, Lq, D]
   const __nv_bfloat16* k;  // [B, Hkv, N, D]
   // decode inputs
@@ -49,7 +74,7 @@ size_t select_scratch_bytes_per_cta(int n_max);
 // decode: one 8-CTA cluster per (batch, kv head) when N / 8 <= 16384 (band
 // scratch also sized for the fused kernel)
 bool select_decode_cluster_ok(int N);
-size_t select_decode_cluster_scratch(int B, int Hkv, int N);   // band entries
+size_t select_decode_cluster_scratch(int B, int problems, int N);   // band entries (problems per batch row)
 cudaError_t launch_select_decode_cluster(const SelArgs& a, cudaStream_t stream);
 // decode: fused scoring + selection (one cluster per (batch, kv head), K
 // streamed once, scores kept on chip) when the shape and device allow it
@@ -64,9 +89,10 @@ struct ScorePoolArgs {
   const __nv_bfloat16* k;  // [B, Hkv, N, D]
   float* row_m2;           // [B, Hq, N]
   double* row_l;           // [B, Hq, N]
-  float* pooled;           // [B, Hkv, sum_t e_t]
+  float* pooled;           // [B, Hkv, sum_t e_t], or [B, Hq, sum_t e_t] with per_head
   int B, Hq, Hkv, G, D, N, tile;
   int flags;
+  bool per_head;           // pool each query head on its own (no GQA mean)
 };
 cudaError_t launch_score_pool(const ScorePoolArgs& a, cudaStream_t stream);
 // tcgen05/TMEM + TMA version (G <= 4); err: device error word (may be NULL)
@@ -83,10 +109,26 @@ struct AttnArgs {
   __nv_bfloat16* o;
   float* lse;                // may be NULL
   int B, Hq, Hkv, G, D, N, tile, num, den;
+  int Hp;                    // problems per batch row (G = query heads per problem)
+  int Gkv;                   // query heads per kv head
+  int n_lists;               // index lists per batch row
+  bool one_list;             // every problem reads list 0 of its row (head_map unused)
   bool causal;               // prefill dense only
   int* err;                  // device error word (a bounded wait gave up), may be NULL
   int flags;                 // KASCADE_FLAG_* bits
 };
+// fp32- and fp16-input variants (q, k, v, o of that type behind the same
+// pointers; half = fp16): scoring with fp64 products into the bf16 path's
+// workspace layouts, then the shared Top-k; fp32 attention on CUDA cores
+cudaError_t launch_decode_score_f32(const DecodeScoreArgs& a, bool half, cudaStream_t stream);
+cudaError_t launch_score_pool_f32(const ScorePoolArgs& a, bool half, cudaStream_t stream);
+cudaError_t launch_sparse_decode_f32(const AttnArgs& a, bool half, cudaStream_t stream);
+cudaError_t launch_sparse_prefill_f32(const AttnArgs& a, bool half, cudaStream_t stream);
+
+// mean over the Hkv rows of pooled scores: out[b, x] = (1/Hkv) sum_h in[b, h, x]
+cudaError_t launch_pool_mean(const float* in, float* out, int B, int Hkv, int64_t row, int flags,
+                             cudaStream_t stream);
+
 // decode: one 16-CTA cluster per (batch, kv head), merge over DSMEM
 cudaError_t launch_decode_attn(const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill_attn(const AttnArgs& a, cudaStream_t stream);

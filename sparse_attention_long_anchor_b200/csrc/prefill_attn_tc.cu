@@ -86,19 +86,19 @@ __device__ __forceinline__ Item item_of(const AttnArgs& a, int it, int T, int RB
   const int bh = it / (RB * T);
   const int rem = it - bh * (RB * T);
   const int t = T - 1 - rem / RB, rb = rem - (rem / RB) * RB;
-  I.b = bh / a.Hkv;
-  I.h = bh - I.b * a.Hkv;
+  I.b = bh / a.Hp;
+  I.h = bh - I.b * a.Hp;        // problem of the batch row
   I.hq0 = I.h * a.G + rb * 4;   // first query head of the row block
   I.i0 = t * a.tile;
   const int e_t = min(I.i0 + a.tile, a.N);
   I.rows_t = e_t - I.i0;
   I.list = nullptr;
   if (a.idx) {
-    const int hm_raw = a.head_map ? a.head_map[I.h] : I.h;
-    const bool hm_ok = hm_raw >= 0 && hm_raw < a.Hkv;
+    const int hm_raw = a.one_list ? 0 : (a.head_map ? a.head_map[I.h] : I.h);
+    const bool hm_ok = hm_raw >= 0 && hm_raw < a.n_lists;
     const int hm = hm_ok ? hm_raw : 0;
     const int64_t row_len = tile_list_offset(T - 1, a.tile, a.num, a.den) + topk_count(a.N, a.num, a.den);
-    I.list = a.idx + (size_t)(I.b * a.Hkv + hm) * row_len + tile_list_offset(t, a.tile, a.num, a.den);
+    I.list = a.idx + (size_t)(I.b * a.n_lists + hm) * row_len + tile_list_offset(t, a.tile, a.num, a.den);
     I.list_len = hm_ok ? topk_count(e_t, a.num, a.den) : 0;
   } else {
     I.list_len = a.causal ? e_t : a.N;
@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar = [&](int slot) { return bar0 + 8u * (uint32_t)slot; };
   const int G = a.G;
   const int T = (a.N + a.tile - 1) / a.tile;
-  const int items = T * RB * a.B * a.Hkv;
+  const int items = T * RB * a.B * a.Hp;
   const bool causal = a.idx != nullptr || a.causal;
   const int heads_rb = min(4, G);   // query heads per row block
   // this pipeline's items: the CTA's share, alternating between pipelines
@@ -222,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int g = 0; g < heads_rb; ++g)
             tc::tma_load_3d(q_s + b * L::QCB + g * 4096, &mq, b * 64, I.i0, I.b * a.Hq + I.hq0 + g, bar(bQFull));
       }
-      const size_t bhoff = (size_t)(I.b * a.Hkv + I.h) * a.N * D;
+      const size_t bhoff = (size_t)kv_slab_of(I.b, I.h * a.G, a.Hkv, a.Gkv) * a.N * D;
       for (int j = 0; j < I.nb; ++j, ++n) {
         if (pf_it != it || pf_j != j) load_keys(I, j, cur);   // not prefetched (rare)
         int nx_it = -1, nx_j = 0;
@@ -498,7 +498,7 @@ cudaError_t launch_prefill_attn_tc(const AttnArgs& a, int num_sms, cudaStream_t 
   if (!tc::make_map_3d(&mq, a.q, (uint64_t)a.D, (uint64_t)a.N, (uint64_t)a.B * a.Hq, 32)) return cudaErrorInvalidValue;
   const int T = (a.N + a.tile - 1) / a.tile;
   const int RB = a.G <= 4 ? 1 : a.G / 4;
-  const long items = (long)T * RB * a.B * a.Hkv;
+  const long items = (long)T * RB * a.B * a.Hp;
   const long long ctas = (items + kSubs - 1) / kSubs;
   const int grid = (int)(ctas < num_sms ? ctas : num_sms);
   const bool pdl = (a.flags & 1) != 0;

@@ -178,7 +178,12 @@ __global__ void __launch_bounds__(kSpWarps * 32) score_pool_kernel(const ScorePo
 
   // ------------------------------------------------------------ pass 2
   const float inv_rows = 1.0f / (float)(G * rows_t);
-  float* pooled = a.pooled + (size_t)bh * (tile_pooled_offset(T - 1, a.tile) + a.N) + tile_pooled_offset(t, a.tile);
+  const float inv_rows_head = 1.0f / (float)rows_t;
+  // pooled rows: one per kv head, or one per query head (per_head: the G
+  // rows of this kv head's query heads, b Hq + h G + hh)
+  const size_t pooled_row = (size_t)(tile_pooled_offset(T - 1, a.tile) + a.N);
+  const size_t prow0 = a.per_head ? (size_t)(b * a.Hq + h * G) : (size_t)bh;
+  float* pooled = a.pooled + prow0 * pooled_row + tile_pooled_offset(t, a.tile);
   issue(0, 0);
   cp_async_commit();
   for (int blk = 0; blk < n_blk; ++blk) {
@@ -198,11 +203,13 @@ __global__ void __launch_bounds__(kSpWarps * 32) score_pool_kernel(const ScorePo
     const int j0 = blk * kSpKeys + warp * 16;
     const int jk[2] = {j0 + g, j0 + g + 8};
     float colsum[2] = {0.f, 0.f};
-    for (int rc = 0; rc < RC; ++rc) {
-#pragma unroll 4
-      for (int nt = 0; nt < 16; ++nt) {
+    // the tile's 32 rows of head hh are rows [32 hh, 32 hh + 32)
+    for (int hh = 0; hh < G; ++hh) {
+      float hsum[2] = {0.f, 0.f};
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        const int rrow = rc * 128 + nt * 8;
+        const int rrow = hh * 32 + nt * 8;
 #pragma unroll
         for (int kk = 0; kk < D / 16; kk += 2) {
           uint32_t r4[4];
@@ -216,15 +223,30 @@ __global__ void __launch_bounds__(kSpWarps * 32) score_pool_kernel(const ScorePo
           const int j = jk[e >> 1];
           const float bb = bcol[r];
           const float p = (j <= rpos[r]) ? exp2f(acc[e] * scale2 - bb) : 0.f;
-          colsum[e >> 1] += p;
+          hsum[e >> 1] += p;
         }
       }
-    }
+      if (a.per_head) {
+        // head hh alone: its own pooled row, mean over the tile's rows
+        float* prow = pooled + (size_t)hh * pooled_row;
 #pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-      colsum[hf] += __shfl_xor_sync(0xffffffffu, colsum[hf], 1);
-      colsum[hf] += __shfl_xor_sync(0xffffffffu, colsum[hf], 2);
-      if (c == 0 && jk[hf] < e_t) pooled[jk[hf]] = colsum[hf] * inv_rows;
+        for (int hf = 0; hf < 2; ++hf) {
+          hsum[hf] += __shfl_xor_sync(0xffffffffu, hsum[hf], 1);
+          hsum[hf] += __shfl_xor_sync(0xffffffffu, hsum[hf], 2);
+          if (c == 0 && jk[hf] < e_t) prow[jk[hf]] = hsum[hf] * inv_rows_head;
+        }
+      } else {
+        colsum[0] += hsum[0];
+        colsum[1] += hsum[1];
+      }
+    }
+    if (!a.per_head) {
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        colsum[hf] += __shfl_xor_sync(0xffffffffu, colsum[hf], 1);
+        colsum[hf] += __shfl_xor_sync(0xffffffffu, colsum[hf], 2);
+        if (c == 0 && jk[hf] < e_t) pooled[jk[hf]] = colsum[hf] * inv_rows;
+      }
     }
     __syncthreads();
   }

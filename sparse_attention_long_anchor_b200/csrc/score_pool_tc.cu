@@ -23,6 +23,7 @@
 //               across the groups per tile), masked column sums (pass 2).
 // All hand-offs are mbarriers; every wait is bounded and a timeout stops the
 // CTA's loops and records an error code.
+#include "../../include/kascade.h"
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -137,9 +138,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nb = (e_t + kKB - 1) / kKB;
         if (qcount > 0 && !mbar_wait_bounded(q_empty, (qcount - 1) & 1)) { fail(); break; }
         mbar_arrive_expect_tx(q_full, (uint32_t)(L::CB * G * 32 * 128));
-        for (int cb = 0; cb < L::CB; ++cb)
-          for (int g = 0; g < G; ++g)
-            tc::tma_load_3d(q_s + cb * L::CBYTES + g * 4096, &mq, cb * 64, i0, b * a.Hq + h * G + g, q_full);
+        // test switch: announce the first query tile but never load it, so
+        // the waits on it give up and report through the error word
+        if (!(qcount == 0 && (a.flags & KASCADE_FLAG_TEST_DROP_LOAD)))
+          for (int cb = 0; cb < L::CB; ++cb)
+            for (int g = 0; g < G; ++g)
+              tc::tma_load_3d(q_s + cb * L::CBYTES + g * 4096, &mq, cb * 64, i0, b * a.Hq + h * G + g, q_full);
         ++qcount;
         for (int pass = 0; pass < 2; ++pass) {
           for (int blk = 0; blk < nb; ++blk) {
@@ -303,8 +307,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       epi_bar();
       // ---- pass 2: pooled score of key j0 + r over this warpgroup's blocks
-      const float inv_rows = 1.0f / (float)(G * rows_t);
-      float* pooled = a.pooled + (size_t)bh * (tile_pooled_offset(T - 1, a.tile) + a.N) + tile_pooled_offset(t, a.tile);
+      const float inv_rows = 1.0f / (float)((a.per_head ? 1 : G) * rows_t);
+      // pooled rows: one per kv head, or with per_head one per query head
+      // (column chunk ch of the accumulator holds query head h G + ch)
+      const size_t pooled_row = (size_t)(tile_pooled_offset(T - 1, a.tile) + a.N);
+      float* pooled = a.pooled + (a.per_head ? (size_t)(b * a.Hq + h * G) : (size_t)bh) * pooled_row +
+                      tile_pooled_offset(t, a.tile);
       for (int blk = 0; blk < nb; ++blk, ++acount) {
         if (acount % kEpiGroups != wg) continue;
         const int buf = acount % kBufs;
@@ -336,11 +344,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             c0 += e0 + e1;
             c1 += e2 + e3;
           }
+          if (a.per_head) {
+            if (ch < G && j < e_t) pooled[(size_t)ch * pooled_row + j] = (c0 + c1) * inv_rows;
+            c0 = c1 = 0.f;
+          }
         }
         tc::fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_empty0 + 8 * buf);
-        if (j < e_t) pooled[j] = (c0 + c1) * inv_rows;
+        if (!a.per_head && j < e_t) pooled[j] = (c0 + c1) * inv_rows;
       }
     }
   }

@@ -492,7 +492,7 @@ __global__ void __cluster_dims__(kFallbackCS, 1, 1) __launch_bounds__(kCNT)
   const int rank = (int)cluster.block_rank();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bh = blockIdx.y;
-  const int b = bh / a.Hkv, h = bh - b * a.Hkv;
+  const int b = bh / a.Hp, h = bh - b * a.Hp;   // problem h of batch row b
   const int G = a.G, D = a.D, N = a.N;
   const int K = topk_count(N, a.num, a.den);
   const int j0 = rank * keys_per_cta;
@@ -544,7 +544,8 @@ __global__ void __cluster_dims__(kFallbackCS, 1, 1) __launch_bounds__(kCNT)
   cluster_wait();   // every CTA's exchange barriers are initialised
   cluster_topk<kFallbackCS>(cluster, sh, rx, v, st, cnt, j0, rank, K, out,
                             a.band_idx + bbase + (size_t)rank * keys_per_cta,
-                            a.band_val + bbase + (size_t)rank * keys_per_cta, qf, a.k + (size_t)bh * N * D, G, D,
+                            a.band_val + bbase + (size_t)rank * keys_per_cta, qf,
+                            a.k + (size_t)kv_slab_of(b, h * G, a.Hkv, a.Gkv) * N * D, G, D,
                             a.err);
 }
 
@@ -579,7 +580,7 @@ __global__ void __launch_bounds__(kCNT, 1) anchor_select_kernel(const SelArgs a,
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, c = lane & 3;
   const int bh = blockIdx.y;
-  const int b = bh / a.Hkv, h = bh - b * a.Hkv;
+  const int b = bh / a.Hp, h = bh - b * a.Hp;   // problem h of batch row b
   const int G = a.G, N = a.N;
   const int K = topk_count(N, a.num, a.den);
   const int j0 = rank * per;
@@ -588,7 +589,7 @@ __global__ void __launch_bounds__(kCNT, 1) anchor_select_kernel(const SelArgs a,
   uint8_t* st = reinterpret_cast<uint8_t*>(sc + (size_t)G * SCS);
   int32_t* out = a.idx + (size_t)bh * K;
   const size_t bbase = (size_t)bh * CS * per;
-  const __nv_bfloat16* kb = a.k + (size_t)bh * N * D;
+  const __nv_bfloat16* kb = a.k + (size_t)kv_slab_of(b, h * G, a.Hkv, a.Gkv) * N * D;
 
   if (K >= N) {   // everything is selected (same branch in every CTA)
     for (int i = tid; i < cnt; i += kCNT) out[j0 + i] = j0 + i;
@@ -845,7 +846,7 @@ int fused_cluster_size(const SelArgs& a) {
     active[i] = cached[dev][i] - 1;
     fits[i] = ASL<D>::bytes(a.G, fused_per(a.N, kFusedSizes[i])) <= max_smem;
   }
-  return choose_cluster_size((long long)a.B * a.Hkv, kFusedSizes, active, fits, kNumFusedSizes);
+  return choose_cluster_size((long long)a.B * a.Hp, kFusedSizes, active, fits, kNumFusedSizes);
 }
 
 template <int CS, int D>
@@ -854,7 +855,7 @@ cudaError_t launch_fused(const SelArgs& a, cudaStream_t stream) {
   const size_t smem = ASL<D>::bytes(a.G, per);
   const cudaError_t e = ensure_func_attrs(reinterpret_cast<const void*>(anchor_select_kernel<CS, D>), smem, CS > 8);
   if (e != cudaSuccess) return e;
-  return launch_ex(anchor_select_kernel<CS, D>, dim3(CS, a.B * a.Hkv), dim3(kCNT), smem, stream,
+  return launch_ex(anchor_select_kernel<CS, D>, dim3(CS, a.B * a.Hp), dim3(kCNT), smem, stream,
                    (a.flags & 1) != 0, CS, a, per);
 }
 
@@ -864,7 +865,7 @@ int select_decode_cluster_keys(int N) { return (N + kFallbackCS - 1) / kFallback
 
 bool select_decode_cluster_ok(int N) { return select_decode_cluster_keys(N) <= 16384; }
 
-size_t select_decode_cluster_scratch(int B, int Hkv, int N) {
+size_t select_decode_cluster_scratch(int B, int problems, int N) {
   // band entries for the fallback layout and both fused cluster sizes
   const size_t fb = (size_t)kFallbackCS * select_decode_cluster_keys(N);
   size_t m = fb;
@@ -872,7 +873,7 @@ size_t select_decode_cluster_scratch(int B, int Hkv, int N) {
     const size_t f = (size_t)kFusedSizes[i] * fused_per(N, kFusedSizes[i]);
     m = f > m ? f : m;
   }
-  return (size_t)B * Hkv * m;
+  return (size_t)B * problems * m;
 }
 
 cudaError_t launch_select_decode_cluster(const SelArgs& a, cudaStream_t stream) {
@@ -880,7 +881,7 @@ cudaError_t launch_select_decode_cluster(const SelArgs& a, cudaStream_t stream) 
   const size_t smem = cluster_dyn_bytes(per);
   const cudaError_t e = ensure_func_attrs(reinterpret_cast<const void*>(select_decode_cluster_kernel), smem, false);
   if (e != cudaSuccess) return e;
-  dim3 grid(kFallbackCS, a.B * a.Hkv);
+  dim3 grid(kFallbackCS, a.B * a.Hp);
   return launch_ex(select_decode_cluster_kernel, grid, dim3(kCNT), smem, stream, (a.flags & 1) != 0, 1, a, per);
 }
 

@@ -49,12 +49,12 @@ __global__ void __launch_bounds__(kPreWarps * 32)
   const int t = T - 1 - (int)(blockIdx.x / row_blocks);
   const int rb = blockIdx.x % row_blocks;
   const int bh = blockIdx.y;
-  const int b = bh / a.Hkv, h = bh - b * a.Hkv;
+  const int b = bh / a.Hp, h = bh - b * a.Hp;   // problem h of batch row b
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, c = lane & 3;
   const int G = a.G;
-  const int hm_raw = a.head_map ? a.head_map[h] : h;
-  const bool hm_ok = hm_raw >= 0 && hm_raw < a.Hkv;
+  const int hm_raw = a.one_list ? 0 : (a.head_map ? a.head_map[h] : h);
+  const bool hm_ok = hm_raw >= 0 && hm_raw < a.n_lists;
   const int hm = hm_ok ? hm_raw : 0;
   const int i0 = t * a.tile;
   const int e_t = min(i0 + a.tile, a.N);
@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(kPreWarps * 32)
   if (a.idx) {
     const int T_last = T - 1;
     const int64_t row_len = tile_list_offset(T_last, a.tile, a.num, a.den) + topk_count(a.N, a.num, a.den);
-    list = a.idx + (size_t)(b * a.Hkv + hm) * row_len + tile_list_offset(t, a.tile, a.num, a.den);
+    list = a.idx + (size_t)(b * a.n_lists + hm) * row_len + tile_list_offset(t, a.tile, a.num, a.den);
     list_len = hm_ok ? topk_count(e_t, a.num, a.den) : 0;
   } else {
     list_len = a.causal ? e_t : a.N;
@@ -95,8 +95,9 @@ __global__ void __launch_bounds__(kPreWarps * 32)
     }
   }
 
-  const __nv_bfloat16* kb = a.k + (size_t)bh * a.N * D;
-  const __nv_bfloat16* vb = a.v + (size_t)bh * a.N * D;
+  const size_t slab = (size_t)kv_slab_of(b, h * G, a.Hkv, a.Gkv);
+  const __nv_bfloat16* kb = a.k + slab * a.N * D;
+  const __nv_bfloat16* vb = a.v + slab * a.N * D;
   const uint32_t sm_u = smem_u32(smem);
   const int n_blocks = (list_len + kPreKeys - 1) / kPreKeys;
   const float scale2 = kLog2e * rsqrtf((float)D);
@@ -251,7 +252,7 @@ size_t prefill_smem() {
 cudaError_t launch_prefill_attn(const AttnArgs& a, cudaStream_t stream) {
   const int T = (a.N + a.tile - 1) / a.tile;
   const int row_blocks = (a.G * a.tile + 127) / 128;
-  dim3 grid(T * row_blocks, a.B * a.Hkv);
+  dim3 grid(T * row_blocks, a.B * a.Hp);
   if (a.D == 128) {
     const size_t sm = prefill_smem<128>();
     const cudaError_t e = ensure_func_attrs(reinterpret_cast<const void*>(prefill_attn_kernel<128>), sm, false);

@@ -19,6 +19,8 @@
 //    largest of those, lower index first on equal values.
 // 4. One ascending pass over the keys writes the selected indices with a
 //    block-wide prefix sum.
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -32,6 +34,7 @@ constexpr int kBins = 2048;
 constexpr float kBandDelta = 1.0f / 8192.0f;
 constexpr float kBandFloor = 0x1p-96f;   // below this fp32 exp2 underflow may hide mass
 constexpr int kMaxD = 128;
+constexpr int kMaxHeads = 64;   // query heads one problem may pool (all heads of a row)
 
 struct SelShared {
   unsigned hist[kBins];
@@ -39,17 +42,17 @@ struct SelShared {
   int bin, above;
   int nb, chi;
   int need_eq_ticket;
-  float m2[8];
-  double l[8];
-  float inv_l[8];
+  float m2[kMaxHeads];
+  double l[kMaxHeads];
+  float inv_l[kMaxHeads];
   int b_idx[kSelThreads];
   double b_val[kSelThreads];
 };
 
 // dynamic shared memory after SelShared (rounded up to 128 bytes): decode q
-// rows as float [8][D], then a per-warp key row as double [warps][D]
+// rows as float [heads][D], then a per-warp key row as double [warps][D]
 constexpr size_t kSelHead = (sizeof(SelShared) + 127) / 128 * 128;
-constexpr size_t kSelQ = (size_t)8 * kMaxD * 4;
+constexpr size_t kSelQ = (size_t)kMaxHeads * kMaxD * 4;
 __host__ __device__ constexpr size_t sel_dyn_bytes() {
   return kSelHead + kSelQ + (size_t)(kSelThreads / 32) * kMaxD * 8;
 }
@@ -92,18 +95,28 @@ struct Problem {
   int i0, rows;            // prefill tile rows [i0, i0 + rows)
   const float* v;          // pooled values (prefill) / scratch (decode)
   int32_t* out;
+  const int32_t* cand;     // decode refine: candidate j is key cand[j] (NULL: key j)
 };
 
+// element i of a q or k tensor of the input type (0 bf16, 1 fp32, 2 fp16)
+__device__ __forceinline__ float elem(const __nv_bfloat16* base, size_t i, int in_type) {
+  if (in_type == 1) return __ldg(reinterpret_cast<const float*>(base) + i);
+  if (in_type == 2) return __half2float(reinterpret_cast<const __half*>(base)[i]);
+  return __bfloat162float(base[i]);
+}
+
 // fp64 pooled score of key j, computed by one warp (all lanes return it).
+// Head g of the problem is query head p.h G + g, scored against its own kv
+// head's key row.
 __device__ double refine_decode(const SelArgs& a, const Problem& p, int j, const float* qf,
                                 const SelShared& sh, double c2) {
   const int lane = threadIdx.x & 31;
-  const __nv_bfloat16* krow = a.k + ((size_t)(p.b * a.Hkv + p.h) * a.N + j) * a.D;
   double total = 0.0;
   for (int g = 0; g < a.G; ++g) {
+    const int slab = kv_slab_of(p.b, p.h * a.G + g, a.Hkv, a.Gkv);
+    const size_t krow = ((size_t)slab * (p.cand ? a.n_ctx : a.N) + (p.cand ? p.cand[j] : j)) * a.D;
     double dot = 0.0;
-    for (int e = lane; e < a.D; e += 32)
-      dot += (double)qf[g * a.D + e] * (double)__bfloat162float(krow[e]);
+    for (int e = lane; e < a.D; e += 32) dot += (double)qf[g * a.D + e] * (double)elem(a.k, krow + e, a.in_type);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
     total += exp2(dot * c2 - (double)sh.m2[g]) / sh.l[g];
@@ -113,23 +126,37 @@ __device__ double refine_decode(const SelArgs& a, const Problem& p, int j, const
 
 __device__ double refine_prefill(const SelArgs& a, const Problem& p, int j, double* kbuf, double c2) {
   const int lane = threadIdx.x & 31;
-  const __nv_bfloat16* krow = a.k + ((size_t)(p.b * a.Hkv + p.h) * a.N + j) * a.D;
-  for (int e = lane; e < a.D; e += 32) kbuf[e] = (double)__bfloat162float(krow[e]);
-  __syncwarp();
   double total = 0.0;
-  const int nrows = a.G * a.tile;
-  for (int r = lane; r < nrows; r += 32) {
-    const int g = r / a.tile, il = r - g * a.tile;
-    const int i = p.i0 + il;
-    if (il >= p.rows || j > i) continue;
-    const __nv_bfloat16* qr = a.q + ((size_t)(p.b * a.Hq + p.h * a.G + g) * a.N + i) * a.D;
-    double dot = 0.0;
-    for (int e = 0; e < a.D; e += 2) {
-      const __nv_bfloat162 q2 = __ldg(reinterpret_cast<const __nv_bfloat162*>(qr + e));
-      dot += (double)__low2float(q2) * kbuf[e] + (double)__high2float(q2) * kbuf[e + 1];
+  // the problem's heads [h0, h0 + G), a run of heads per kv head: one key
+  // row per run, then the tile's rows of those heads
+  const int h0 = p.h * a.G;
+  for (int g0 = 0; g0 < a.G;) {
+    const int qh0 = h0 + g0;
+    const int run = min(a.G - g0, a.Gkv - qh0 % a.Gkv);
+    const size_t krow = ((size_t)kv_slab_of(p.b, qh0, a.Hkv, a.Gkv) * a.N + j) * a.D;
+    __syncwarp();
+    for (int e = lane; e < a.D; e += 32) kbuf[e] = (double)elem(a.k, krow + e, a.in_type);
+    __syncwarp();
+    const int nrows = run * a.tile;
+    for (int r = lane; r < nrows; r += 32) {
+      const int g = r / a.tile, il = r - g * a.tile;
+      const int i = p.i0 + il;
+      if (il >= p.rows || j > i) continue;
+      const size_t qoff = ((size_t)(p.b * a.Hq + qh0 + g) * a.N + i) * a.D;
+      double dot = 0.0;
+      if (a.in_type != 0) {
+        for (int e = 0; e < a.D; ++e) dot += (double)elem(a.q, qoff + e, a.in_type) * kbuf[e];
+      } else {
+        const __nv_bfloat16* qr = a.q + qoff;
+        for (int e = 0; e < a.D; e += 2) {
+          const __nv_bfloat162 q2 = __ldg(reinterpret_cast<const __nv_bfloat162*>(qr + e));
+          dot += (double)__low2float(q2) * kbuf[e] + (double)__high2float(q2) * kbuf[e + 1];
+        }
+      }
+      const size_t srow = (size_t)(p.b * a.Hq + qh0 + g) * a.N + i;
+      total += exp2(dot * c2 - (double)a.row_m2[srow]) / a.row_l[srow];
     }
-    const size_t srow = (size_t)(p.b * a.Hq + p.h * a.G + g) * a.N + i;
-    total += exp2(dot * c2 - (double)a.row_m2[srow]) / a.row_l[srow];
+    g0 += run;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
@@ -146,7 +173,7 @@ __device__ void run_problem(const SelArgs& a, Problem& p, SelShared& sh, float* 
 
   // fast path: everything is selected
   if (p.k >= p.n) {
-    for (int j = tid; j < p.n; j += NT) p.out[j] = j;
+    for (int j = tid; j < p.n; j += NT) p.out[j] = p.cand ? p.cand[j] : j;
     return;
   }
 
@@ -156,9 +183,9 @@ __device__ void run_problem(const SelArgs& a, Problem& p, SelShared& sh, float* 
   const float* v = p.v;
   clear_hist(sh);
   if (!a.prefill) {
-    // combine split statistics of the G query heads (fp64)
-    if (warp < a.G) {
-      const size_t row = (size_t)(p.b * a.Hq + p.h * a.G + warp) * a.splits;
+    // combine split statistics of the G query heads (fp64), a warp per head
+    for (int hw = warp; hw < a.G; hw += NT / 32) {
+      const size_t row = (size_t)(p.b * a.Hq + p.h * a.G + hw) * a.splits;
       float m = -INFINITY;
       for (int s = lane; s < a.splits; s += 32) m = fmaxf(m, a.m_part[row + s]);
 #pragma unroll
@@ -169,14 +196,14 @@ __device__ void run_problem(const SelArgs& a, Problem& p, SelShared& sh, float* 
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
       if (lane == 0) {
-        sh.m2[warp] = m;
-        sh.l[warp] = l;
-        sh.inv_l[warp] = (float)(1.0 / l);
+        sh.m2[hw] = m;
+        sh.l[hw] = l;
+        sh.inv_l[hw] = (float)(1.0 / l);
       }
     }
     for (int e = tid; e < a.G * a.D; e += NT) {
       const int g = e / a.D, dd = e - g * a.D;
-      qf[e] = __bfloat162float(a.q[(size_t)(p.b * a.Hq + p.h * a.G + g) * a.D + dd]);
+      qf[e] = elem(a.q, (size_t)(p.b * a.Hq + p.h * a.G + g) * a.D + dd, a.in_type);
     }
     __syncthreads();
     const float* srow = a.s2 + (size_t)(p.b * a.Hq + p.h * a.G) * a.N;
@@ -316,7 +343,7 @@ __device__ void run_problem(const SelArgs& a, Problem& p, SelShared& sh, float* 
     const int incl = block_inclusive_scan<NT>(c, sh.scan_buf, nullptr);
     int w = incl - c;
     for (int j = j0; j < j1; ++j)
-      if (flag_of(j)) p.out[w++] = j;
+      if (flag_of(j)) p.out[w++] = p.cand ? p.cand[j] : j;
     return;
   }
   int written = 0, ties_taken = 0;
@@ -341,7 +368,7 @@ __device__ void run_problem(const SelArgs& a, Problem& p, SelShared& sh, float* 
     }
     int total;
     const int incl = block_inclusive_scan<NT>(flag, sh.scan_buf, &total);
-    if (flag) p.out[written + incl - 1] = j;
+    if (flag) p.out[written + incl - 1] = p.cand ? p.cand[j] : j;
     written += total;
   }
 }
@@ -359,16 +386,23 @@ __global__ void __launch_bounds__(NT, kSelCtasPerSM) select_kernel(const SelArgs
   double* band_val = a.band_val + (size_t)cta * a.n_max;
   uint8_t* state = a.state + (size_t)cta * a.n_max;
 
-  const int BH = a.B * a.Hkv;
+  const int BH = a.B * a.Hp;   // problems: (batch row, problem of the row)
   if (!a.prefill) {
-    const int64_t K = topk_count(a.N, a.num, a.den);
+    // with candidates, N counts the candidates and k follows the context
+    const int64_t K = topk_count(a.cand ? a.n_ctx : a.N, a.num, a.den);
     for (int prob = cta; prob < BH; prob += gridDim.x) {
       Problem p;
-      p.b = prob / a.Hkv;
-      p.h = prob - p.b * a.Hkv;
+      p.b = prob / a.Hp;
+      p.h = prob - p.b * a.Hp;
       p.t = 0;
       p.n = a.N;
       p.k = (int)K;
+      p.cand = nullptr;
+      if (a.cand) {
+        int hm = a.cand_map ? a.cand_map[p.h] : p.h;
+        if (hm < 0 || hm >= a.cand_lists) hm = 0;
+        p.cand = a.cand + (size_t)(p.b * a.cand_lists + hm) * a.N;
+      }
       p.i0 = 0;
       p.rows = 1;
       p.v = vscr;
@@ -386,14 +420,15 @@ __global__ void __launch_bounds__(NT, kSelCtasPerSM) select_kernel(const SelArgs
       const int t = T - 1 - (int)(prob / BH);   // longest tiles first
       const int bh = (int)(prob % BH);
       Problem p;
-      p.b = bh / a.Hkv;
-      p.h = bh - p.b * a.Hkv;
+      p.b = bh / a.Hp;
+      p.h = bh - p.b * a.Hp;
       p.t = t;
       p.i0 = t * a.tile;
       p.n = min((t + 1) * a.tile, a.N);
       p.rows = p.n - p.i0;
       p.k = topk_count(p.n, a.num, a.den);
       p.v = a.pooled + (size_t)bh * pooled_len + tile_pooled_offset(t, a.tile);
+      p.cand = nullptr;
       p.out = a.idx + (size_t)bh * row_len + tile_list_offset(t, a.tile, a.num, a.den);
       run_problem<NT>(a, p, sh, vscr, band_idx, band_val, state, dyn);
       __syncthreads();
@@ -402,6 +437,27 @@ __global__ void __launch_bounds__(NT, kSelCtasPerSM) select_kernel(const SelArgs
 }
 
 }  // namespace
+
+// pooled scores of all heads: the mean over a batch row's kv-head rows (each
+// already the mean over its G query heads, so this is the mean over all Hq)
+__global__ void pool_mean_kernel(const float* __restrict__ in, float* __restrict__ out, int Hkv, int64_t row) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int b = blockIdx.y;
+  const float inv = 1.0f / (float)Hkv;
+  for (int64_t x = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; x < row; x += (int64_t)gridDim.x * blockDim.x) {
+    float acc = 0.f;
+    for (int h = 0; h < Hkv; ++h) acc += in[((int64_t)b * Hkv + h) * row + x];
+    out[(int64_t)b * row + x] = acc * inv;
+  }
+}
+
+cudaError_t launch_pool_mean(const float* in, float* out, int B, int Hkv, int64_t row, int flags,
+                             cudaStream_t stream) {
+  int blocks = (int)((row + 255) / 256);
+  if (blocks > 4096) blocks = 4096;
+  return launch_ex(pool_mean_kernel, dim3(blocks, B), dim3(256), 0, stream, (flags & 1) != 0, 1, in, out, Hkv, row);
+}
 
 size_t select_scratch_bytes_per_cta(int n_max) {
   return (size_t)n_max * (sizeof(float) + sizeof(int32_t) + sizeof(double) + 1);

@@ -14,19 +14,25 @@ import torch
 
 __all__ = ["Shape", "KascadeError", "lib", "OP_SELECT", "OP_SPARSE_DECODE", "OP_SPARSE_PREFILL",
            "OP_DENSE", "workspace_bytes", "index_count", "index_offsets", "Workspace", "select",
-           "sparse_decode", "sparse_prefill", "dense_ref", "status_str", "launch_count", "EXPORTS", "LIB_PATH"]
+           "sparse_decode", "sparse_prefill", "dense_ref", "status_str", "launch_count", "EXPORTS", "LIB_PATH",
+           "select_decode_static", "select_decode_static_error", "refine_select", "OP_REFINE",
+           "index_overlap", "plan_anchors"]
 
 LIB_PATH = os.environ.get("KASCADE_LIB") or os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkascade.so")
 
-OP_SELECT, OP_SPARSE_DECODE, OP_SPARSE_PREFILL, OP_DENSE = 0, 1, 2, 3
+OP_SELECT, OP_SPARSE_DECODE, OP_SPARSE_PREFILL, OP_DENSE, OP_REFINE = 0, 1, 2, 3, 4
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TOO_LARGE = 0, 1, 2, 3, 4, 5
-FLAG_PDL, FLAG_INPUTS_STABLE = 1, 2
+FLAG_PDL, FLAG_INPUTS_STABLE, FLAG_TEST_DROP_LOAD = 1, 2, 1 << 30
+DEVERR_SCORE_POOL, DEVERR_DECODE_MERGE, DEVERR_PREFILL_ATTN, DEVERR_DECODE_SELECT = 2, 3, 4, 5
+SELECT_GQA, SELECT_PER_HEAD, SELECT_ALL_HEADS = 0, 1, 2
+DTYPE_BF16, DTYPE_F32, DTYPE_F16 = 0, 1, 2
 
 EXPORTS = ("kascade_workspace_bytes", "kascade_index_count", "kascade_index_offsets",
            "kascade_workspace_init", "kascade_select", "kascade_sparse_decode",
            "kascade_sparse_prefill", "kascade_dense_ref", "kascade_workspace_error",
            "kascade_status_str", "kascade_select_decode_static", "kascade_select_decode_static_max_bytes",
-           "kascade_launch_count")
+           "kascade_launch_count", "kascade_select_decode_static_error", "kascade_refine_select",
+           "kascade_index_overlap", "kascade_plan_anchors")
 
 
 class KascadeError(RuntimeError):
@@ -40,15 +46,21 @@ class Shape(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("q_len", ctypes.c_int32), ("kv_len", ctypes.c_int32), ("tile", ctypes.c_int32),
-                ("topk_num", ctypes.c_int32), ("topk_den", ctypes.c_int32), ("flags", ctypes.c_int32)]
+                ("topk_num", ctypes.c_int32), ("topk_den", ctypes.c_int32), ("flags", ctypes.c_int32),
+                ("select_mode", ctypes.c_int32), ("dtype", ctypes.c_int32)]
 
     @classmethod
-    def make(cls, batch, hq, hkv, d, q_len, kv_len, frac=(10, 100), tile=32, flags=0):
-        return cls(batch, hq, hkv, d, q_len, kv_len, tile, frac[0], frac[1], flags)
+    def make(cls, batch, hq, hkv, d, q_len, kv_len, frac=(10, 100), tile=32, flags=0, mode=0, dtype=0):
+        return cls(batch, hq, hkv, d, q_len, kv_len, tile, frac[0], frac[1], flags, mode, dtype)
 
     def with_flags(self, flags: int) -> "Shape":
         return Shape(self.batch, self.num_q_heads, self.num_kv_heads, self.head_dim, self.q_len,
-                     self.kv_len, self.tile, self.topk_num, self.topk_den, flags)
+                     self.kv_len, self.tile, self.topk_num, self.topk_den, flags, self.select_mode, self.dtype)
+
+    @property
+    def n_lists(self) -> int:
+        """Index lists per batch row under the shape's selection mode."""
+        return {SELECT_PER_HEAD: self.num_q_heads, SELECT_ALL_HEADS: 1}.get(self.select_mode, self.num_kv_heads)
 
     @property
     def decode(self) -> bool:
@@ -79,8 +91,17 @@ def _load():
     so.kascade_dense_ref.restype = ctypes.c_int
     so.kascade_workspace_error.argtypes = [P, ctypes.POINTER(ctypes.c_int), ctypes.c_int, P]
     so.kascade_workspace_error.restype = ctypes.c_int
+    so.kascade_index_overlap.argtypes = [SP, P, P, P, P]
+    so.kascade_index_overlap.restype = ctypes.c_int
+    so.kascade_plan_anchors.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.c_int32, ctypes.c_int32,
+                                        ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_double)]
+    so.kascade_plan_anchors.restype = ctypes.c_int
+    so.kascade_refine_select.argtypes = [SP, P, P, P, ctypes.c_int32, P, P, P, ctypes.c_size_t, P]
+    so.kascade_refine_select.restype = ctypes.c_int
     so.kascade_select_decode_static.argtypes = [SP, P, P, P, P]
     so.kascade_select_decode_static.restype = ctypes.c_int
+    so.kascade_select_decode_static_error.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.c_int, P]
+    so.kascade_select_decode_static_error.restype = ctypes.c_int
     so.kascade_select_decode_static_max_bytes.argtypes = []
     so.kascade_select_decode_static_max_bytes.restype = ctypes.c_size_t
     so.kascade_launch_count.argtypes = [SP, ctypes.c_int]
@@ -155,7 +176,7 @@ def index_offsets(shape: Shape) -> np.ndarray:
 class Workspace:
     """A zero-initialised device workspace large enough for the given ops."""
 
-    def __init__(self, shape: Shape, ops=(OP_SELECT, OP_SPARSE_DECODE, OP_SPARSE_PREFILL, OP_DENSE),
+    def __init__(self, shape: Shape, ops=(OP_SELECT, OP_SPARSE_DECODE, OP_SPARSE_PREFILL, OP_DENSE, OP_REFINE),
                  device="cuda", nbytes=None):
         need = nbytes if nbytes is not None else max([workspace_bytes(shape, op) for op in ops] + [256])
         self.buf = torch.zeros(need + 256, dtype=torch.uint8, device=device)
@@ -192,6 +213,40 @@ def select(shape: Shape, q, k, idx=None, ws=None, stream=None):
     return idx
 
 
+def refine_select(shape: Shape, q, k, pool, pool_len: int, head_map=None, idx=None, ws=None, stream=None):
+    """kascade_refine_select: a refined decode layer's own Top-k from the
+    proposal layer's pool [B, Hkv, pool_len]."""
+    if idx is None:
+        idx = torch.empty(index_count(shape), dtype=torch.int32, device=q.device)
+    if ws is None:
+        ws = Workspace(shape, (OP_REFINE,))
+    p, n = ws.args()
+    _check(lib.kascade_refine_select(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(pool), int(pool_len),
+                                     _ptr(head_map), _ptr(idx), p, n, _stream(stream)), "kascade_refine_select")
+    return idx
+
+
+def index_overlap(shape: Shape, a, b, counts=None, stream=None):
+    """kascade_index_overlap: |a and b| per (batch row, list), summed over tiles."""
+    if counts is None:
+        counts = torch.empty(shape.batch * shape.n_lists, dtype=torch.int64, device=a.device)
+    _check(lib.kascade_index_overlap(ctypes.byref(shape), _ptr(a), _ptr(b), _ptr(counts), _stream(stream)),
+           "kascade_index_overlap")
+    return counts
+
+
+def plan_anchors(sim, n_anchors: int):
+    """kascade_plan_anchors: (anchor layers, objective) for a host
+    similarity matrix sim[a][l]."""
+    sim = np.ascontiguousarray(np.asarray(sim, dtype=np.float64))
+    n = sim.shape[0]
+    out = (ctypes.c_int32 * max(n_anchors, 1))()
+    obj = ctypes.c_double(0.0)
+    _check(lib.kascade_plan_anchors(sim.ctypes.data_as(ctypes.POINTER(ctypes.c_double)), n, n_anchors, out,
+                                    ctypes.byref(obj)), "kascade_plan_anchors")
+    return list(out)[:n_anchors], obj.value
+
+
 def select_decode_static(shape: Shape, q, k, idx=None, stream=None):
     """kascade_select_decode_static: decode anchor selection with the library's
     fixed scratch array instead of a workspace (nothing is allocated)."""
@@ -200,6 +255,15 @@ def select_decode_static(shape: Shape, q, k, idx=None, stream=None):
     _check(lib.kascade_select_decode_static(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(idx), _stream(stream)),
            "kascade_select_decode_static")
     return idx
+
+
+def select_decode_static_error(clear=True, stream=None) -> int:
+    """The device error word of kascade_select_decode_static on the current
+    device (0 = no kernel gave up on a bounded wait)."""
+    out = ctypes.c_int(0)
+    _check(lib.kascade_select_decode_static_error(ctypes.byref(out), int(clear), _stream(stream)),
+           "kascade_select_decode_static_error")
+    return out.value
 
 
 def _attn(fn, name, shape, q, k, v, idx, head_map, o, lse, ws, stream, op):

@@ -58,6 +58,8 @@ def test_workspace_sizes_positive():
     (dict(head_dim=96), 2), (dict(head_dim=0), 2), (dict(num_q_heads=12, num_kv_heads=8), 1),
     (dict(num_q_heads=64, num_kv_heads=4), 2), (dict(topk_num=0), 1), (dict(topk_num=11, topk_den=10), 1),
     (dict(tile=16, q_len=64, kv_len=64), 2), (dict(q_len=7), 2), (dict(batch=0), 1), (dict(kv_len=0), 1),
+    (dict(select_mode=3), 1), (dict(select_mode=-1), 1), (dict(dtype=3), 2),
+    (dict(select_mode=2, num_q_heads=128, num_kv_heads=64), 2),
 ])
 def test_bad_shapes_are_rejected(bad, status):
     kc = _kc()
@@ -105,3 +107,18 @@ def test_status_strings():
     for st in range(5):
         assert isinstance(kc.status_str(st), str) and kc.status_str(st)
     assert kc.status_str(99) == "unknown status"
+
+
+@pytest.mark.parametrize("mode,lists", [(0, 2), (1, 8), (2, 1)])
+def test_index_layout_per_selection_mode(mode, lists):
+    """L lists per batch row: Hkv (GQA), Hq (per query head), 1 (all heads)."""
+    kc = _kc()
+    d = kc.Shape.make(3, 8, 2, 64, 1, 1000, mode=mode)
+    assert d.n_lists == lists
+    assert kc.index_count(d) == 3 * lists * O.topk_count(1000, 10, 100)
+    p = kc.Shape.make(3, 8, 2, 64, 1000, 1000, mode=mode)
+    assert kc.index_count(p) == 3 * lists * int(O.index_offsets(1000, 32, 10, 100)[-1])
+    for dt in (0, 1, 2):
+        for sh in (d, p):
+            sh.dtype = dt
+            assert kc.workspace_bytes(sh, kc.OP_SELECT) > 0

@@ -178,3 +178,27 @@ def test_decode_long_context_takes_the_two_kernel_path():
     tally.assert_ok()
     o_ref, _ = O.sparse_decode(qn, kn, vn, idx_g)
     check_out(np64(o).reshape(B, Hq, d), o_ref, "long-context decode")
+
+
+def test_decode_beyond_the_cluster_select_range():
+    """N > 131072 (the 8-CTA cluster select holds up to 16384 keys per CTA):
+    scoring kernel plus the one-CTA-per-problem Top-k, up to the largest
+    context the library accepts."""
+    kc = _kc()
+    for N, seed in ((200003, 41), (1 << 20, 42)):
+        B, Hq, Hkv, d, frac = 1, 4, 1, 64, (10, 100)
+        s = kc.Shape.make(B, Hq, Hkv, d, 1, N, frac)
+        assert kc.launch_count(s, kc.OP_SELECT) == 2
+        q, k, v = gen_inputs(dict(B=B, Hq=Hq, Hkv=Hkv, d=d, N=N), seed=seed)
+        ws = kc.Workspace(s)
+        idx = kc.select(s, q, k, ws=ws)
+        o = kc.sparse_decode(s, q, k, v, idx, None, ws=ws)
+        torch.cuda.synchronize()
+        assert ws.error() == 0
+        kk = O.topk_count(N, *frac)
+        idx_g = idx.view(B, Hkv, kk).cpu().numpy()
+        qn, kn, vn = np64(q), np64(k), np64(v)
+        _, tally = decode_idx_check(qn, kn, idx_g, frac)
+        tally.assert_ok()
+        o_ref, _ = O.sparse_decode(qn, kn, vn, idx_g)
+        check_out(np64(o).reshape(B, Hq, d), o_ref, f"decode N={N}")

@@ -136,3 +136,14 @@ def test_prefill_qwen_stack_sampled():
     tiles = sorted(set([0, 1, 2, T - 1] + rng.integers(3, T - 1, size=8).tolist()))
     _judge(q1, k1, v1, idx.cpu().numpy(), o1, lse, 1, cfg.hkv, cfg.n_ctx, frac, tiles, head_map=hm,
            sel_inputs=(np64(q0), np64(k0)))
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(10, 2), (12, 2), (14, 2)])
+def test_prefill_groups_of_five_to_seven(Hq, Hkv):
+    """G in {5, 6, 7}: warp-MMA scoring (G > 4) and the warp-MMA sparse
+    prefill (the tensor-core kernel takes G <= 4 or multiples of 4)."""
+    B, d, N, frac = 1, 128, 330, (10, 100)
+    q, k, v, idx, o, lse = _prefill(B, Hq, Hkv, d, N, frac, seed=Hq, head_map=[1, 0], reuse_seed=Hq + 100)
+    qs, ks, _ = gen_inputs(dict(mode="prefill", B=B, Hq=Hq, Hkv=Hkv, d=d, N=N), seed=Hq)
+    _judge(q, k, v, idx, o, lse, B, Hkv, N, frac, range(-(-N // 32)), head_map=[1, 0],
+           sel_inputs=(np64(qs), np64(ks)))

@@ -35,6 +35,10 @@ def test_static_scratch_select_matches_workspace_select(B, Hq, Hkv, d, N):
     torch.cuda.synchronize()
     assert torch.equal(first, ref)
     assert torch.equal(second, ref)
+    # no bounded wait gave up in either call (the static path's own error word)
+    err = ctypes.c_int(-1)
+    st = kc.lib.kascade_select_decode_static_error(ctypes.byref(err), 1, torch.cuda.current_stream().cuda_stream)
+    assert st == kc.OK and err.value == 0
 
 
 def test_static_scratch_rejects_oversized_and_prefill_shapes():
@@ -45,3 +49,9 @@ def test_static_scratch_rejects_oversized_and_prefill_shapes():
     assert st == kc.ERR_TOO_LARGE and "scratch" in kc.status_str(st)
     pre = kc.Shape.make(1, 8, 2, 64, 256, 256)
     assert kc.lib.kascade_select_decode_static(ctypes.byref(pre), 256, 256, 256, None) == kc.ERR_UNSUPPORTED
+    # shapes kascade_select refuses get the same status here
+    for bad in (kc.Shape.make(1, 8, 2, 96, 1, 1024), kc.Shape.make(1, 32, 2, 128, 1, 1024),
+                kc.Shape.make(1, 8, 3, 64, 1, 1024), kc.Shape.make(1, 8, 2, 64, 1, 1024, (0, 100))):
+        want = kc.lib.kascade_select(ctypes.byref(bad), 256, 256, 256, None, 0, None)
+        assert want in (kc.ERR_UNSUPPORTED, kc.ERR_INVALID_ARG)
+        assert kc.lib.kascade_select_decode_static(ctypes.byref(bad), 256, 256, 256, None) == want
