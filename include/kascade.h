@@ -14,7 +14,7 @@
  * Conventions shared by every call
  * --------------------------------
  * Tensors are dense, row-major, bf16 (or the shape's KASCADE_DTYPE_*):
- *   q   [B, Hq,  L, d]   L = q_len (1 in decode, N in prefill)
+ *   q   [B, Hq,  L, d]   L = q_len (1 in decode; N, or a chunk's rows, in prefill)
  *   k,v [B, Hkv, N, d]   one contiguous [N, d] slab per (batch, kv head)
  *   o   [B, Hq,  L, d]   output, the input type
  *   lse [B, Hq,  L]      fp32 natural-log softmax denominator of the scaled
@@ -25,9 +25,10 @@
  * Index sets (int32, ascending within each list), L lists per batch row
  * (L = Hkv in the default GQA mode; see KASCADE_SELECT_*):
  *   decode  idx [B, L, K]            K = ceil(frac * N)
- *   prefill idx [B, L, S]            S = sum_t k_t, k_t = ceil(frac * e_t),
- *                                    e_t = min(32 (t+1), N); the list of tile t
- *                                    starts at offsets[t] (kascade_index_offsets)
+ *   prefill idx [B, L, S]            S = sum_t k_t over the call's query tiles,
+ *                                    k_t = ceil(frac * e_t), e_t = min(32 (t+1), N);
+ *                                    the list of the call's i-th tile starts at
+ *                                    offsets[i] (kascade_index_offsets)
  *
  * Ownership: the caller owns every buffer (device memory for tensors, index
  * lists and the workspace; host memory for kascade_shape and offsets).  The
@@ -102,7 +103,12 @@ typedef struct kascade_shape {
   int32_t num_q_heads;  /* Hq >= 1, multiple of Hkv */
   int32_t num_kv_heads; /* Hkv >= 1 */
   int32_t head_dim;     /* d: 64 or 128 */
-  int32_t q_len;        /* 1 = decode; == kv_len = causal prefill */
+  int32_t q_len;        /* 1 = decode; else causal prefill of the last q_len positions
+                           of the context: q_len == kv_len is the whole prompt,
+                           q_len < kv_len a rolling chunk (README, Python API,
+                           rolling_prefill) whose first position kv_len - q_len is a
+                           multiple of 32; the call then covers only the chunk's query
+                           tiles, exactly as the whole prompt's call computes them */
   int32_t kv_len;       /* N >= 1 (N <= 2^20) */
   int32_t tile;         /* prefill query tile; must be 32 (ignored in decode) */
   int32_t topk_num;     /* frac = topk_num / topk_den, 0 < frac <= 1, */

@@ -29,7 +29,9 @@ int check_shape(const kascade_shape* s) {
   if (s->num_q_heads / s->num_kv_heads > 8) return KASCADE_ERR_UNSUPPORTED;
   if (s->kv_len > (1 << 20)) return KASCADE_ERR_UNSUPPORTED;
   if (s->topk_den > (1 << 20)) return KASCADE_ERR_UNSUPPORTED;
-  if (s->q_len != 1 && s->q_len != s->kv_len) return KASCADE_ERR_UNSUPPORTED;
+  // prefill: the query rows are the last q_len positions of the context (a
+  // rolling chunk when q_len < kv_len), starting on a tile boundary
+  if (s->q_len > s->kv_len || (s->q_len != 1 && (s->kv_len - s->q_len) % 32 != 0)) return KASCADE_ERR_UNSUPPORTED;
   if (s->q_len != 1 && s->tile != 32) return KASCADE_ERR_UNSUPPORTED;
   if (s->flags & ~(KASCADE_FLAG_PDL | KASCADE_FLAG_INPUTS_STABLE | KASCADE_FLAG_TEST_DROP_LOAD))
     return KASCADE_ERR_INVALID_ARG;
@@ -52,17 +54,19 @@ int n_lists(const kascade_shape* s) {
 int sel_heads(const kascade_shape* s) { return s->num_q_heads / n_lists(s); }
 
 bool is_decode(const kascade_shape* s) { return s->q_len == 1; }
+// prefill: first query position and first query tile of the call
+int q_first(const kascade_shape* s) { return is_decode(s) ? 0 : s->kv_len - s->q_len; }
+int t_first(const kascade_shape* s) { return q_first(s) / 32; }
 // fp32 and fp16 inputs run the CUDA-core path (is_f32: either of them)
 bool is_f32(const kascade_shape* s) { return s->dtype == KASCADE_DTYPE_F32 || s->dtype == KASCADE_DTYPE_F16; }
 bool is_f16(const kascade_shape* s) { return s->dtype == KASCADE_DTYPE_F16; }
 int n_tiles(const kascade_shape* s) { return (s->kv_len + 31) / 32; }
 
 int64_t prefill_row_len(const kascade_shape* s) {
-  const int T = n_tiles(s);
-  return tile_list_offset(T - 1, 32, s->topk_num, s->topk_den) + topk_count(s->kv_len, s->topk_num, s->topk_den);
+  return chunk_row_len(s->kv_len, t_first(s), 32, s->topk_num, s->topk_den);
 }
 
-int64_t pooled_row_len(const kascade_shape* s) { return tile_pooled_offset(n_tiles(s) - 1, 32) + s->kv_len; }
+int64_t pooled_row_len(const kascade_shape* s) { return chunk_pooled_len(s->kv_len, t_first(s), 32); }
 
 // ----------------------------------------------------------------- workspace plans
 
@@ -121,14 +125,15 @@ SelectPlan plan_select(const kascade_shape* s, void* ws) {
     p.grid = select_grid(false, (int)(B * n_lists(s)), kPlanSMs);
     p.v_scratch = cv.take<float>((size_t)p.grid * n_max);
   } else {
-    p.row_m2 = cv.take<float>(B * Hq * N);
-    p.row_l = cv.take<double>(B * Hq * N);
+    const size_t Lq = s->q_len;   // row statistics of the call's query rows
+    p.row_m2 = cv.take<float>(B * Hq * Lq);
+    p.row_l = cv.take<double>(B * Hq * Lq);
     // scoring writes one pooled row per kv head (per query head in the
     // per-head mode); the all-heads mode adds their mean per batch row
     const size_t score_rows = s->select_mode == KASCADE_SELECT_PER_HEAD ? Hq : Hkv;
     p.pooled = cv.take<float>(B * score_rows * (size_t)pooled_row_len(s));
     p.pooled_all = s->select_mode == KASCADE_SELECT_ALL_HEADS ? cv.take<float>(B * (size_t)pooled_row_len(s)) : nullptr;
-    const int64_t problems = (int64_t)B * n_lists(s) * n_tiles(s);
+    const int64_t problems = (int64_t)B * n_lists(s) * (n_tiles(s) - t_first(s));
     p.grid = select_grid(true, (int)(problems < (1 << 30) ? problems : (1 << 30)), kPlanSMs);
     p.v_scratch = nullptr;
   }
@@ -214,6 +219,8 @@ AttnArgs attn_args(const kascade_shape* s, const void* q, const void* k, const v
   a.flags = s->flags;
   a.Gkv = a.G;
   a.Hp = a.Hkv;
+  a.q0 = q_first(s);
+  a.Lq = s->q_len;
   a.n_lists = n_lists(s);
   a.one_list = false;
   if (idx && s->select_mode == KASCADE_SELECT_PER_HEAD) {   // one problem per query head
@@ -264,9 +271,9 @@ int kascade_index_offsets(const kascade_shape* s, int64_t* offsets) {
     offsets[1] = topk_count(s->kv_len, s->topk_num, s->topk_den);
     return KASCADE_OK;
   }
-  const int T = n_tiles(s);
-  for (int t = 0; t < T; ++t) offsets[t] = tile_list_offset(t, 32, s->topk_num, s->topk_den);
-  offsets[T] = prefill_row_len(s);
+  const int T = n_tiles(s), t0 = t_first(s);
+  for (int t = t0; t < T; ++t) offsets[t - t0] = chunk_list_offset(t, t0, 32, s->topk_num, s->topk_den);
+  offsets[T - t0] = prefill_row_len(s);
   return KASCADE_OK;
 }
 
@@ -315,6 +322,8 @@ int kascade_select(const kascade_shape* s, const void* q, const void* k, int32_t
   a.Gkv = a.Hq / a.Hkv;
   a.D = s->head_dim;
   a.N = s->kv_len;
+  a.q0 = q_first(s);
+  a.Lq = s->q_len;
   a.tile = 32;
   a.num = s->topk_num;
   a.den = s->topk_den;
@@ -367,6 +376,8 @@ int kascade_select(const kascade_shape* s, const void* q, const void* k, int32_t
     sp.G = a.Gkv;   // scoring runs per kv head over its query heads
     sp.D = a.D;
     sp.N = a.N;
+    sp.q0 = a.q0;
+    sp.Lq = a.Lq;
     sp.tile = 32;
     sp.per_head = s->select_mode == KASCADE_SELECT_PER_HEAD;
     rc = cuda_status(is_f32(s) ? launch_score_pool_f32(sp, is_f16(s), st)
@@ -481,7 +492,7 @@ int kascade_sparse_prefill(const kascade_shape* s, const void* q, const void* k,
   int rc = check_shape(s);
   if (rc) return rc;
   // N = 1 is both a decode and a prefill shape; both index layouts coincide there
-  if (s->q_len != s->kv_len) return KASCADE_ERR_UNSUPPORTED;
+  if (is_decode(s) && s->kv_len != 1) return KASCADE_ERR_UNSUPPORTED;
   if (!v || !idx) return KASCADE_ERR_INVALID_ARG;
   rc = check_tensors(q, k, v, o);
   if (rc) return rc;

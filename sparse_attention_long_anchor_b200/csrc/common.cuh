@@ -61,6 +61,27 @@ __host__ __device__ inline int64_t tile_pooled_offset(int64_t t, int tile) {
   return (int64_t)tile * t * (t + 1) / 2;
 }
 
+// Rolling (chunked) prefill: the query rows are the last Lq positions
+// [q0, N) of an N-key context, q0 a multiple of the tile, so the call covers
+// tiles t0 = q0 / tile .. T - 1.  Index lists and pooled rows of such a call
+// hold only those tiles; offsets are relative to tile t0 (t0 = 0 for a full
+// prefill).
+__host__ __device__ inline int64_t chunk_list_offset(int64_t t, int64_t t0, int tile, int num, int den) {
+  return tile_list_offset(t, tile, num, den) - tile_list_offset(t0, tile, num, den);
+}
+__host__ __device__ inline int64_t chunk_pooled_offset(int64_t t, int64_t t0, int tile) {
+  return tile_pooled_offset(t, tile) - tile_pooled_offset(t0, tile);
+}
+// length of one (batch row, list) index row / pooled row of the chunk
+__host__ __device__ inline int64_t chunk_row_len(int N, int64_t t0, int tile, int num, int den) {
+  const int64_t T = (N + tile - 1) / tile;
+  return chunk_list_offset(T - 1, t0, tile, num, den) + topk_count(N, num, den);
+}
+__host__ __device__ inline int64_t chunk_pooled_len(int N, int64_t t0, int tile) {
+  const int64_t T = (N + tile - 1) / tile;
+  return chunk_pooled_offset(T - 1, t0, tile) + N;
+}
+
 // ---------------------------------------------------------------------------
 // bf16 helpers
 

@@ -147,6 +147,7 @@ __global__ void __launch_bounds__(256) score_pool_f32_kernel(const ScorePoolArgs
   const T* q = reinterpret_cast<const T*>(a.q);
   const T* k = reinterpret_cast<const T*>(a.k);
   const int nT = (a.N + a.tile - 1) / a.tile;
+  const int t0 = a.q0 / a.tile;   // first query tile of the call (rolling chunks)
   const int t = nT - 1 - (int)blockIdx.x;
   const int bh = blockIdx.y;
   const int b = bh / a.Hkv, h = bh - b * a.Hkv;
@@ -160,7 +161,8 @@ __global__ void __launch_bounds__(256) score_pool_f32_kernel(const ScorePoolArgs
   for (int e = threadIdx.x; e < G * 32 * D; e += 256) {
     const int rr = e / D, dd = e - rr * D;
     const int gi = rr >> 5, li = rr & 31;
-    qs[rr * (D + 1) + dd] = li < rows_t ? to_f(q[((size_t)(b * a.Hq + h * G + gi) * a.N + i0 + li) * D + dd]) : 0.f;
+    qs[rr * (D + 1) + dd] =
+        li < rows_t ? to_f(q[((size_t)(b * a.Hq + h * G + gi) * a.Lq + (i0 - a.q0) + li) * D + dd]) : 0.f;
   }
   const float* qrow = qs + r * (D + 1);
   const T* kb = k + (size_t)bh * a.N * D;
@@ -196,14 +198,14 @@ __global__ void __launch_bounds__(256) score_pool_f32_kernel(const ScorePoolArgs
   const float m2 = (float)mx;
   const double lsum = valid ? l * exp2(mx - (double)m2) : 1.0;
   if (valid) {
-    const size_t srow = (size_t)(b * a.Hq + h * G + g) * a.N + pos;
+    const size_t srow = (size_t)(b * a.Hq + h * G + g) * a.Lq + (pos - a.q0);
     a.row_m2[srow] = m2;
     a.row_l[srow] = lsum;
   }
   // pass 2: pooled score of each key, summed over the rows (per head with
   // per_head: a warp holds one head's 32 rows)
   __shared__ float part[8][KB];
-  const size_t prow = (size_t)(tile_pooled_offset(nT - 1, a.tile) + a.N);
+  const size_t prow = (size_t)chunk_pooled_len(a.N, t0, a.tile);
   const float inv = 1.0f / (float)((a.per_head ? 1 : G) * rows_t);
   for (int j0 = 0; j0 < e_t; j0 += KB) {
     stage(j0);
@@ -220,11 +222,11 @@ __global__ void __launch_bounds__(256) score_pool_f32_kernel(const ScorePoolArgs
       const int j = j0 + threadIdx.x;
       if (a.per_head) {
         for (int gg = 0; gg < G; ++gg)
-          a.pooled[(size_t)(b * a.Hq + h * G + gg) * prow + tile_pooled_offset(t, a.tile) + j] = part[gg][threadIdx.x] * inv;
+          a.pooled[(size_t)(b * a.Hq + h * G + gg) * prow + chunk_pooled_offset(t, t0, a.tile) + j] = part[gg][threadIdx.x] * inv;
       } else {
         float sum = 0.f;
         for (int gg = 0; gg < G; ++gg) sum += part[gg][threadIdx.x];
-        a.pooled[(size_t)bh * prow + tile_pooled_offset(t, a.tile) + j] = sum * inv;
+        a.pooled[(size_t)bh * prow + chunk_pooled_offset(t, t0, a.tile) + j] = sum * inv;
       }
     }
   }
@@ -248,9 +250,9 @@ __device__ __forceinline__ ListRef list_ref(const AttnArgs& a, int b, int h, int
   const bool ok = hm_raw >= 0 && hm_raw < a.n_lists;
   const int hm = ok ? hm_raw : 0;
   if (prefill) {
-    const int T = (a.N + a.tile - 1) / a.tile;
-    const int64_t row_len = tile_list_offset(T - 1, a.tile, a.num, a.den) + topk_count(a.N, a.num, a.den);
-    r.list = a.idx + (size_t)(b * a.n_lists + hm) * row_len + tile_list_offset(t, a.tile, a.num, a.den);
+    const int t0 = a.q0 / a.tile;
+    const int64_t row_len = chunk_row_len(a.N, t0, a.tile, a.num, a.den);
+    r.list = a.idx + (size_t)(b * a.n_lists + hm) * row_len + chunk_list_offset(t, t0, a.tile, a.num, a.den);
     r.len = ok ? topk_count(e_t, a.num, a.den) : 0;
   } else {
     const int K = topk_count(a.N, a.num, a.den);
@@ -367,8 +369,8 @@ __global__ void __launch_bounds__(256) sparse_prefill_f32_kernel(const AttnArgs 
   const bool causal = a.idx != nullptr || a.causal;
   const float scale2 = (float)(1.4426950408889634 / sqrt((double)D));
   float qv[HD], o[HD];
-  const T* qr = reinterpret_cast<const T*>(a.q) + ((size_t)(b * a.Hq + h * G + (valid ? g : 0)) * a.N +
-                                                           (valid ? pos : 0)) * D + half * HD;
+  const T* qr = reinterpret_cast<const T*>(a.q) + ((size_t)(b * a.Hq + h * G + (valid ? g : 0)) * a.Lq +
+                                                   (valid ? pos - a.q0 : 0)) * D + half * HD;
 #pragma unroll
   for (int e = 0; e < HD; ++e) {
     qv[e] = valid ? to_f(qr[e]) : 0.f;
@@ -405,7 +407,7 @@ __global__ void __launch_bounds__(256) sparse_prefill_f32_kernel(const AttnArgs 
     }
   }
   if (!valid) return;
-  const size_t orow = (size_t)(b * a.Hq + h * G + g) * a.N + pos;
+  const size_t orow = (size_t)(b * a.Hq + h * G + g) * a.Lq + (pos - a.q0);
   T* od = reinterpret_cast<T*>(a.o) + orow * D + half * HD;
 #pragma unroll
   for (int e = 0; e < HD; ++e) od[e] = from_f<T>(l > 0.f ? o[e] / l : 0.f);
@@ -438,7 +440,7 @@ cudaError_t launch_decode_score_f32(const DecodeScoreArgs& a, bool half, cudaStr
 }
 
 cudaError_t launch_score_pool_f32(const ScorePoolArgs& a, bool half, cudaStream_t stream) {
-  const int T = (a.N + a.tile - 1) / a.tile;
+  const int T = (a.N + a.tile - 1) / a.tile - a.q0 / a.tile;   // the call's query tiles
   const dim3 grid(T, a.B * a.Hkv);
   auto go = [&](auto tag) -> cudaError_t {
     using E = std::remove_pointer_t<decltype(tag)>;
@@ -469,7 +471,7 @@ cudaError_t launch_sparse_decode_f32(const AttnArgs& a, bool half, cudaStream_t 
 }
 
 cudaError_t launch_sparse_prefill_f32(const AttnArgs& a, bool half, cudaStream_t stream) {
-  const int T = (a.N + a.tile - 1) / a.tile;
+  const int T = (a.N + a.tile - 1) / a.tile - a.q0 / a.tile;   // the call's query tiles
   const int row_blocks = (a.G * a.tile + 127) / 128;
   const dim3 grid(T * row_blocks, a.B * a.Hp);
   auto go = [&](auto tag) -> cudaError_t {

@@ -40,6 +40,7 @@ struct SelArgs {
   int B, Hq, Hkv, G, D, N, tile, num, den;
   int Hp;                  // problems per batch row (index lists per row)
   int Gkv;                 // query heads per kv head
+  int q0, Lq;              // prefill: query rows are positions [q0, q0 + Lq = N) (rolling chunk)
   int in_type;             // element type of q and k: 0 bf16, 1 fp32, 2 fp16 (pointers reinterpreted)
   // decode proposal-refine: the N candidates of problem (b, h) are the keys
   // cand[(b * cand_lists + cand_map[h]) * N + j] (cand_map NULL = h); K slabs
@@ -89,8 +90,9 @@ struct ScorePoolArgs {
   const __nv_bfloat16* k;  // [B, Hkv, N, D]
   float* row_m2;           // [B, Hq, N]
   double* row_l;           // [B, Hq, N]
-  float* pooled;           // [B, Hkv, sum_t e_t], or [B, Hq, sum_t e_t] with per_head
+  float* pooled;           // [B, Hkv, sum_t e_t], or [B, Hq, sum_t e_t] with per_head (the chunk's tiles)
   int B, Hq, Hkv, G, D, N, tile;
+  int q0, Lq;              // query rows: positions [q0, q0 + Lq = N); row stats are [B, Hq, Lq]
   int flags;
   bool per_head;           // pool each query head on its own (no GQA mean)
 };
@@ -111,6 +113,7 @@ struct AttnArgs {
   int B, Hq, Hkv, G, D, N, tile, num, den;
   int Hp;                    // problems per batch row (G = query heads per problem)
   int Gkv;                   // query heads per kv head
+  int q0, Lq;                // prefill: query (and o, lse) rows are positions [q0, q0 + Lq = N)
   int n_lists;               // index lists per batch row
   bool one_list;             // every problem reads list 0 of its row (head_map unused)
   bool causal;               // prefill dense only

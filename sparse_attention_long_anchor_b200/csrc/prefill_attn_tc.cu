@@ -83,8 +83,10 @@ __device__ __forceinline__ Item item_of(const AttnArgs& a, int it, int T, int RB
   // head-major, longest tile first within a head: the CTAs in flight share
   // one head's K and V, which then stay in L2
   Item I;
-  const int bh = it / (RB * T);
-  const int rem = it - bh * (RB * T);
+  const int t0 = a.q0 / a.tile;   // first query tile of the call (rolling chunks)
+  const int Tc = T - t0;
+  const int bh = it / (RB * Tc);
+  const int rem = it - bh * (RB * Tc);
   const int t = T - 1 - rem / RB, rb = rem - (rem / RB) * RB;
   I.b = bh / a.Hp;
   I.h = bh - I.b * a.Hp;        // problem of the batch row
@@ -97,8 +99,8 @@ __device__ __forceinline__ Item item_of(const AttnArgs& a, int it, int T, int RB
     const int hm_raw = a.one_list ? 0 : (a.head_map ? a.head_map[I.h] : I.h);
     const bool hm_ok = hm_raw >= 0 && hm_raw < a.n_lists;
     const int hm = hm_ok ? hm_raw : 0;
-    const int64_t row_len = tile_list_offset(T - 1, a.tile, a.num, a.den) + topk_count(a.N, a.num, a.den);
-    I.list = a.idx + (size_t)(I.b * a.n_lists + hm) * row_len + tile_list_offset(t, a.tile, a.num, a.den);
+    const int64_t row_len = chunk_row_len(a.N, t0, a.tile, a.num, a.den);
+    I.list = a.idx + (size_t)(I.b * a.n_lists + hm) * row_len + chunk_list_offset(t, t0, a.tile, a.num, a.den);
     I.list_len = hm_ok ? topk_count(e_t, a.num, a.den) : 0;
   } else {
     I.list_len = a.causal ? e_t : a.N;
@@ -129,7 +131,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar = [&](int slot) { return bar0 + 8u * (uint32_t)slot; };
   const int G = a.G;
   const int T = (a.N + a.tile - 1) / a.tile;
-  const int items = T * RB * a.B * a.Hp;
+  const int items = (T - a.q0 / a.tile) * RB * a.B * a.Hp;
   const bool causal = a.idx != nullptr || a.causal;
   const int heads_rb = min(4, G);   // query heads per row block
   // this pipeline's items: the CTA's share, alternating between pipelines
@@ -220,7 +222,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(bar(bQFull), (uint32_t)(CB * heads_rb * 32 * 128));
         for (int b = 0; b < CB; ++b)
           for (int g = 0; g < heads_rb; ++g)
-            tc::tma_load_3d(q_s + b * L::QCB + g * 4096, &mq, b * 64, I.i0, I.b * a.Hq + I.hq0 + g, bar(bQFull));
+            tc::tma_load_3d(q_s + b * L::QCB + g * 4096, &mq, b * 64, I.i0 - a.q0, I.b * a.Hq + I.hq0 + g,
+                            bar(bQFull));
       }
       const size_t bhoff = (size_t)kv_slab_of(I.b, I.h * a.G, a.Hkv, a.Gkv) * a.N * D;
       for (int j = 0; j < I.nb; ++j, ++n) {
@@ -447,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ocnt += I.nb;
       const float inv = l > 0.f ? 1.0f / l : 0.0f;
-      __nv_bfloat16* orow = a.o + ((size_t)(I.b * a.Hq + I.hq0 + g) * a.N + pos) * D;
+      __nv_bfloat16* orow = a.o + ((size_t)(I.b * a.Hq + I.hq0 + g) * a.Lq + (pos - a.q0)) * D;
 #pragma unroll 1
       for (int c32 = 0; c32 < D / 32; ++c32) {
         float o[32];
@@ -470,7 +473,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (valid && a.lse)
-        a.lse[(size_t)(I.b * a.Hq + I.hq0 + g) * a.N + pos] = l > 0.f ? (m_used + log2f(l)) * (float)kLn2 : -INFINITY;
+        a.lse[(size_t)(I.b * a.Hq + I.hq0 + g) * a.Lq + (pos - a.q0)] =
+            l > 0.f ? (m_used + log2f(l)) * (float)kLn2 : -INFINITY;
       tc::fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(bOEmpty));
@@ -495,8 +499,8 @@ bool prefill_attn_tc_supported(const AttnArgs& a) {
 
 cudaError_t launch_prefill_attn_tc(const AttnArgs& a, int num_sms, cudaStream_t stream) {
   CUtensorMap mq;
-  if (!tc::make_map_3d(&mq, a.q, (uint64_t)a.D, (uint64_t)a.N, (uint64_t)a.B * a.Hq, 32)) return cudaErrorInvalidValue;
-  const int T = (a.N + a.tile - 1) / a.tile;
+  if (!tc::make_map_3d(&mq, a.q, (uint64_t)a.D, (uint64_t)a.Lq, (uint64_t)a.B * a.Hq, 32)) return cudaErrorInvalidValue;
+  const int T = (a.N + a.tile - 1) / a.tile - a.q0 / a.tile;   // the call's query tiles
   const int RB = a.G <= 4 ? 1 : a.G / 4;
   const long items = (long)T * RB * a.B * a.Hp;
   const long long ctas = (items + kSubs - 1) / kSubs;

@@ -44,6 +44,7 @@ __global__ void __launch_bounds__(kSpWarps * 32) score_pool_kernel(const ScorePo
   int* rpos = reinterpret_cast<int*>(bcol + kSpMaxRows);                   // [256]
 
   const int T = (a.N + a.tile - 1) / a.tile;
+  const int t0 = a.q0 / a.tile;   // first query tile of the call (rolling chunks)
   const int t = T - 1 - (int)blockIdx.x;
   const int bh = blockIdx.y;
   const int b = bh / a.Hkv, h = bh - b * a.Hkv;
@@ -63,7 +64,8 @@ __global__ void __launch_bounds__(kSpWarps * 32) score_pool_kernel(const ScorePo
     const int r = e / CH, ch = e - r * CH;
     const int gi = r / a.tile, il = r - gi * a.tile;
     const bool ok = r < R && il < rows_t;
-    const __nv_bfloat16* src = a.q + ((size_t)(b * a.Hq + h * G + (ok ? gi : 0)) * a.N + i0 + (ok ? il : 0)) * D + ch * 8;
+    const __nv_bfloat16* src =
+        a.q + ((size_t)(b * a.Hq + h * G + (ok ? gi : 0)) * a.Lq + (i0 - a.q0) + (ok ? il : 0)) * D + ch * 8;
     cp_async_16(q_u + sp_swz<D>(r, ch), src, ok ? 16 : 0);
   }
   cp_async_commit();
@@ -164,7 +166,7 @@ __global__ void __launch_bounds__(kSpWarps * 32) score_pool_kernel(const ScorePo
       if (c == 0) {
         if (ipos[hf] >= 0) {
           const int gi = r / a.tile;
-          const size_t srow = (size_t)(b * a.Hq + h * G + gi) * a.N + ipos[hf];
+          const size_t srow = (size_t)(b * a.Hq + h * G + gi) * a.Lq + (ipos[hf] - a.q0);
           a.row_m2[srow] = m_run[hf];
           a.row_l[srow] = l_run[hf];
           bcol[r] = (float)((double)m_run[hf] + log2(l_run[hf]));
@@ -181,9 +183,9 @@ __global__ void __launch_bounds__(kSpWarps * 32) score_pool_kernel(const ScorePo
   const float inv_rows_head = 1.0f / (float)rows_t;
   // pooled rows: one per kv head, or one per query head (per_head: the G
   // rows of this kv head's query heads, b Hq + h G + hh)
-  const size_t pooled_row = (size_t)(tile_pooled_offset(T - 1, a.tile) + a.N);
+  const size_t pooled_row = (size_t)chunk_pooled_len(a.N, t0, a.tile);
   const size_t prow0 = a.per_head ? (size_t)(b * a.Hq + h * G) : (size_t)bh;
-  float* pooled = a.pooled + prow0 * pooled_row + tile_pooled_offset(t, a.tile);
+  float* pooled = a.pooled + prow0 * pooled_row + chunk_pooled_offset(t, t0, a.tile);
   issue(0, 0);
   cp_async_commit();
   for (int blk = 0; blk < n_blk; ++blk) {
@@ -261,7 +263,7 @@ size_t score_pool_smem() {
 }  // namespace
 
 cudaError_t launch_score_pool(const ScorePoolArgs& a, cudaStream_t stream) {
-  const int T = (a.N + a.tile - 1) / a.tile;
+  const int T = (a.N + a.tile - 1) / a.tile - a.q0 / a.tile;   // the call's query tiles
   dim3 grid(T, a.B * a.Hkv);
   if (a.D == 128) {
     const size_t sm = score_pool_smem<128>();

@@ -85,8 +85,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = a.G;
   const int T = (a.N + a.tile - 1) / a.tile;
+  const int t0 = a.q0 / a.tile;   // first query tile of the call (rolling chunks)
   const int BH = a.B * a.Hkv;
-  const int items = T * BH;
+  const int items = (T - t0) * BH;
   const uint32_t idesc = tc::idesc_bf16_f32(128, 128);
 
   if (threadIdx.x == 0) {
@@ -143,7 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(qcount == 0 && (a.flags & KASCADE_FLAG_TEST_DROP_LOAD)))
           for (int cb = 0; cb < L::CB; ++cb)
             for (int g = 0; g < G; ++g)
-              tc::tma_load_3d(q_s + cb * L::CBYTES + g * 4096, &mq, cb * 64, i0, b * a.Hq + h * G + g, q_full);
+              tc::tma_load_3d(q_s + cb * L::CBYTES + g * 4096, &mq, cb * 64, i0 - a.q0, b * a.Hq + h * G + g, q_full);
         ++qcount;
         for (int pass = 0; pass < 2; ++pass) {
           for (int blk = 0; blk < nb; ++blk) {
@@ -298,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (valid) {
-          const size_t srow = (size_t)(b * a.Hq + h * G + quarter) * a.N + pos;
+          const size_t srow = (size_t)(b * a.Hq + h * G + quarter) * a.Lq + (pos - a.q0);
           a.row_m2[srow] = M2;
           a.row_l[srow] = Ls;
         }
@@ -310,9 +311,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv_rows = 1.0f / (float)((a.per_head ? 1 : G) * rows_t);
       // pooled rows: one per kv head, or with per_head one per query head
       // (column chunk ch of the accumulator holds query head h G + ch)
-      const size_t pooled_row = (size_t)(tile_pooled_offset(T - 1, a.tile) + a.N);
+      const size_t pooled_row = (size_t)chunk_pooled_len(a.N, t0, a.tile);
       float* pooled = a.pooled + (a.per_head ? (size_t)(b * a.Hq + h * G) : (size_t)bh) * pooled_row +
-                      tile_pooled_offset(t, a.tile);
+                      chunk_pooled_offset(t, t0, a.tile);
       for (int blk = 0; blk < nb; ++blk, ++acount) {
         if (acount % kEpiGroups != wg) continue;
         const int buf = acount % kBufs;
@@ -372,10 +373,10 @@ bool score_pool_tc_supported(const ScorePoolArgs& a) { return a.G <= 4 && (a.D =
 
 cudaError_t launch_score_pool_tc(const ScorePoolArgs& a, int* err, int num_sms, cudaStream_t stream) {
   CUtensorMap mq, mk;
-  if (!tc::make_map_3d(&mq, a.q, (uint64_t)a.D, (uint64_t)a.N, (uint64_t)a.B * a.Hq, 32) ||
+  if (!tc::make_map_3d(&mq, a.q, (uint64_t)a.D, (uint64_t)a.Lq, (uint64_t)a.B * a.Hq, 32) ||
       !tc::make_map_3d(&mk, a.k, (uint64_t)a.D, (uint64_t)a.N, (uint64_t)a.B * a.Hkv, kKB))
     return cudaErrorInvalidValue;
-  const int T = (a.N + a.tile - 1) / a.tile;
+  const int T = (a.N + a.tile - 1) / a.tile - a.q0 / a.tile;   // the call's query tiles
   const long items = (long)T * a.B * a.Hkv;
   const int grid = (int)(items < num_sms ? items : num_sms);
   const bool pdl = (a.flags & 1) != 0;

@@ -46,6 +46,7 @@ __global__ void __launch_bounds__(kPreWarps * 32)
   int* key_s = reinterpret_cast<int*>(smem + kPreStages * STAGE_BYTES);   // [stages][64]
 
   const int T = (a.N + a.tile - 1) / a.tile;
+  const int t0 = a.q0 / a.tile;   // first query tile of the call (rolling chunks)
   const int t = T - 1 - (int)(blockIdx.x / row_blocks);
   const int rb = blockIdx.x % row_blocks;
   const int bh = blockIdx.y;
@@ -63,9 +64,8 @@ __global__ void __launch_bounds__(kPreWarps * 32)
   int list_len;
   const int32_t* list = nullptr;
   if (a.idx) {
-    const int T_last = T - 1;
-    const int64_t row_len = tile_list_offset(T_last, a.tile, a.num, a.den) + topk_count(a.N, a.num, a.den);
-    list = a.idx + (size_t)(b * a.n_lists + hm) * row_len + tile_list_offset(t, a.tile, a.num, a.den);
+    const int64_t row_len = chunk_row_len(a.N, t0, a.tile, a.num, a.den);
+    list = a.idx + (size_t)(b * a.n_lists + hm) * row_len + chunk_list_offset(t, t0, a.tile, a.num, a.den);
     list_len = hm_ok ? topk_count(e_t, a.num, a.den) : 0;
   } else {
     list_len = a.causal ? e_t : a.N;
@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(kPreWarps * 32)
     const int gi = r / a.tile, il = r - gi * a.tile;
     qrow_ok[hf] = gi < G && il < rows_t;
     qrow_i[hf] = i0 + il;
-    qrow_off[hf] = qrow_ok[hf] ? ((size_t)(b * a.Hq + h * G + gi) * a.N + i0 + il) * D : 0;
+    qrow_off[hf] = qrow_ok[hf] ? ((size_t)(b * a.Hq + h * G + gi) * a.Lq + (i0 - a.q0) + il) * D : 0;
   }
   uint32_t qa[D / 16][4];
 #pragma unroll
@@ -250,7 +250,7 @@ size_t prefill_smem() {
 }  // namespace
 
 cudaError_t launch_prefill_attn(const AttnArgs& a, cudaStream_t stream) {
-  const int T = (a.N + a.tile - 1) / a.tile;
+  const int T = (a.N + a.tile - 1) / a.tile - a.q0 / a.tile;   // the call's query tiles
   const int row_blocks = (a.G * a.tile + 127) / 128;
   dim3 grid(T * row_blocks, a.B * a.Hp);
   if (a.D == 128) {

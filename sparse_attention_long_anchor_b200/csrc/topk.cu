@@ -142,7 +142,7 @@ __device__ double refine_prefill(const SelArgs& a, const Problem& p, int j, doub
       const int g = r / a.tile, il = r - g * a.tile;
       const int i = p.i0 + il;
       if (il >= p.rows || j > i) continue;
-      const size_t qoff = ((size_t)(p.b * a.Hq + qh0 + g) * a.N + i) * a.D;
+      const size_t qoff = ((size_t)(p.b * a.Hq + qh0 + g) * a.Lq + (i - a.q0)) * a.D;
       double dot = 0.0;
       if (a.in_type != 0) {
         for (int e = 0; e < a.D; ++e) dot += (double)elem(a.q, qoff + e, a.in_type) * kbuf[e];
@@ -153,7 +153,7 @@ __device__ double refine_prefill(const SelArgs& a, const Problem& p, int j, doub
           dot += (double)__low2float(q2) * kbuf[e] + (double)__high2float(q2) * kbuf[e + 1];
         }
       }
-      const size_t srow = (size_t)(p.b * a.Hq + qh0 + g) * a.N + i;
+      const size_t srow = (size_t)(p.b * a.Hq + qh0 + g) * a.Lq + (i - a.q0);
       total += exp2(dot * c2 - (double)a.row_m2[srow]) / a.row_l[srow];
     }
     g0 += run;
@@ -412,10 +412,10 @@ __global__ void __launch_bounds__(NT, kSelCtasPerSM) select_kernel(const SelArgs
     }
   } else {
     const int T = (a.N + a.tile - 1) / a.tile;
-    const int64_t T_last = T - 1;
-    const int64_t row_len = tile_list_offset(T_last, a.tile, a.num, a.den) + topk_count(a.N, a.num, a.den);
-    const int64_t pooled_len = tile_pooled_offset(T_last, a.tile) + a.N;
-    const int64_t total = (int64_t)T * BH;
+    const int t0 = a.q0 / a.tile;   // first query tile of the call (rolling chunks)
+    const int64_t row_len = chunk_row_len(a.N, t0, a.tile, a.num, a.den);
+    const int64_t pooled_len = chunk_pooled_len(a.N, t0, a.tile);
+    const int64_t total = (int64_t)(T - t0) * BH;
     for (int64_t prob = cta; prob < total; prob += gridDim.x) {
       const int t = T - 1 - (int)(prob / BH);   // longest tiles first
       const int bh = (int)(prob % BH);
@@ -427,9 +427,9 @@ __global__ void __launch_bounds__(NT, kSelCtasPerSM) select_kernel(const SelArgs
       p.n = min((t + 1) * a.tile, a.N);
       p.rows = p.n - p.i0;
       p.k = topk_count(p.n, a.num, a.den);
-      p.v = a.pooled + (size_t)bh * pooled_len + tile_pooled_offset(t, a.tile);
+      p.v = a.pooled + (size_t)bh * pooled_len + chunk_pooled_offset(t, t0, a.tile);
       p.cand = nullptr;
-      p.out = a.idx + (size_t)bh * row_len + tile_list_offset(t, a.tile, a.num, a.den);
+      p.out = a.idx + (size_t)bh * row_len + chunk_list_offset(t, t0, a.tile, a.num, a.den);
       run_problem<NT>(a, p, sh, vscr, band_idx, band_val, state, dyn);
       __syncthreads();
     }

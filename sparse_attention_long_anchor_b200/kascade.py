@@ -166,7 +166,8 @@ def index_count(shape: Shape) -> int:
 
 
 def index_offsets(shape: Shape) -> np.ndarray:
-    n_t = 1 if shape.decode else -(-shape.kv_len // 32)
+    """Tile offsets of one index row (the call's tiles: a rolling chunk's own)."""
+    n_t = 1 if shape.decode else -(-shape.kv_len // 32) - (shape.kv_len - shape.q_len) // 32
     out = np.zeros(n_t + 1, dtype=np.int64)
     _check(lib.kascade_index_offsets(ctypes.byref(shape), out.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))),
            "kascade_index_offsets")
