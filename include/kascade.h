@@ -97,6 +97,7 @@ extern "C" {
 #define KASCADE_OP_SPARSE_PREFILL 2
 #define KASCADE_OP_DENSE 3
 #define KASCADE_OP_REFINE 4   /* kascade_refine_select, any pool length up to N */
+#define KASCADE_OP_SELECT_VARLEN 5   /* kascade_select_varlen */
 
 typedef struct kascade_shape {
   int32_t batch;        /* B  >= 1 */
@@ -263,6 +264,54 @@ KASCADE_API int kascade_refine_select(const kascade_shape* shape, const void* q,
 KASCADE_API int kascade_sparse_decode(const kascade_shape* shape, const void* q, const void* k,
                           const void* v, const int32_t* idx, const int32_t* head_map,
                           void* o, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Variable-length decode batches (README, Kernel Benchmarks note: varlen
+ * kernels are planned).  Batch row b holds kv_lens[b] keys, 1 <= kv_lens[b]
+ * <= N = shape->kv_len (device int32 [B], not checked on the device), in
+ * the first kv_lens[b] rows of its [N, d] slabs.  Row b's selection and
+ * attention are those of a batch of one with context kv_lens[b].
+ *
+ * kascade_select_varlen: as kascade_select for a decode shape (any selection
+ * mode), each row selecting ceil(frac kv_lens[b]) of its keys.  The index
+ * buffer keeps the layout of kv_len = N, [B, L, ceil(frac N)]: row b's lists
+ * hold their ceil(frac kv_lens[b]) keys ascending, then -1.  Workspace:
+ * kascade_workspace_bytes(shape, KASCADE_OP_SELECT_VARLEN).  bf16.
+ *
+ * kascade_sparse_decode_varlen: as kascade_sparse_decode, row b attending
+ * over the first ceil(frac kv_lens[b]) entries of its list (idx NULL: dense
+ * over its kv_lens[b] keys).  With KASCADE_FLAG_INPUTS_STABLE, kv_lens counts
+ * among the inputs that must be two launches old.  bf16.
+ */
+KASCADE_API int kascade_select_varlen(const kascade_shape* shape, const void* q, const void* k,
+                                      const int32_t* kv_lens, int32_t* idx, void* ws, size_t ws_bytes,
+                                      void* stream);
+KASCADE_API int kascade_sparse_decode_varlen(const kascade_shape* shape, const void* q, const void* k,
+                                             const void* v, const int32_t* kv_lens, const int32_t* idx,
+                                             const int32_t* head_map, void* o, float* lse, void* ws,
+                                             size_t ws_bytes, void* stream);
+
+/*
+ * kascade_sparse_decode over a paged KV cache (README, Kernel Benchmarks
+ * note: paged kernels are planned; a paged cache stores the same keys in
+ * fixed-size pages, so the results are those of kascade_sparse_decode on the
+ * contiguous cache, bit for bit).
+ *   k_pages, v_pages  device bf16 [num_pages, Hkv, page_size, d]: page p
+ *             holds page_size consecutive positions of one sequence for
+ *             every kv head
+ *   page_table device int32 [B, max_pages]: key j of batch row b is row
+ *             j % page_size of page page_table[b * max_pages + j / page_size]
+ *             (entries must name allocated pages; not checked on the device)
+ *   page_size a power of two in [16, 2^20]; max_pages >= ceil(N / page_size)
+ *   idx       as for kascade_sparse_decode, or NULL for dense decode over
+ *             the whole paged context
+ * Other arguments as kascade_sparse_decode.  bf16 only.  Anchor selection
+ * reads a contiguous K (kascade_select); this call serves the reuse layers.
+ */
+KASCADE_API int kascade_sparse_decode_paged(const kascade_shape* shape, const void* q, const void* k_pages,
+                                            const void* v_pages, const int32_t* page_table, int32_t page_size,
+                                            int32_t max_pages, const int32_t* idx, const int32_t* head_map,
+                                            void* o, float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Sparse causal prefill attention of an anchor or reuse layer (README

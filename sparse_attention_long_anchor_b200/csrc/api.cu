@@ -103,7 +103,7 @@ struct SelectPlan {
 // device error word (set when a bounded wait in a kernel gives up).
 constexpr size_t kHeader = 256;
 
-SelectPlan plan_select(const kascade_shape* s, void* ws) {
+SelectPlan plan_select(const kascade_shape* s, void* ws, bool one_cta = false) {
   SelectPlan p{};
   Carver cv{static_cast<char*>(ws)};
   cv.take<char>(kHeader);
@@ -114,7 +114,7 @@ SelectPlan plan_select(const kascade_shape* s, void* ws) {
     p.s2 = cv.take<float>(B * Hq * N);
     p.m_part = cv.take<float>(B * Hq * p.splits);
     p.l_part = cv.take<double>(B * Hq * p.splits);
-    if (s->select_mode != KASCADE_SELECT_ALL_HEADS && !is_f32(s) && select_decode_cluster_ok(s->kv_len)) {
+    if (!one_cta && s->select_mode != KASCADE_SELECT_ALL_HEADS && !is_f32(s) && select_decode_cluster_ok(s->kv_len)) {
       p.cluster = true;
       const size_t entries = select_decode_cluster_scratch(s->batch, n_lists(s), s->kv_len);
       p.band_idx = cv.take<int32_t>(entries);
@@ -250,6 +250,8 @@ size_t kascade_workspace_bytes(const kascade_shape* s, int op) {
       return kHeader;   // only the error word: partial results stay on chip
     case KASCADE_OP_REFINE:   // covers every pool length up to N
       return is_decode(s) ? plan_refine(s, s->kv_len, nullptr).bytes : 0;
+    case KASCADE_OP_SELECT_VARLEN:
+      return is_decode(s) ? plan_select(s, nullptr, true).bytes : 0;
     default:
       return 0;
   }
@@ -483,6 +485,111 @@ int kascade_sparse_decode(const kascade_shape* s, const void* q, const void* k, 
   AttnArgs a = attn_args(s, q, k, v, idx, head_map, o, lse);
   a.err = err_word(ws, ws_bytes);
   if (is_f32(s)) return cuda_status(launch_sparse_decode_f32(a, is_f16(s), static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_decode_attn(a, static_cast<cudaStream_t>(stream)));
+}
+
+int kascade_select_varlen(const kascade_shape* s, const void* q, const void* k, const int32_t* kv_lens,
+                          int32_t* idx, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_shape(s);
+  if (rc) return rc;
+  if (!is_decode(s) || s->dtype != KASCADE_DTYPE_BF16) return KASCADE_ERR_UNSUPPORTED;
+  if (!q || !k || !kv_lens || !idx) return KASCADE_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(idx, 4) || !aligned(kv_lens, 4)) return KASCADE_ERR_UNSUPPORTED;
+  SelectPlan pl = plan_select(s, nullptr, true);
+  rc = check_ws(ws, ws_bytes, pl.bytes);
+  if (rc) return rc;
+  pl = plan_select(s, ws, true);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int flags = s->flags & KASCADE_FLAG_PDL;
+  DecodeScoreArgs d{};
+  d.flags = flags;
+  d.q = static_cast<const __nv_bfloat16*>(q);
+  d.k = static_cast<const __nv_bfloat16*>(k);
+  d.s2 = pl.s2;
+  d.m_part = pl.m_part;
+  d.l_part = pl.l_part;
+  d.B = s->batch;
+  d.Hq = s->num_q_heads;
+  d.Hkv = s->num_kv_heads;
+  d.G = d.Hq / d.Hkv;
+  d.D = s->head_dim;
+  d.N = s->kv_len;
+  d.kv_lens = kv_lens;
+  rc = cuda_status(launch_decode_score(d, st));
+  if (rc) return rc;
+  SelArgs a{};
+  a.prefill = false;
+  a.B = d.B;
+  a.Hq = d.Hq;
+  a.Hkv = d.Hkv;
+  a.Hp = n_lists(s);
+  a.G = sel_heads(s);
+  a.Gkv = d.G;
+  a.D = d.D;
+  a.N = d.N;
+  a.kv_lens = kv_lens;
+  a.tile = 32;
+  a.num = s->topk_num;
+  a.den = s->topk_den;
+  a.q = d.q;
+  a.k = d.k;
+  a.s2 = pl.s2;
+  a.m_part = pl.m_part;
+  a.l_part = pl.l_part;
+  a.splits = pl.splits;
+  a.v_scratch = pl.v_scratch;
+  a.band_idx = pl.band_idx;
+  a.band_val = pl.band_val;
+  a.state = pl.state;
+  a.n_max = s->kv_len;
+  a.grid = pl.grid;
+  a.idx = idx;
+  a.flags = flags;
+  a.err = err_word(ws, ws_bytes);
+  return cuda_status(launch_select(a, st));
+}
+
+int kascade_sparse_decode_varlen(const kascade_shape* s, const void* q, const void* k, const void* v,
+                                 const int32_t* kv_lens, const int32_t* idx, const int32_t* head_map, void* o,
+                                 float* lse, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_shape(s);
+  if (rc) return rc;
+  if (!is_decode(s) || s->dtype != KASCADE_DTYPE_BF16) return KASCADE_ERR_UNSUPPORTED;
+  if (!v || !kv_lens) return KASCADE_ERR_INVALID_ARG;
+  rc = check_tensors(q, k, v, o);
+  if (rc) return rc;
+  if (!aligned(kv_lens, 4) || (idx && !aligned(idx, 4)) || (head_map && !aligned(head_map, 4)) ||
+      (lse && !aligned(lse, 4)))
+    return KASCADE_ERR_UNSUPPORTED;
+  AttnArgs a = attn_args(s, q, k, v, idx, head_map, o, lse);
+  a.err = err_word(ws, ws_bytes);
+  a.kv_lens = kv_lens;
+  return cuda_status(launch_decode_attn(a, static_cast<cudaStream_t>(stream)));
+}
+
+int kascade_sparse_decode_paged(const kascade_shape* s, const void* q, const void* k_pages, const void* v_pages,
+                                const int32_t* page_table, int32_t page_size, int32_t max_pages, const int32_t* idx,
+                                const int32_t* head_map, void* o, float* lse, void* ws, size_t ws_bytes,
+                                void* stream) {
+  int rc = check_shape(s);
+  if (rc) return rc;
+  if (!is_decode(s) || s->dtype != KASCADE_DTYPE_BF16) return KASCADE_ERR_UNSUPPORTED;
+  if (!v_pages || !page_table) return KASCADE_ERR_INVALID_ARG;
+  rc = check_tensors(q, k_pages, v_pages, o);
+  if (rc) return rc;
+  if (page_size < 16 || page_size > (1 << 20) || (page_size & (page_size - 1)) != 0) return KASCADE_ERR_UNSUPPORTED;
+  if (max_pages < (s->kv_len + page_size - 1) / page_size) return KASCADE_ERR_INVALID_ARG;
+  if (!aligned(page_table, 4) || (idx && !aligned(idx, 4)) || (head_map && !aligned(head_map, 4)) ||
+      (lse && !aligned(lse, 4)))
+    return KASCADE_ERR_UNSUPPORTED;
+  AttnArgs a = attn_args(s, q, k_pages, v_pages, idx, head_map, o, lse);
+  a.err = err_word(ws, ws_bytes);
+  a.page_table = page_table;
+  a.page_size = page_size;
+  a.max_pages = max_pages;
+  int sh = 0;
+  while ((1 << sh) < page_size) ++sh;
+  a.page_shift = sh;
   return cuda_status(launch_decode_attn(a, static_cast<cudaStream_t>(stream)));
 }
 

@@ -132,8 +132,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const AttnArgs
   const int hm_raw = a.one_list ? 0 : (a.head_map ? a.head_map[h] : h);
   const bool hm_ok = hm_raw >= 0 && hm_raw < a.n_lists;
   const int hm = hm_ok ? hm_raw : 0;
-  const int list_full = a.idx ? topk_count(a.N, a.num, a.den) : a.N;
-  const int list_len = hm_ok ? list_full : 0;
+  const int list_full = a.idx ? topk_count(a.N, a.num, a.den) : a.N;   // list stride
+  // a varlen row attends over its own first ceil(frac N_b) entries (dense: N_b keys)
+  const int n_b = a.kv_lens ? min(a.N, a.kv_lens[b]) : a.N;
+  const int list_len = hm_ok ? (a.idx ? topk_count(n_b, a.num, a.den) : n_b) : 0;
   const int32_t* list = a.idx ? a.idx + (size_t)(b * a.n_lists + hm) * list_full : nullptr;
   const int c0 = min(list_len, rank * per);
   const int c1 = min(list_len, c0 + per);
@@ -141,8 +143,17 @@ __global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const AttnArgs
   int* idx_s = reinterpret_cast<int*>(smem + L::idx);
   const bool staged = list != nullptr && (c1 - c0) <= kIdxStage;
   const size_t slab = (size_t)kv_slab_of(b, h * G, a.Hkv, a.Gkv);
-  const __nv_bfloat16* kb = a.k + slab * a.N * D;
-  const __nv_bfloat16* vb = a.v + slab * a.N * D;
+  // contiguous cache: row key of the slab; paged cache: row key % P of page
+  // page_table[b][key / P], pages [num_pages, Hkv, P, D]
+  const int kvh = (int)(slab - (size_t)b * a.Hkv);
+  const __nv_bfloat16* kb = a.page_table ? a.k + (size_t)kvh * a.page_size * D : a.k + slab * a.N * D;
+  const __nv_bfloat16* vb = a.page_table ? a.v + (size_t)kvh * a.page_size * D : a.v + slab * a.N * D;
+  const int32_t* ptab = a.page_table ? a.page_table + (size_t)b * a.max_pages : nullptr;
+  auto row_off = [&](int key) -> size_t {
+    if (!ptab) return (size_t)key * D;
+    const int pg = __ldg(ptab + (key >> a.page_shift));
+    return ((size_t)pg * a.Hkv * a.page_size + (key & (a.page_size - 1))) * D;
+  };
 
   if (staged)
     for (int i = threadIdx.x; i < c1 - c0; i += kThreads) idx_s[i] = __ldg(list + c0 + i);
@@ -165,7 +176,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const AttnArgs
       const bool have = c0 + rel < c1;
       const int key = have ? key_of(rel) : 0;
       const int pch = is_k ? (ch ^ ((r & 1) << 2)) : (ch ^ (r & 7));
-      cp_async_16(dst + r * L::ROWB + pch * 16, base + (size_t)key * D + ch * 8, have ? 16 : 0);
+      cp_async_16(dst + r * L::ROWB + pch * 16, base + row_off(key) + ch * 8, have ? 16 : 0);
     }
   };
   // K rows g and 8+g of slice s into registers (zero past the list end)
@@ -175,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const AttnArgs
     for (int t = 0; t < 2; ++t) {
       const int rel = s * 16 + t * 8 + g;
       const bool have = c0 + rel < c1;
-      const __nv_bfloat16* row = kb + (size_t)(have ? key_of(rel) : 0) * D + 8 * c;
+      const __nv_bfloat16* row = kb + row_off(have ? key_of(rel) : 0) + 8 * c;
 #pragma unroll
       for (int q = 0; q < KS; ++q) kr[t][q] = have ? ldg_nc_v4(row + 32 * q) : make_uint4(0, 0, 0, 0);
     }

@@ -28,7 +28,7 @@ __global__ void __launch_bounds__(kScoreWarps * 32)
                         float* __restrict__ s2, float* __restrict__ m_part,
                         double* __restrict__ l_part, int N, int Hq, int Hkv, int G, int splits,
                         float scale2, const int32_t* __restrict__ cand, const int32_t* __restrict__ cand_map,
-                        int cand_lists, int n_ctx) {
+                        int cand_lists, int n_ctx, const int32_t* __restrict__ kv_lens) {
   pdl_wait();
   pdl_launch_dependents();
   constexpr int CH = D / 32;
@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(kScoreWarps * 32)
     clist = cand + (size_t)(b * cand_lists + hm) * N;
   }
   const int j0 = split * KEYS;
-  const int j1 = min(N, j0 + KEYS);
+  const int j1 = min(kv_lens ? min(N, kv_lens[b]) : N, j0 + KEYS);   // a varlen row ends at its own length
 
   float sc[kGroupsPerWarp][4];
   uint4 ra[CH], rb[CH];
@@ -140,8 +140,8 @@ __global__ void __launch_bounds__(kScoreWarps * 32)
   float su0 = 0.f, su1 = 0.f;
 #pragma unroll
   for (int it = 0; it < kGroupsPerWarp; ++it) {
-    su0 += exp2f(sc[it][0] - m0) + exp2f(sc[it][2] - m0);
-    su1 += exp2f(sc[it][1] - m1) + exp2f(sc[it][3] - m1);
+    if (m0 != -INFINITY) su0 += exp2f(sc[it][0] - m0) + exp2f(sc[it][2] - m0);   // a split past a
+    if (m1 != -INFINITY) su1 += exp2f(sc[it][1] - m1) + exp2f(sc[it][3] - m1);   // varlen row's end: 0
   }
   double d0 = su0, d1 = su1;
 #pragma unroll
@@ -182,10 +182,10 @@ cudaError_t launch_decode_score(const DecodeScoreArgs& a, cudaStream_t stream) {
   if (a.D == 128)
     return launch_ex(decode_score_kernel<128>, grid, dim3(kScoreWarps * 32), 0, stream, pdl, 1, a.q, a.k, a.s2,
                      a.m_part, a.l_part, a.N, a.Hq, a.Hkv, a.G, splits, scale2, a.cand, a.cand_map, a.cand_lists,
-                     n_ctx);
+                     n_ctx, a.kv_lens);
   return launch_ex(decode_score_kernel<64>, grid, dim3(kScoreWarps * 32), 0, stream, pdl, 1, a.q, a.k, a.s2,
                    a.m_part, a.l_part, a.N, a.Hq, a.Hkv, a.G, splits, scale2, a.cand, a.cand_map, a.cand_lists,
-                   n_ctx);
+                   n_ctx, a.kv_lens);
 }
 
 }  // namespace kascade

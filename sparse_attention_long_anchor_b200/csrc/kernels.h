@@ -30,6 +30,7 @@ struct DecodeScoreArgs {
   const int32_t* cand_map;
   int cand_lists;
   int n_ctx;
+  const int32_t* kv_lens;  // varlen: batch row b scores keys [0, kv_lens[b]) (NULL: all N)
 };
 int decode_score_keys_per_split();
 cudaError_t launch_decode_score(const DecodeScoreArgs& a, cudaStream_t stream);
@@ -49,6 +50,8 @@ struct SelArgs {
   const int32_t* cand_map;
   int cand_lists;
   int n_ctx;
+  const int32_t* kv_lens;  // decode varlen: batch row b selects among keys [0, kv_lens[b]) (NULL: N);
+                           // lists keep the stride of N and end in -1 past ceil(frac kv_lens[b])
   const __nv_bfloat16* q;  // [B, Hq, Lq, D]
   const __nv_bfloat16* k;  // [B, Hkv, N, D]
   // decode inputs
@@ -114,6 +117,13 @@ struct AttnArgs {
   int Hp;                    // problems per batch row (G = query heads per problem)
   int Gkv;                   // query heads per kv head
   int q0, Lq;                // prefill: query (and o, lse) rows are positions [q0, q0 + Lq = N)
+  // decode over a paged cache (NULL: contiguous slabs): k and v are pages
+  // [num_pages, Hkv, page_size, D]; key j of batch row b is row j % page_size
+  // of page page_table[b * max_pages + j / page_size]
+  const int32_t* page_table;
+  int page_size, page_shift, max_pages;
+  const int32_t* kv_lens;    // decode varlen: batch row b attends over its first ceil(frac kv_lens[b])
+                             // list entries (dense: keys [0, kv_lens[b])); NULL: all
   int n_lists;               // index lists per batch row
   bool one_list;             // every problem reads list 0 of its row (head_map unused)
   bool causal;               // prefill dense only

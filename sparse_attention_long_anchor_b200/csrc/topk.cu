@@ -397,6 +397,10 @@ __global__ void __launch_bounds__(NT, kSelCtasPerSM) select_kernel(const SelArgs
       p.t = 0;
       p.n = a.N;
       p.k = (int)K;
+      if (a.kv_lens) {   // varlen row: its own candidates and budget
+        p.n = min(a.N, a.kv_lens[p.b]);
+        p.k = topk_count(p.n, a.num, a.den);
+      }
       p.cand = nullptr;
       if (a.cand) {
         int hm = a.cand_map ? a.cand_map[p.h] : p.h;
@@ -408,6 +412,7 @@ __global__ void __launch_bounds__(NT, kSelCtasPerSM) select_kernel(const SelArgs
       p.v = vscr;
       p.out = a.idx + (size_t)prob * K;
       run_problem<NT>(a, p, sh, vscr, band_idx, band_val, state, dyn);
+      for (int j = p.k + threadIdx.x; j < K; j += NT) p.out[j] = -1;   // a varlen row's unused tail
       __syncthreads();
     }
   } else {

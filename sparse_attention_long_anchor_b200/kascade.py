@@ -16,11 +16,11 @@ __all__ = ["Shape", "KascadeError", "lib", "OP_SELECT", "OP_SPARSE_DECODE", "OP_
            "OP_DENSE", "workspace_bytes", "index_count", "index_offsets", "Workspace", "select",
            "sparse_decode", "sparse_prefill", "dense_ref", "status_str", "launch_count", "EXPORTS", "LIB_PATH",
            "select_decode_static", "select_decode_static_error", "refine_select", "OP_REFINE",
-           "index_overlap", "plan_anchors"]
+           "index_overlap", "plan_anchors", "sparse_decode_paged", "select_varlen", "sparse_decode_varlen"]
 
 LIB_PATH = os.environ.get("KASCADE_LIB") or os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkascade.so")
 
-OP_SELECT, OP_SPARSE_DECODE, OP_SPARSE_PREFILL, OP_DENSE, OP_REFINE = 0, 1, 2, 3, 4
+OP_SELECT, OP_SPARSE_DECODE, OP_SPARSE_PREFILL, OP_DENSE, OP_REFINE, OP_SELECT_VARLEN = 0, 1, 2, 3, 4, 5
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TOO_LARGE = 0, 1, 2, 3, 4, 5
 FLAG_PDL, FLAG_INPUTS_STABLE, FLAG_TEST_DROP_LOAD = 1, 2, 1 << 30
 DEVERR_SCORE_POOL, DEVERR_DECODE_MERGE, DEVERR_PREFILL_ATTN, DEVERR_DECODE_SELECT = 2, 3, 4, 5
@@ -32,7 +32,8 @@ EXPORTS = ("kascade_workspace_bytes", "kascade_index_count", "kascade_index_offs
            "kascade_sparse_prefill", "kascade_dense_ref", "kascade_workspace_error",
            "kascade_status_str", "kascade_select_decode_static", "kascade_select_decode_static_max_bytes",
            "kascade_launch_count", "kascade_select_decode_static_error", "kascade_refine_select",
-           "kascade_index_overlap", "kascade_plan_anchors")
+           "kascade_index_overlap", "kascade_plan_anchors", "kascade_sparse_decode_paged",
+           "kascade_select_varlen", "kascade_sparse_decode_varlen")
 
 
 class KascadeError(RuntimeError):
@@ -91,6 +92,13 @@ def _load():
     so.kascade_dense_ref.restype = ctypes.c_int
     so.kascade_workspace_error.argtypes = [P, ctypes.POINTER(ctypes.c_int), ctypes.c_int, P]
     so.kascade_workspace_error.restype = ctypes.c_int
+    so.kascade_select_varlen.argtypes = [SP, P, P, P, P, P, ctypes.c_size_t, P]
+    so.kascade_select_varlen.restype = ctypes.c_int
+    so.kascade_sparse_decode_varlen.argtypes = [SP, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    so.kascade_sparse_decode_varlen.restype = ctypes.c_int
+    so.kascade_sparse_decode_paged.argtypes = [SP, P, P, P, P, ctypes.c_int32, ctypes.c_int32, P, P, P, P, P,
+                                               ctypes.c_size_t, P]
+    so.kascade_sparse_decode_paged.restype = ctypes.c_int
     so.kascade_index_overlap.argtypes = [SP, P, P, P, P]
     so.kascade_index_overlap.restype = ctypes.c_int
     so.kascade_plan_anchors.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.c_int32, ctypes.c_int32,
@@ -280,6 +288,46 @@ def sparse_decode(shape: Shape, q, k, v, idx, head_map=None, o=None, lse=None, w
     """kascade_sparse_decode: kv head h attends over anchor list head_map[h]."""
     return _attn(lib.kascade_sparse_decode, "kascade_sparse_decode", shape, q, k, v, idx, head_map, o, lse,
                  ws, stream, OP_SPARSE_DECODE)
+
+
+def select_varlen(shape: Shape, q, k, kv_lens, idx=None, ws=None, stream=None):
+    """kascade_select_varlen: decode selection with a context length per batch
+    row (lists padded with -1 to the layout of kv_len)."""
+    if idx is None:
+        idx = torch.empty(index_count(shape), dtype=torch.int32, device=q.device)
+    if ws is None:
+        ws = Workspace(shape, (OP_SELECT_VARLEN,))
+    p, n = ws.args()
+    _check(lib.kascade_select_varlen(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(kv_lens), _ptr(idx), p, n,
+                                     _stream(stream)), "kascade_select_varlen")
+    return idx
+
+
+def sparse_decode_varlen(shape: Shape, q, k, v, kv_lens, idx, head_map=None, o=None, lse=None, ws=None,
+                         stream=None):
+    """kascade_sparse_decode_varlen: sparse (idx None: dense) decode with a
+    context length per batch row."""
+    if o is None:
+        o = torch.empty_like(q)
+    p, n = _ws(ws, shape, OP_SPARSE_DECODE)
+    _check(lib.kascade_sparse_decode_varlen(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(kv_lens),
+                                            _ptr(idx), _ptr(head_map), _ptr(o), _ptr(lse), p, n, _stream(stream)),
+           "kascade_sparse_decode_varlen")
+    return o
+
+
+def sparse_decode_paged(shape: Shape, q, k_pages, v_pages, page_table, page_size: int, idx, head_map=None, o=None,
+                        lse=None, ws=None, stream=None):
+    """kascade_sparse_decode_paged: sparse (or, with idx None, dense) decode
+    over pages [num_pages, Hkv, page_size, d] named by page_table [B, max_pages]."""
+    if o is None:
+        o = torch.empty_like(q)
+    p, n = _ws(ws, shape, OP_SPARSE_DECODE)
+    _check(lib.kascade_sparse_decode_paged(ctypes.byref(shape), _ptr(q), _ptr(k_pages), _ptr(v_pages),
+                                           _ptr(page_table), int(page_size), int(page_table.shape[-1]), _ptr(idx),
+                                           _ptr(head_map), _ptr(o), _ptr(lse), p, n, _stream(stream)),
+           "kascade_sparse_decode_paged")
+    return o
 
 
 def sparse_prefill(shape: Shape, q, k, v, idx, head_map=None, o=None, lse=None, ws=None, stream=None):
