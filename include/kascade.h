@@ -47,7 +47,8 @@
  * Zero the workspace once before first use (kascade_workspace_init);
  * nothing else depends on its initial contents.  The attention calls need
  * only this 256-byte header (their partial results stay on chip) and accept
- * ws = NULL, in which case no error word is kept.  One workspace sized for
+ * ws = NULL, in which case no error word is kept (with
+ * KASCADE_FLAG_CHECK_INDICES they need more, below).  One workspace sized for
  * the largest op serves every call of a shape; calls that may run
  * concurrently must not share a workspace.
  *
@@ -90,6 +91,8 @@ extern "C" {
 #define KASCADE_DEVERR_DECODE_MERGE 3    /* sparse decode: a peer CTA's partial never arrived */
 #define KASCADE_DEVERR_PREFILL_ATTN 4    /* sparse prefill: a gather or MMA stage never completed */
 #define KASCADE_DEVERR_DECODE_SELECT 5   /* decode selection: a cluster exchange never completed */
+#define KASCADE_DEVERR_DECODE_GATHER 6   /* sparse decode: a bulk-copied K or V row never arrived */
+#define KASCADE_DEVERR_INDEX_LIST 7      /* KASCADE_FLAG_CHECK_INDICES: an index input out of range or unsorted */
 
 /* Operations for kascade_workspace_bytes(). */
 #define KASCADE_OP_SELECT 0
@@ -169,6 +172,23 @@ typedef struct kascade_shape {
  * reads KASCADE_DEVERR_SCORE_POOL and the call's outputs are not valid.  No
  * other call reads the flag. */
 #define KASCADE_FLAG_TEST_DROP_LOAD (1 << 30)
+/* Index validation, a debugging aid (the method has no counterpart): the
+ * sparse decode calls (contiguous, paged, varlen), kascade_sparse_prefill and
+ * kascade_refine_select first copy their index lists, head_map and kv_lens
+ * into the workspace through a checking kernel, and the attention or refine
+ * kernels read the copies.  Entries out of range (list entries outside the
+ * keys their list may name: [0, ceil(frac n_b)) entries in [0, n_b) for a
+ * decode row of n_b keys, tile t's entries in [0, min(32 (t + 1), N)), pool
+ * entries in [0, N); head_map outside [0, lists per row); kv_lens outside
+ * [1, N]) set the workspace error word to KASCADE_DEVERR_INDEX_LIST and are
+ * clamped into range in the copy, so no load leaves the K and V buffers;
+ * lists that are not strictly ascending set the word too.  The results of a
+ * call that set the word are not valid.  Page-table entries are not checked
+ * (the call carries no page count).  Requires a workspace of
+ * kascade_workspace_bytes(shape, op) with the flag in shape->flags (the
+ * copies live there); clears KASCADE_FLAG_INPUTS_STABLE for the call.  One
+ * extra launch per call. */
+#define KASCADE_FLAG_CHECK_INDICES 4
 
 /* Bytes of workspace that `op` needs for `shape` (0 on an invalid shape). */
 KASCADE_API size_t kascade_workspace_bytes(const kascade_shape* shape, int op);
@@ -177,7 +197,8 @@ KASCADE_API size_t kascade_workspace_bytes(const kascade_shape* shape, int op);
  * (what a CUDA graph capturing the call will hold): KASCADE_OP_SELECT
  * launches 1 for decode shapes whose scores fit on chip (fused scoring and
  * selection in one cluster launch) and 2 otherwise (scoring, then
- * selection); the attention ops launch 1.  Host-only query (it reads the
+ * selection); the attention ops launch 1 (2 with KASCADE_FLAG_CHECK_INDICES,
+ * except the dense form).  Host-only query (it reads the
  * device's cluster occupancy once).  Returns -1 on an invalid shape or op.
  * The pages describe no such call; it exists for callers that size graphs. */
 KASCADE_API int kascade_launch_count(const kascade_shape* shape, int op);

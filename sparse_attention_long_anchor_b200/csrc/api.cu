@@ -33,7 +33,8 @@ int check_shape(const kascade_shape* s) {
   // rolling chunk when q_len < kv_len), starting on a tile boundary
   if (s->q_len > s->kv_len || (s->q_len != 1 && (s->kv_len - s->q_len) % 32 != 0)) return KASCADE_ERR_UNSUPPORTED;
   if (s->q_len != 1 && s->tile != 32) return KASCADE_ERR_UNSUPPORTED;
-  if (s->flags & ~(KASCADE_FLAG_PDL | KASCADE_FLAG_INPUTS_STABLE | KASCADE_FLAG_TEST_DROP_LOAD))
+  if (s->flags & ~(KASCADE_FLAG_PDL | KASCADE_FLAG_INPUTS_STABLE | KASCADE_FLAG_CHECK_INDICES |
+                   KASCADE_FLAG_TEST_DROP_LOAD))
     return KASCADE_ERR_INVALID_ARG;
   if (s->select_mode < KASCADE_SELECT_GQA || s->select_mode > KASCADE_SELECT_ALL_HEADS) return KASCADE_ERR_INVALID_ARG;
   if (s->select_mode == KASCADE_SELECT_ALL_HEADS && s->num_q_heads > 64) return KASCADE_ERR_UNSUPPORTED;
@@ -197,6 +198,81 @@ int check_tensors(const void* q, const void* k, const void* v, const void* o) {
   return KASCADE_OK;
 }
 
+// ----------------------------------------------------------------- index checks
+
+bool checking(const kascade_shape* s) { return (s->flags & KASCADE_FLAG_CHECK_INDICES) != 0; }
+
+int64_t index_entries(const kascade_shape* s) {
+  const int64_t BH = (int64_t)s->batch * n_lists(s);
+  return is_decode(s) ? BH * topk_count(s->kv_len, s->topk_num, s->topk_den) : BH * prefill_row_len(s);
+}
+
+// the checked copies (index rows, head_map, kv_lens) carved at `offset`
+struct CheckPlan {
+  int32_t* idx;
+  int32_t* hm;
+  int32_t* kv;
+  size_t bytes;   // offset + the copies
+};
+CheckPlan plan_check(const kascade_shape* s, int64_t entries, size_t offset, void* ws) {
+  CheckPlan p{};
+  Carver cv{static_cast<char*>(ws), offset};
+  p.idx = cv.take<int32_t>((size_t)entries);
+  p.hm = cv.take<int32_t>((size_t)s->num_q_heads);
+  p.kv = cv.take<int32_t>((size_t)s->batch);
+  p.bytes = cv.off;
+  return p;
+}
+
+// Runs the checking kernel and points idx / head_map / kv_lens at the
+// copies.  rows: B * lists rows of row_len entries.
+int run_check(const kascade_shape* s, int lists, int64_t row_len, bool pool, const int32_t*& idx,
+              const int32_t*& head_map, const int32_t*& kv_lens, void* ws, size_t ws_bytes, size_t offset,
+              cudaStream_t st) {
+  const CheckPlan need = plan_check(s, (int64_t)s->batch * lists * row_len, offset, nullptr);
+  if (!ws || !aligned(ws, kAlign) || ws_bytes < need.bytes) return KASCADE_ERR_WORKSPACE;
+  const CheckPlan pl = plan_check(s, (int64_t)s->batch * lists * row_len, offset, ws);
+  CheckArgs c{};
+  c.idx = idx;
+  c.idx_out = pl.idx;
+  c.head_map = head_map;
+  c.hm_out = pl.hm;
+  c.n_map = head_map ? lists : 0;
+  c.kv_lens = kv_lens;
+  c.kv_out = pl.kv;
+  c.B = s->batch;
+  c.L = lists;
+  c.N = s->kv_len;
+  c.num = s->topk_num;
+  c.den = s->topk_den;
+  c.t0 = t_first(s);
+  c.row_len = row_len;
+  c.prefill = !is_decode(s);
+  c.pool = pool;
+  c.pdl = (s->flags & KASCADE_FLAG_PDL) != 0;
+  c.err = static_cast<int*>(ws);
+  const int rc = cuda_status(launch_check_lists(c, st));
+  if (rc) return rc;
+  idx = pl.idx;
+  if (head_map) head_map = pl.hm;
+  if (kv_lens) kv_lens = pl.kv;
+  return KASCADE_OK;
+}
+
+// KASCADE_FLAG_CHECK_INDICES for an attention call: checked copies of the
+// lists (none for the dense form), head_map and kv_lens
+int check_attn_inputs(const kascade_shape* s, AttnArgs& a, void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (!checking(s)) return KASCADE_OK;
+  const int64_t row_len =
+      !a.idx ? 0 : is_decode(s) ? topk_count(s->kv_len, s->topk_num, s->topk_den) : prefill_row_len(s);
+  const int32_t* hm = a.one_list ? nullptr : a.head_map;   // all heads pooled: one list, no map
+  const int rc = run_check(s, n_lists(s), row_len, false, a.idx, hm, a.kv_lens, ws, ws_bytes, kHeader, st);
+  if (rc) return rc;
+  if (!a.one_list) a.head_map = hm;
+  a.flags &= ~KASCADE_FLAG_INPUTS_STABLE;   // the copies are written just before
+  return KASCADE_OK;
+}
+
 AttnArgs attn_args(const kascade_shape* s, const void* q, const void* k, const void* v,
                    const int32_t* idx, const int32_t* head_map, void* o, float* lse) {
   AttnArgs a{};
@@ -246,10 +322,16 @@ size_t kascade_workspace_bytes(const kascade_shape* s, int op) {
       return plan_select(s, nullptr).bytes;
     case KASCADE_OP_SPARSE_DECODE:
     case KASCADE_OP_SPARSE_PREFILL:
+      // only the error word (partial results stay on chip), plus the checked
+      // index copies with KASCADE_FLAG_CHECK_INDICES
+      return checking(s) ? plan_check(s, index_entries(s), kHeader, nullptr).bytes : kHeader;
     case KASCADE_OP_DENSE:
-      return kHeader;   // only the error word: partial results stay on chip
-    case KASCADE_OP_REFINE:   // covers every pool length up to N
-      return is_decode(s) ? plan_refine(s, s->kv_len, nullptr).bytes : 0;
+      return kHeader;
+    case KASCADE_OP_REFINE: {   // covers every pool length up to N
+      if (!is_decode(s)) return 0;
+      const size_t b = plan_refine(s, s->kv_len, nullptr).bytes;
+      return checking(s) ? plan_check(s, (int64_t)s->batch * s->num_kv_heads * s->kv_len, b, nullptr).bytes : b;
+    }
     case KASCADE_OP_SELECT_VARLEN:
       return is_decode(s) ? plan_select(s, nullptr, true).bytes : 0;
     default:
@@ -281,7 +363,8 @@ int kascade_index_offsets(const kascade_shape* s, int64_t* offsets) {
 
 int kascade_launch_count(const kascade_shape* s, int op) {
   if (check_shape(s)) return -1;
-  if (op == KASCADE_OP_SPARSE_DECODE || op == KASCADE_OP_SPARSE_PREFILL || op == KASCADE_OP_DENSE) return 1;
+  if (op == KASCADE_OP_DENSE) return 1;
+  if (op == KASCADE_OP_SPARSE_DECODE || op == KASCADE_OP_SPARSE_PREFILL) return checking(s) ? 2 : 1;
   if (op != KASCADE_OP_SELECT) return -1;
   if (!is_decode(s)) return s->select_mode == KASCADE_SELECT_ALL_HEADS ? 3 : 2;
   if (s->select_mode == KASCADE_SELECT_ALL_HEADS || is_f32(s) || !select_decode_cluster_ok(s->kv_len)) return 2;
@@ -416,6 +499,11 @@ int kascade_refine_select(const kascade_shape* s, const void* q, const void* k, 
   pl = plan_refine(s, pool_len, ws);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int flags = s->flags & KASCADE_FLAG_PDL;
+  if (checking(s)) {
+    const int32_t* no_lens = nullptr;
+    rc = run_check(s, s->num_kv_heads, pool_len, true, pool, head_map, no_lens, ws, ws_bytes, pl.bytes, st);
+    if (rc) return rc;
+  }
   DecodeScoreArgs d{};
   d.flags = flags;
   d.q = static_cast<const __nv_bfloat16*>(q);
@@ -484,8 +572,11 @@ int kascade_sparse_decode(const kascade_shape* s, const void* q, const void* k, 
     return KASCADE_ERR_UNSUPPORTED;
   AttnArgs a = attn_args(s, q, k, v, idx, head_map, o, lse);
   a.err = err_word(ws, ws_bytes);
-  if (is_f32(s)) return cuda_status(launch_sparse_decode_f32(a, is_f16(s), static_cast<cudaStream_t>(stream)));
-  return cuda_status(launch_decode_attn(a, static_cast<cudaStream_t>(stream)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  rc = check_attn_inputs(s, a, ws, ws_bytes, st);
+  if (rc) return rc;
+  if (is_f32(s)) return cuda_status(launch_sparse_decode_f32(a, is_f16(s), st));
+  return cuda_status(launch_decode_attn(a, st));
 }
 
 int kascade_select_varlen(const kascade_shape* s, const void* q, const void* k, const int32_t* kv_lens,
@@ -564,7 +655,10 @@ int kascade_sparse_decode_varlen(const kascade_shape* s, const void* q, const vo
   AttnArgs a = attn_args(s, q, k, v, idx, head_map, o, lse);
   a.err = err_word(ws, ws_bytes);
   a.kv_lens = kv_lens;
-  return cuda_status(launch_decode_attn(a, static_cast<cudaStream_t>(stream)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  rc = check_attn_inputs(s, a, ws, ws_bytes, st);
+  if (rc) return rc;
+  return cuda_status(launch_decode_attn(a, st));
 }
 
 int kascade_sparse_decode_paged(const kascade_shape* s, const void* q, const void* k_pages, const void* v_pages,
@@ -590,7 +684,10 @@ int kascade_sparse_decode_paged(const kascade_shape* s, const void* q, const voi
   int sh = 0;
   while ((1 << sh) < page_size) ++sh;
   a.page_shift = sh;
-  return cuda_status(launch_decode_attn(a, static_cast<cudaStream_t>(stream)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  rc = check_attn_inputs(s, a, ws, ws_bytes, st);
+  if (rc) return rc;
+  return cuda_status(launch_decode_attn(a, st));
 }
 
 int kascade_sparse_prefill(const kascade_shape* s, const void* q, const void* k, const void* v,
@@ -607,8 +704,11 @@ int kascade_sparse_prefill(const kascade_shape* s, const void* q, const void* k,
     return KASCADE_ERR_UNSUPPORTED;
   AttnArgs a = attn_args(s, q, k, v, idx, head_map, o, lse);
   a.err = err_word(ws, ws_bytes);
-  if (is_f32(s)) return cuda_status(launch_sparse_prefill_f32(a, is_f16(s), static_cast<cudaStream_t>(stream)));
-  return cuda_status(launch_prefill(a, static_cast<cudaStream_t>(stream)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  rc = check_attn_inputs(s, a, ws, ws_bytes, st);
+  if (rc) return rc;
+  if (is_f32(s)) return cuda_status(launch_sparse_prefill_f32(a, is_f16(s), st));
+  return cuda_status(launch_prefill(a, st));
 }
 
 int kascade_dense_ref(const kascade_shape* s, const void* q, const void* k, const void* v, int causal,

@@ -1,5 +1,5 @@
-// Cluster size of the fused decode select (host side, plain C++ with no CUDA
-// dependency, so the rule is unit-tested on the CPU).
+// Cluster sizes of the decode select and the sparse decode (host side, plain
+// C++ with no CUDA dependency, so the rules are unit-tested on the CPU).
 //
 // One thread-block cluster handles one (batch, kv head) problem; its CTAs
 // split the problem's keys, so K streams at a rate that grows with the
@@ -26,6 +26,26 @@ inline int choose_cluster_size(long long problems, const int* sizes, const int* 
     }
   }
   return best;
+}
+
+// Waves that `problems` clusters of the chosen size take (0 if `chosen` is
+// not one of sizes[] or none of it runs).
+inline long long cluster_waves(long long problems, const int* sizes, const int* active, int n, int chosen) {
+  for (int i = 0; i < n; ++i)
+    if (sizes[i] == chosen && active[i] > 0) return problems <= 0 ? 1 : (problems + active[i] - 1) / active[i];
+  return 0;
+}
+
+// The fused decode select keeps a problem's scores on chip and runs its
+// Top-k right after the scoring, so the SMs of a finished wave wait out the
+// Top-k of the slowest cluster before the next wave's K stream starts.  It
+// is taken only when every problem runs in one wave; with more, scoring into
+// global memory at full occupancy and selecting in a second kernel is
+// faster (batch 8 of the 8-kv-head shape at 64K keys: 271 us against 348).
+inline int choose_fused_select_size(long long problems, const int* sizes, const int* active, const bool* fits,
+                                    int n) {
+  const int cs = choose_cluster_size(problems, sizes, active, fits, n);
+  return cs && cluster_waves(problems, sizes, active, n, cs) == 1 ? cs : 0;
 }
 
 }  // namespace kascade

@@ -44,8 +44,10 @@ namespace {
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kMaxCS = 16;
-constexpr int kIdxStage = 2048;     // index entries staged in shared memory (a 4-CTA cluster's share of 64K at 10 %)
+constexpr int kIdxStage = 512;      // index entries staged in shared memory, modes 0 and 1
+constexpr int kIdxStageB = 3584;    // the bulk mode's (a 2-CTA cluster's share of 64K at 10 %)
 constexpr int kErrMergeTimeout = 3; // device error word: a merge wait gave up
+constexpr int kErrGather = 6;       // device error word: a bulk-copied row never arrived
 
 template <int D>
 struct Lay {
@@ -53,9 +55,10 @@ struct Lay {
   static constexpr int SLAB = 16 * ROWB;                   // one 16-key slab
   static constexpr int WARPB = 3 * SLAB;                   // V slot 0, V slot 1, K slot
   static constexpr size_t slabs = 0;
+  static constexpr int IDXN = kIdxStage;
   static constexpr size_t qs = slabs + (size_t)kWarps * WARPB;   // [8][D] bf16 query rows
   static constexpr size_t idx = qs + 8 * D * 2;
-  static constexpr size_t recv_o = idx + kIdxStage * 4;    // [G*D] f32, written by the peers
+  static constexpr size_t recv_o = idx + IDXN * 4;         // [G*D] f32, written by the peers
   static constexpr size_t recv_ml = recv_o + 8 * D * 4;    // [16][8] (m, l)
   static constexpr size_t bar = recv_ml + kMaxCS * 8 * 8;  // mbarrier of the incoming partials
   static constexpr size_t total = bar + 16;
@@ -72,6 +75,52 @@ struct Lay {
   // two CTAs per SM: 228 KB per SM less 1 KB reserved per CTA
   static_assert(total <= (228 * 1024 - 2 * 1024) / 2, "two CTAs per SM");
 };
+
+// Bulk mode (many keys per CTA, one CTA per SM): each warp owns kStagesB
+// stages of one 16-key slice, K rows then V rows, every row landing by one
+// untiled bulk copy at a padded pitch of 2 D + 16 bytes.  Rows at that pitch
+// shift by one 16-byte bank group, so the ldmatrix.trans reads of V (8 rows,
+// one chunk) and the K reads below (lane (g, c) takes chunks
+// 8 (q>>1) + 2c + (q&1) of rows g and g + 8) are conflict-free.
+constexpr int kStagesB = 3;
+
+template <int D>
+struct BLay {
+  static constexpr int ROWB = D * 2;
+  static constexpr int PITCH = ROWB + 16;
+  static constexpr int TB = 16 * PITCH;                    // 16 rows of one tensor
+  static constexpr int STAGE = 2 * TB;                     // K rows, then V rows
+  static constexpr int WARPB = kStagesB * STAGE;
+  static constexpr int SLAB = 16 * ROWB;                   // (the two-slab modes' unit; unused here)
+  static constexpr int IDXN = kIdxStageB;
+  static constexpr size_t slabs = 0;
+  static constexpr size_t qs = slabs + (size_t)kWarps * WARPB;
+  static constexpr size_t idx = qs + 8 * D * 2;
+  static constexpr size_t recv_o = idx + IDXN * 4;
+  static constexpr size_t recv_ml = recv_o + 8 * D * 4;
+  static constexpr size_t bar = recv_ml + kMaxCS * 8 * 8;
+  static constexpr size_t sbar = bar + 16;                 // [warps][stages] mbarriers of the stages
+  static constexpr size_t total = sbar + (size_t)kWarps * kStagesB * 8;
+  static constexpr int RO = D + 4;
+  static constexpr size_t red_o = 0;
+  static constexpr size_t red_ml = red_o + (size_t)kWarps * 8 * RO * 4;
+  static constexpr size_t wf = red_ml + kWarps * 8 * 8;
+  static constexpr size_t pml = wf + kWarps * 8 * 4;
+  static constexpr size_t wts = pml + 8 * 8;
+  static constexpr size_t head = wts + kMaxCS * 8 * 4;
+  static_assert(PITCH % 16 == 0 && (PITCH / 16) % 8 == 1, "pitch must shift rows by one 16-byte bank group");
+  static_assert(head + 8 * 8 <= qs, "post-loop scratch must fit in the stages");
+  static_assert(recv_o % 16 == 0 && recv_ml % 8 == 0 && bar % 8 == 0, "alignment");
+  static_assert(total <= 227 * 1024, "one CTA per SM");
+};
+
+// kMode bits 0-1: 0 = every warp owns at most two slices, all issued up
+// front by cp.async (two CTAs per SM); 2 = bulk-copied stages refilled as
+// they are consumed (one CTA per SM).  Bit 2 (kPagedBit): rows addressed
+// through a page table.
+constexpr int kPagedBit = 4;
+template <int D, int kMode>
+using LayOf = typename std::conditional<(kMode & 3) == 2, BLay<D>, Lay<D>>::type;
 
 __device__ __forceinline__ float scale_from(float m_old, float m_new) {
   return m_old == -INFINITY ? 0.0f : exp2f(m_old - m_new);
@@ -93,11 +142,15 @@ __device__ __forceinline__ void merge_weights(int n, const float2* ml, float* w,
   if (lane == 0) *out = make_float2(M, ls);
 }
 
-// kRing = false: every warp owns at most two slices (per <= 16 * 2 * kWarps),
-// all issued up front; kRing = true: the slabs are refilled two slices ahead.
-template <int D, bool kRing>
-__global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const AttnArgs a, int per) {
-  using L = Lay<D>;
+// kMode & 3 == 0: every warp owns at most two slices (per <= 16 * 2 *
+// kWarps), all issued up front; == 2: kStagesB bulk-copied stages per warp
+// refilled as they are consumed (one CTA per SM, for many keys per CTA).
+// kMode & kPagedBit: K and V rows through the page table.
+template <int D, int kMode>
+__global__ void __launch_bounds__(kThreads, (kMode & 3) == 2 ? 1 : 2) decode_attn_kernel(const AttnArgs a, int per) {
+  using L = LayOf<D, kMode>;
+  constexpr bool kBulk = (kMode & 3) == 2;
+  constexpr bool kPaged = (kMode & kPagedBit) != 0;
   constexpr int KS = D / 32;          // 16-byte K loads per key row per lane
   constexpr int CH = D / 8;           // 16-byte chunks per row
   extern __shared__ __align__(128) char smem[];
@@ -127,6 +180,15 @@ __global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const AttnArgs
     mbar_arrive_expect_tx(bar, (uint32_t)(E * 4 + CS * G * 8));
   }
   cluster_arrive_release();   // the matching wait comes before the first push
+  [[maybe_unused]] const uint32_t sbar0 =
+      kBulk ? sbase + (uint32_t)(BLay<D>::sbar + warp * kStagesB * 8) : 0u;
+  if constexpr (kBulk) {
+    if (lane == 0) {
+      for (int st = 0; st < kStagesB; ++st) mbar_init(sbar0 + 8 * st, 1);
+      mbar_fence_init();
+    }
+    __syncwarp();
+  }
 
   // an out-of-range head_map entry reads as an empty list (output 0, lse -inf)
   const int hm_raw = a.one_list ? 0 : (a.head_map ? a.head_map[h] : h);
@@ -141,18 +203,21 @@ __global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const AttnArgs
   const int c1 = min(list_len, c0 + per);
   const int n_slices = (c1 - c0 + 15) / 16;
   int* idx_s = reinterpret_cast<int*>(smem + L::idx);
-  const bool staged = list != nullptr && (c1 - c0) <= kIdxStage;
+  const bool staged = list != nullptr && (c1 - c0) <= L::IDXN;
   const size_t slab = (size_t)kv_slab_of(b, h * G, a.Hkv, a.Gkv);
   // contiguous cache: row key of the slab; paged cache: row key % P of page
   // page_table[b][key / P], pages [num_pages, Hkv, P, D]
   const int kvh = (int)(slab - (size_t)b * a.Hkv);
-  const __nv_bfloat16* kb = a.page_table ? a.k + (size_t)kvh * a.page_size * D : a.k + slab * a.N * D;
-  const __nv_bfloat16* vb = a.page_table ? a.v + (size_t)kvh * a.page_size * D : a.v + slab * a.N * D;
-  const int32_t* ptab = a.page_table ? a.page_table + (size_t)b * a.max_pages : nullptr;
+  const __nv_bfloat16* kb = kPaged ? a.k + (size_t)kvh * a.page_size * D : a.k + slab * a.N * D;
+  const __nv_bfloat16* vb = kPaged ? a.v + (size_t)kvh * a.page_size * D : a.v + slab * a.N * D;
+  [[maybe_unused]] const int32_t* ptab = kPaged ? a.page_table + (size_t)b * a.max_pages : nullptr;
   auto row_off = [&](int key) -> size_t {
-    if (!ptab) return (size_t)key * D;
-    const int pg = __ldg(ptab + (key >> a.page_shift));
-    return ((size_t)pg * a.Hkv * a.page_size + (key & (a.page_size - 1))) * D;
+    if constexpr (kPaged) {
+      const int pg = __ldg(ptab + (key >> a.page_shift));
+      return ((size_t)pg * a.Hkv * a.page_size + (key & (a.page_size - 1))) * D;
+    } else {
+      return (size_t)key * D;
+    }
   };
 
   if (staged)
@@ -201,15 +266,35 @@ __global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const AttnArgs
   const float scale2 = kLog2e * rsqrtf((float)D);
   const char* qrow = smem + L::qs + (size_t)(g * D + 8 * c) * 2;
 
-  // prologue: this warp's first two slices (one cp.async group each)
-  if (warp < n_slices) issue_rows(warp, wbase, vb, false);
-  if constexpr (kRing) cp_async_commit();
-  if (warp + kWarps < n_slices) {
-    issue_rows(warp + kWarps, wbase + L::SLAB, vb, false);
-    issue_rows(warp + kWarps, kslot, kb, true);
+  // bulk mode: this warp's slices warp, warp + kWarps, ..., the it-th in
+  // stage it % kStagesB; K rows by lanes 0-15, V rows by lanes 16-31, rows
+  // past the list repeating its last key (finite data, masked out)
+  const int n_my = warp < n_slices ? (n_slices - warp + kWarps - 1) / kWarps : 0;
+  [[maybe_unused]] auto issue_bulk = [&](int it) {
+    using B = BLay<D>;
+    const int sl = warp + kWarps * it;
+    const int st = it % kStagesB;
+    const uint32_t sb = sbar0 + 8 * st;
+    if (lane == 0) mbar_arrive_expect_tx(sb, (uint32_t)(2 * 16 * B::ROWB));
+    __syncwarp();
+    const int r = lane & 15;
+    const int rel = min(sl * 16 + r, c1 - c0 - 1);
+    bulk_g2s(wbase + (uint32_t)(st * B::STAGE + (lane < 16 ? 0 : B::TB) + r * B::PITCH),
+             (lane < 16 ? kb : vb) + row_off(key_of(rel)), (uint32_t)B::ROWB, sb);
+  };
+
+  if constexpr (kBulk) {
+    for (int j = 0; j < kStagesB && j < n_my; ++j) issue_bulk(j);
+  } else {
+    // prologue: this warp's first two slices
+    if (warp < n_slices) issue_rows(warp, wbase, vb, false);
+    if (warp + kWarps < n_slices) {
+      issue_rows(warp + kWarps, wbase + L::SLAB, vb, false);
+      issue_rows(warp + kWarps, kslot, kb, true);
+    }
+    cp_async_commit();
+    if (warp < n_slices) load_k(warp);
   }
-  cp_async_commit();
-  if (warp < n_slices) load_k(warp);
   if (early) {
     pdl_wait();
     pdl_launch_dependents();
@@ -362,24 +447,83 @@ __global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const AttnArgs
     }
   };
 
-  if constexpr (kRing) {
-    int it = 0;
-    for (int s = warp; s < n_slices; s += kWarps, ++it) {
-      cp_async_wait<1>();   // the group of slice `it`; one later group is always committed
-      __syncwarp();
-      const int slot = it & 1;
-      if (slot) step(s, 1, std::true_type{});
-      else step(s, 0, std::false_type{});
-      __syncwarp();
-      // refill what this slice used with the slice two iterations ahead
-      const int s2 = s + 2 * kWarps;
-      if (s2 < n_slices) {
-        issue_rows(s2, wbase + slot * L::SLAB, vb, false);
-        if (slot) issue_rows(s2, kslot, kb, true);
-      }
-      cp_async_commit();
-      if (!slot && s2 < n_slices) load_k(s2);
+  // bulk mode: one slice from stage st (K reads in the pitch-padded chunk
+  // order above; the query rows read with the same chunk order)
+  [[maybe_unused]] auto step_bulk = [&](int sl, int st) {
+    using B = BLay<D>;
+    const uint32_t kst = wbase + (uint32_t)(st * B::STAGE);
+    const uint32_t vst = kst + (uint32_t)B::TB;
+    const char* qg = smem + L::qs + (size_t)(g * D) * 2;
+    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int q = 0; q < KS; ++q) {
+      const int ch = 8 * (q >> 1) + 2 * c + (q & 1);
+      const uint2 qlo = *reinterpret_cast<const uint2*>(qg + ch * 16);
+      const uint2 qhi = *reinterpret_cast<const uint2*>(qg + ch * 16 + 8);
+      const uint4 k0 = lds_v4(kst + g * B::PITCH + ch * 16);
+      const uint4 k1 = lds_v4(kst + (8 + g) * B::PITCH + ch * 16);
+      const uint32_t a0[4] = {k0.x, k1.x, k0.y, k1.y};
+      const uint32_t a1[4] = {k0.z, k1.z, k0.w, k1.w};
+      mma_bf16_16816(q & 1 ? sb : sa, a0, qlo.x, qlo.y);
+      mma_bf16_16816(q & 1 ? sb : sa, a1, qhi.x, qhi.y);
     }
+    const int kbase = c0 + sl * 16;
+    const bool v_lo = kbase + g < c1, v_hi = kbase + 8 + g < c1;
+    float sv[4];
+    sv[0] = v_lo ? (sa[0] + sb[0]) * scale2 : -INFINITY;
+    sv[1] = v_lo ? (sa[1] + sb[1]) * scale2 : -INFINITY;
+    sv[2] = v_hi ? (sa[2] + sb[2]) * scale2 : -INFINITY;
+    sv[3] = v_hi ? (sa[3] + sb[3]) * scale2 : -INFINITY;
+    float mx0 = fmaxf(sv[0], sv[2]), mx1 = fmaxf(sv[1], sv[3]);
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+    const float al0 = scale_from(m_run[0], mn0), al1 = scale_from(m_run[1], mn1);
+    const float p0 = exp2f(sv[0] - mn0), p1 = exp2f(sv[1] - mn1);
+    const float p2 = exp2f(sv[2] - mn0), p3 = exp2f(sv[3] - mn1);
+    l_run[0] = l_run[0] * al0 + (p0 + p2);
+    l_run[1] = l_run[1] * al1 + (p1 + p3);
+    m_run[0] = mn0;
+    m_run[1] = mn1;
+    const uint32_t b0 = movmatrix_trans(pack_bf16(p0, p1));
+    const uint32_t b1 = movmatrix_trans(pack_bf16(p2, p3));
+    const int vrow = ((lane >> 4) << 3) + (lane & 7);
+    const int vch = (lane >> 3) & 1;
+#pragma unroll
+    for (int i = 0; i < D / 16; ++i) {
+      uint32_t r4[4];
+      ldmatrix_x4_trans(r4, vst + vrow * B::PITCH + (2 * i + vch) * 16);
+      float t[4] = {oacc[i][0] * al0, oacc[i][1] * al1, oacc[i][2] * al0, oacc[i][3] * al1};
+      mma_bf16_16816(t, r4, b0, b1);
+      oacc[i][0] = t[0];
+      oacc[i][1] = t[1];
+      oacc[i][2] = t[2];
+      oacc[i][3] = t[3];
+    }
+  };
+
+  if constexpr (kBulk) {
+    int it = 0;
+    bool failed = false;
+    for (; it < n_my; ++it) {
+      const int st = it % kStagesB;
+      if (!mbar_wait_bounded(sbar0 + 8 * st, (uint32_t)((it / kStagesB) & 1))) {
+        if (lane == 0) raise_error(a.err, kErrGather);
+        failed = true;
+        break;
+      }
+      step_bulk(warp + kWarps * it, st);
+      __syncwarp();   // every lane is done with stage st
+      if (it + kStagesB < n_my) issue_bulk(it + kStagesB);
+    }
+    // after a wait gave up: let the copies still in flight land (bounded)
+    // before the stages become the merge's scratch
+    if (failed)
+      for (int j = it + 1; j < n_my && j < it + kStagesB; ++j)
+        mbar_wait_bounded(sbar0 + 8 * (j % kStagesB), (uint32_t)((j / kStagesB) & 1));
   } else {
     cp_async_wait<0>();
     __syncwarp();
@@ -465,12 +609,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const AttnArgs
   }
 }
 
-template <int D, bool kRing>
+template <int D, int kMode>
 cudaLaunchConfig_t make_cfg(int cs, int bh, cudaStream_t stream, cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cs, bh, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = Lay<D>::total;
+  cfg.dynamicSmemBytes = LayOf<D, kMode>::total;
   cfg.stream = stream;
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = cs;
@@ -482,26 +626,28 @@ cudaLaunchConfig_t make_cfg(int cs, int bh, cudaStream_t stream, cudaLaunchAttri
 }
 
 // Cluster sizes of the sparse decode, largest first.  One cluster per
-// (batch, kv head) problem: at batch 1 the largest cluster spreads the
-// gathers widest (the kernel is latency-bound there); with many problems the
-// fewest waves matter (choose_cluster_size).
-constexpr int kDecSizes[] = {16, 8, 4};
-constexpr int kNumDecSizes = 3;
+// (batch, list) problem: at batch 1 the largest cluster spreads the gathers
+// widest (the kernel is latency-bound there); with many problems the fewest
+// waves matter (choose_cluster_size).  The bulk mode (one CTA per SM) also
+// takes pairs, so 64 problems still fit one wave.
+constexpr int kDecSizes[] = {16, 8, 4, 2};
+constexpr int kNumDecSizes = 4;
 
-template <int D, bool kRing>
+template <int D, int kMode>
 int decode_cluster_size(long long problems) {
   static int cached[64][kNumDecSizes] = {{0}};   // max active clusters + 1 (0 = unknown)
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 8;
+  const int n_sizes = (kMode & 3) == 2 ? kNumDecSizes : kNumDecSizes - 1;
   if (!cached[dev][0]) {
-    for (int i = 0; i < kNumDecSizes; ++i) {
+    for (int i = 0; i < n_sizes; ++i) {
       const int cs = kDecSizes[i];
       int n = 0;
-      if (ensure_func_attrs(reinterpret_cast<const void*>(decode_attn_kernel<D, kRing>), Lay<D>::total, cs > 8) ==
-          cudaSuccess) {
+      if (ensure_func_attrs(reinterpret_cast<const void*>(decode_attn_kernel<D, kMode>), LayOf<D, kMode>::total,
+                            cs > 8) == cudaSuccess) {
         cudaLaunchAttribute attr[1];
-        cudaLaunchConfig_t cfg = make_cfg<D, kRing>(cs, 1, nullptr, attr);
-        if (cudaOccupancyMaxActiveClusters(&n, decode_attn_kernel<D, kRing>, &cfg) != cudaSuccess) n = 0;
+        cudaLaunchConfig_t cfg = make_cfg<D, kMode>(cs, 1, nullptr, attr);
+        if (cudaOccupancyMaxActiveClusters(&n, decode_attn_kernel<D, kMode>, &cfg) != cudaSuccess) n = 0;
       }
       cached[dev][i] = 1 + n;
     }
@@ -509,40 +655,49 @@ int decode_cluster_size(long long problems) {
   }
   int active[kNumDecSizes];
   bool fits[kNumDecSizes];
-  for (int i = 0; i < kNumDecSizes; ++i) {
+  for (int i = 0; i < n_sizes; ++i) {
     active[i] = cached[dev][i] - 1;
     fits[i] = true;
   }
-  const int cs = choose_cluster_size(problems, kDecSizes, active, fits, kNumDecSizes);
+  const int cs = choose_cluster_size(problems, kDecSizes, active, fits, n_sizes);
   return cs > 0 ? cs : 8;
 }
 
-template <int D, bool kRing>
+template <int D, int kMode>
 cudaError_t launch_cs(const AttnArgs& a, int cs, int per, cudaStream_t stream) {
-  const cudaError_t e =
-      ensure_func_attrs(reinterpret_cast<const void*>(decode_attn_kernel<D, kRing>), Lay<D>::total, cs > 8);
+  const size_t smem = LayOf<D, kMode>::total;
+  const cudaError_t e = ensure_func_attrs(reinterpret_cast<const void*>(decode_attn_kernel<D, kMode>), smem, cs > 8);
   if (e != cudaSuccess) return e;
-  return launch_ex(decode_attn_kernel<D, kRing>, dim3(cs, a.B * a.Hp), dim3(kThreads), Lay<D>::total, stream,
+  return launch_ex(decode_attn_kernel<D, kMode>, dim3(cs, a.B * a.Hp), dim3(kThreads), smem, stream,
                    (a.flags & 1) != 0, cs, a, per);
 }
 
-template <int D>
-cudaError_t launch(const AttnArgs& a, cudaStream_t stream) {
-  // both variants share the shared-memory size and cluster shape, so one
-  // occupancy answer serves both
-  const int cs = decode_cluster_size<D, false>((long long)a.B * a.Hp);
-  const int list_len = a.idx ? topk_count(a.N, a.num, a.den) : a.N;
+int share_of(int list_len, int cs) {
   int per = (list_len + cs - 1) / cs;
   per = (per + 15) / 16 * 16;
-  if (per < 16) per = 16;
+  return per < 16 ? 16 : per;
+}
+
+template <int D, int kPaged>
+cudaError_t launch(const AttnArgs& a, cudaStream_t stream) {
+  const long long problems = (long long)a.B * a.Hp;
+  const int list_len = a.idx ? topk_count(a.N, a.num, a.den) : a.N;
+  // few keys per CTA: every warp's slices issued up front, two CTAs per SM
+  const int cs = decode_cluster_size<D, 0 | kPaged>(problems);
+  const int per = share_of(list_len, cs);
   if ((a.G * D) % cs != 0) return cudaErrorInvalidValue;
-  return per <= 2 * 16 * kWarps ? launch_cs<D, false>(a, cs, per, stream) : launch_cs<D, true>(a, cs, per, stream);
+  if (per <= 2 * 16 * kWarps) return launch_cs<D, 0 | kPaged>(a, cs, per, stream);
+  // many keys per CTA: bulk-copied stages, one CTA per SM
+  const int csb = decode_cluster_size<D, 2 | kPaged>(problems);
+  if ((a.G * D) % csb != 0) return cudaErrorInvalidValue;
+  return launch_cs<D, 2 | kPaged>(a, csb, share_of(list_len, csb), stream);
 }
 
 }  // namespace
 
 cudaError_t launch_decode_attn(const AttnArgs& a, cudaStream_t stream) {
-  return a.D == 128 ? launch<128>(a, stream) : launch<64>(a, stream);
+  if (a.page_table) return a.D == 128 ? launch<128, kPagedBit>(a, stream) : launch<64, kPagedBit>(a, stream);
+  return a.D == 128 ? launch<128, 0>(a, stream) : launch<64, 0>(a, stream);
 }
 
 }  // namespace kascade

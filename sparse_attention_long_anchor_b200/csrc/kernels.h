@@ -143,6 +143,26 @@ cudaError_t launch_pool_mean(const float* in, float* out, int B, int Hkv, int64_
                              cudaStream_t stream);
 
 // decode: one 16-CTA cluster per (batch, kv head), merge over DSMEM
+// Checked copies of index inputs (KASCADE_FLAG_CHECK_INDICES): rows of
+// `row_len` entries, B * L of them (L lists per batch row); decode lists,
+// prefill tile lists (tiles t0 .. T - 1) or refine pools (`pool`: every
+// entry in [0, N)); head_map (n_map entries, in [0, L)) and kv_lens (B
+// entries, NULL = none) copied to hm_out / kv_out.
+struct CheckArgs {
+  const int32_t* idx;
+  int32_t* idx_out;
+  const int32_t* head_map;
+  int32_t* hm_out;
+  int n_map;
+  const int32_t* kv_lens;
+  int32_t* kv_out;
+  int B, L, N, num, den, t0;
+  int64_t row_len;
+  bool prefill, pool, pdl;
+  int* err;
+};
+cudaError_t launch_check_lists(const CheckArgs& c, cudaStream_t stream);
+
 cudaError_t launch_decode_attn(const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill_attn(const AttnArgs& a, cudaStream_t stream);
 // prefill on tcgen05 (G <= 4 or a multiple of 4, d in {64, 128}, tile 32)

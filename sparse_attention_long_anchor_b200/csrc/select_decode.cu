@@ -824,8 +824,8 @@ constexpr int kFusedSizes[] = {16, 12, 10, 9, 8};
 constexpr int kNumFusedSizes = 5;
 
 // Cluster size of the fused kernel for this shape on the current device
-// (choose_cluster_size: fewest waves, then the most CTAs); 0 when the scores
-// do not fit on chip.
+// (fewest waves, then the most CTAs); 0 when the scores do not fit on chip
+// or the problems take more than one wave (choose_fused_select_size).
 template <int D>
 int fused_cluster_size(const SelArgs& a) {
   static int cached[64][kNumFusedSizes] = {{0}};   // max active clusters (+1; 0 = unknown)
@@ -846,7 +846,7 @@ int fused_cluster_size(const SelArgs& a) {
     active[i] = cached[dev][i] - 1;
     fits[i] = ASL<D>::bytes(a.G, fused_per(a.N, kFusedSizes[i])) <= max_smem;
   }
-  return choose_cluster_size((long long)a.B * a.Hp, kFusedSizes, active, fits, kNumFusedSizes);
+  return choose_fused_select_size((long long)a.B * a.Hp, kFusedSizes, active, fits, kNumFusedSizes);
 }
 
 template <int CS, int D>

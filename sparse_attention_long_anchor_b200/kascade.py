@@ -22,8 +22,9 @@ LIB_PATH = os.environ.get("KASCADE_LIB") or os.path.join(os.path.dirname(os.path
 
 OP_SELECT, OP_SPARSE_DECODE, OP_SPARSE_PREFILL, OP_DENSE, OP_REFINE, OP_SELECT_VARLEN = 0, 1, 2, 3, 4, 5
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TOO_LARGE = 0, 1, 2, 3, 4, 5
-FLAG_PDL, FLAG_INPUTS_STABLE, FLAG_TEST_DROP_LOAD = 1, 2, 1 << 30
+FLAG_PDL, FLAG_INPUTS_STABLE, FLAG_CHECK_INDICES, FLAG_TEST_DROP_LOAD = 1, 2, 4, 1 << 30
 DEVERR_SCORE_POOL, DEVERR_DECODE_MERGE, DEVERR_PREFILL_ATTN, DEVERR_DECODE_SELECT = 2, 3, 4, 5
+DEVERR_DECODE_GATHER, DEVERR_INDEX_LIST = 6, 7
 SELECT_GQA, SELECT_PER_HEAD, SELECT_ALL_HEADS = 0, 1, 2
 DTYPE_BF16, DTYPE_F32, DTYPE_F16 = 0, 1, 2
 
@@ -206,7 +207,7 @@ class Workspace:
 
 def _ws(ws, shape, op):
     if ws is None:
-        if op != OP_SELECT:
+        if op != OP_SELECT and not shape.flags & FLAG_CHECK_INDICES:
             return None, 0       # attention calls run without an error word
         ws = Workspace(shape, (op,))
     return ws.args()

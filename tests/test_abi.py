@@ -122,3 +122,32 @@ def test_index_layout_per_selection_mode(mode, lists):
         for sh in (d, p):
             sh.dtype = dt
             assert kc.workspace_bytes(sh, kc.OP_SELECT) > 0
+
+
+def test_index_check_flag_workspace_and_launches():
+    """KASCADE_FLAG_CHECK_INDICES: the attention and refine workspaces grow by
+    the checked copies (lists, head_map, kv_lens), the attention calls count
+    one more launch, and a call without a workspace large enough is refused
+    on the host."""
+    kc = _kc()
+    for q_len, n in ((1, 32768), (4096, 4096), (64, 4096)):
+        s = kc.Shape.make(2, 32, 8, 128, q_len, n)
+        c = s.with_flags(kc.FLAG_CHECK_INDICES)
+        entries = kc.index_count(s)
+        for op in (kc.OP_SPARSE_DECODE, kc.OP_SPARSE_PREFILL):
+            assert kc.workspace_bytes(c, op) >= 256 + 4 * entries + 4 * 32 + 4 * 2
+            assert kc.workspace_bytes(c, op) % 256 == 0
+            assert kc.launch_count(c, op) == 2 and kc.launch_count(s, op) == 1
+        assert kc.workspace_bytes(c, kc.OP_DENSE) == 256 and kc.launch_count(c, kc.OP_DENSE) == 1
+        if q_len == 1:
+            assert kc.workspace_bytes(c, kc.OP_REFINE) >= kc.workspace_bytes(s, kc.OP_REFINE) + 4 * 2 * 8 * n
+    s = kc.Shape.make(1, 8, 2, 64, 1, 256).with_flags(kc.FLAG_CHECK_INDICES)
+    need = kc.workspace_bytes(s, kc.OP_SPARSE_DECODE)
+    L = kc.lib
+    args = (ctypes.byref(s), 256, 256, 256, 256, None, 256, None)
+    assert L.kascade_sparse_decode(*args, None, 0, None) == kc.ERR_WORKSPACE
+    assert L.kascade_sparse_decode(*args, 256, need - 1, None) == kc.ERR_WORKSPACE
+    assert L.kascade_sparse_decode(*args, 258, need, None) == kc.ERR_WORKSPACE
+    p = kc.Shape.make(1, 8, 2, 64, 256, 256).with_flags(kc.FLAG_CHECK_INDICES)
+    assert L.kascade_sparse_prefill(ctypes.byref(p), 256, 256, 256, 256, None, 256, None, None, 0, None) \
+        == kc.ERR_WORKSPACE

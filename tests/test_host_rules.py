@@ -5,7 +5,9 @@ choose_cluster_size (csrc/cluster_choice.h) picks the cluster size of the fused
 decode select: the fewest waves of (batch, kv head) clusters, then the largest
 size.  The active-cluster counts below are the ones the occupancy query
 reports on a 148-SM B200 at one CTA per SM (15 clusters of 8 or 9 CTAs, 11 of
-10, 7 of 12 or 16)."""
+10, 7 of 12 or 16).  choose_fused_select_size keeps that choice only when all
+problems run in one wave (else the library scores in one kernel and selects
+in a second)."""
 import os
 import shutil
 import subprocess
@@ -46,6 +48,55 @@ def _program() -> str:
         lines.append('    std::printf("%%d\\n", kascade::choose_cluster_size(%dLL, sizes, a, f, 5)); }' % p)
     lines += ["  return 0;", "}"]
     return "\n".join(lines) + "\n"
+
+
+# (problems, active, fits, expected) for choose_fused_select_size: the same
+# choice, kept only when every problem runs in one wave
+FUSED_CASES = [
+    (1, B200_ACTIVE, [1] * 5, 16),
+    (7, B200_ACTIVE, [1] * 5, 16),
+    (8, B200_ACTIVE, [1] * 5, 10),      # the Llama-shaped layer at batch 1: fused
+    (15, B200_ACTIVE, [1] * 5, 9),      # 15 clusters of 9 run at once
+    (16, B200_ACTIVE, [1] * 5, 0),      # two waves: scoring kernel + select
+    (64, B200_ACTIVE, [1] * 5, 0),      # batch 8: five waves
+    (4, B200_ACTIVE, [0, 0, 0, 0, 1], 8),
+    (16, B200_ACTIVE, [0, 0, 0, 0, 1], 0),
+    (4, [0] * 5, [1] * 5, 0),
+]
+
+
+def _compile_and_run(tmp_path_factory, body):
+    cxx = shutil.which("g++") or shutil.which("c++")
+    if cxx is None:
+        pytest.skip("no host C++ compiler")
+    d = tmp_path_factory.mktemp("host_rules")
+    src, exe = d / "t.cpp", d / "t"
+    src.write_text(body)
+    subprocess.run([cxx, "-std=c++17", "-O1", "-I", CSRC, str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    return [int(x) for x in out]
+
+
+def _fused_program() -> str:
+    lines = ['#include <cstdio>', '#include "cluster_choice.h"', "int main() {",
+             "  const int sizes[5] = {%s};" % ", ".join(map(str, SIZES))]
+    for p, act, fits, _ in FUSED_CASES:
+        lines.append("  { const int a[5] = {%s}; const bool f[5] = {%s};"
+                     % (", ".join(map(str, act)), ", ".join("true" if x else "false" for x in fits)))
+        lines.append('    std::printf("%%d\\n", kascade::choose_fused_select_size(%dLL, sizes, a, f, 5)); }' % p)
+    lines += ["  return 0;", "}"]
+    return "\n".join(lines) + "\n"
+
+
+@pytest.fixture(scope="module")
+def fused_chosen(tmp_path_factory):
+    return _compile_and_run(tmp_path_factory, _fused_program())
+
+
+@pytest.mark.parametrize("case", range(len(FUSED_CASES)))
+def test_fused_select_one_wave_rule(fused_chosen, case):
+    problems, active, fits, expected = FUSED_CASES[case]
+    assert fused_chosen[case] == expected, (problems, active, fits)
 
 
 @pytest.fixture(scope="module")
