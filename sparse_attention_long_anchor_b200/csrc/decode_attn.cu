@@ -267,24 +267,36 @@ __global__ void __launch_bounds__(kThreads, (kMode & 3) == 2 ? 1 : 2) decode_att
   const char* qrow = smem + L::qs + (size_t)(g * D + 8 * c) * 2;
 
   // bulk mode: this warp's slices warp, warp + kWarps, ..., the it-th in
-  // stage it % kStagesB; K rows by lanes 0-15, V rows by lanes 16-31, rows
-  // past the list repeating its last key (finite data, masked out)
+  // stage it % kStagesB, rows past the list repeating its last key (finite
+  // data, masked out).  The two tensors take different copy engines, which
+  // each sustain only so many row-sized requests per SM: K rows by one bulk
+  // copy each (lanes 0-15, completing on the stage's mbarrier), V rows by
+  // 16-byte cp.async (every lane, one commit group per stage).
   const int n_my = warp < n_slices ? (n_slices - warp + kWarps - 1) / kWarps : 0;
   [[maybe_unused]] auto issue_bulk = [&](int it) {
     using B = BLay<D>;
     const int sl = warp + kWarps * it;
     const int st = it % kStagesB;
     const uint32_t sb = sbar0 + 8 * st;
-    if (lane == 0) mbar_arrive_expect_tx(sb, (uint32_t)(2 * 16 * B::ROWB));
+    const uint32_t kdst = wbase + (uint32_t)(st * B::STAGE);
+    if (lane == 0) mbar_arrive_expect_tx(sb, (uint32_t)(16 * B::ROWB));
     __syncwarp();
-    const int r = lane & 15;
-    const int rel = min(sl * 16 + r, c1 - c0 - 1);
-    bulk_g2s(wbase + (uint32_t)(st * B::STAGE + (lane < 16 ? 0 : B::TB) + r * B::PITCH),
-             (lane < 16 ? kb : vb) + row_off(key_of(rel)), (uint32_t)B::ROWB, sb);
+    const unsigned long long off = row_off(key_of(min(sl * 16 + (lane & 15), c1 - c0 - 1)));
+    if (lane < 16) bulk_g2s(kdst + lane * B::PITCH, kb + off, (uint32_t)B::ROWB, sb);
+#pragma unroll
+    for (int i = 0; i < CH / 2; ++i) {   // 16 rows x CH chunks over 32 lanes
+      const int e = lane + 32 * i;
+      const int r = e / CH, ch = e - r * CH;
+      const unsigned long long ro = __shfl_sync(0xffffffffu, off, r);
+      cp_async_16(kdst + (uint32_t)(B::TB + r * B::PITCH + ch * 16), vb + ro + ch * 8, 16);
+    }
   };
 
   if constexpr (kBulk) {
-    for (int j = 0; j < kStagesB && j < n_my; ++j) issue_bulk(j);
+    for (int j = 0; j < kStagesB; ++j) {
+      if (j < n_my) issue_bulk(j);
+      cp_async_commit();   // one group per stage, empty past the warp's slices
+    }
   } else {
     // prologue: this warp's first two slices
     if (warp < n_slices) issue_rows(warp, wbase, vb, false);
@@ -510,14 +522,18 @@ __global__ void __launch_bounds__(kThreads, (kMode & 3) == 2 ? 1 : 2) decode_att
     bool failed = false;
     for (; it < n_my; ++it) {
       const int st = it % kStagesB;
-      if (!mbar_wait_bounded(sbar0 + 8 * st, (uint32_t)((it / kStagesB) & 1))) {
+      // warp-uniform verdict, so that no lane reaches a warp-wide step alone
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(sbar0 + 8 * st, (uint32_t)((it / kStagesB) & 1)))) {
         if (lane == 0) raise_error(a.err, kErrGather);
         failed = true;
         break;
       }
+      cp_async_wait<kStagesB - 1>();   // this lane's V chunks of stage st
+      __syncwarp();                    // ... and every other lane's
       step_bulk(warp + kWarps * it, st);
       __syncwarp();   // every lane is done with stage st
       if (it + kStagesB < n_my) issue_bulk(it + kStagesB);
+      cp_async_commit();
     }
     // after a wait gave up: let the copies still in flight land (bounded)
     // before the stages become the merge's scratch
