@@ -88,6 +88,24 @@ __device__ __forceinline__ void clear_hist(SelShared& sh) {
   __syncthreads();
 }
 
+// f(j, v[j]) for j = tid, tid + NT, ... < n.  The loads of kBatch indices
+// are issued before any of them is used, so a thread waits on the memory
+// latency once per batch rather than once per element (each pass over a
+// problem's scores is otherwise a chain of dependent L2 round trips).
+constexpr int kBatch = 8;
+template <int NT, class F>
+__device__ __forceinline__ void for_each_value(const float* v, int n, F&& f) {
+  int j = threadIdx.x;
+  for (; j + (kBatch - 1) * NT < n; j += kBatch * NT) {
+    float x[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) x[u] = v[j + u * NT];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) f(j + u * NT, x[u]);
+  }
+  for (; j < n; j += NT) f(j, v[j]);
+}
+
 // Problem description handed to the per-problem routine.
 struct Problem {
   int b, h, t;
@@ -217,7 +235,7 @@ __device__ void run_problem(const SelArgs& a, Problem& p, SelShared& sh, float* 
     }
     v = vscr;
   } else {
-    for (int j = tid; j < p.n; j += NT) atomicAdd(&sh.hist[__float_as_uint(v[j]) >> 21], 1u);
+    for_each_value<NT>(v, p.n, [&](int, float x) { atomicAdd(&sh.hist[__float_as_uint(x) >> 21], 1u); });
   }
   __syncthreads();
 
@@ -229,20 +247,20 @@ __device__ void run_problem(const SelArgs& a, Problem& p, SelShared& sh, float* 
   need -= sh.above;
   __syncthreads();
   clear_hist(sh);
-  for (int j = tid; j < p.n; j += NT) {
-    const unsigned x = __float_as_uint(v[j]);
+  for_each_value<NT>(v, p.n, [&](int, float xf) {
+    const unsigned x = __float_as_uint(xf);
     if ((x >> 21) == (prefix >> 21)) atomicAdd(&sh.hist[(x >> 10) & 2047u], 1u);
-  }
+  });
   __syncthreads();
   find_bin<NT>(sh.hist, need, sh);
   prefix |= (unsigned)sh.bin << 10;
   need -= sh.above;
   __syncthreads();
   clear_hist(sh);
-  for (int j = tid; j < p.n; j += NT) {
-    const unsigned x = __float_as_uint(v[j]);
+  for_each_value<NT>(v, p.n, [&](int, float xf) {
+    const unsigned x = __float_as_uint(xf);
     if ((x >> 10) == (prefix >> 10)) atomicAdd(&sh.hist[x & 1023u], 1u);
-  }
+  });
   __syncthreads();
   find_bin<NT>(sh.hist, need, sh);
   prefix |= (unsigned)sh.bin;
@@ -258,15 +276,14 @@ __device__ void run_problem(const SelArgs& a, Problem& p, SelShared& sh, float* 
   }
   __syncthreads();
   int my_hi = 0;
-  for (int j = tid; j < p.n; j += NT) {
-    const float x = v[j];
+  for_each_value<NT>(v, p.n, [&](int j, float x) {
     if (x > hi) {
       ++my_hi;
     } else if (x >= lo) {
       const int pos = atomicAdd(&sh.nb, 1);
       band_idx[pos] = j;
     }
-  }
+  });
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) my_hi += __shfl_xor_sync(0xffffffffu, my_hi, o);
   if (lane == 0) atomicAdd(&sh.chi, my_hi);
@@ -331,19 +348,50 @@ __device__ void run_problem(const SelArgs& a, Problem& p, SelShared& sh, float* 
 
   // ascending compaction
   if (need_tie == 0) {
-    // one scan: thread t owns the consecutive keys [t * kpt, (t + 1) * kpt)
-    const int kpt = (p.n + NT - 1) / NT;
-    const int j0 = min(p.n, tid * kpt), j1 = min(p.n, j0 + kpt);
-    auto flag_of = [&](int j) -> int {
-      const float x = v[j];
-      return x > hi || (x >= lo && state[j] == 1);
+    // warp w owns the consecutive keys [s0, s1) and walks them 32 at a time
+    // (coalesced loads, ballot counts): one pass counts, the warps' counts
+    // give each warp its output offset, a second pass writes
+    constexpr int W = NT / 32;
+    constexpr int C = 4;   // 32-key chunks whose loads are in flight together
+    const int seg = ((p.n + W - 1) / W + 31) & ~31;
+    const int s0 = min(p.n, warp * seg), s1 = min(p.n, s0 + seg);
+    auto flags = [&](int base, uint32_t (&m)[C]) {
+      float x[C];
+#pragma unroll
+      for (int u = 0; u < C; ++u) {
+        const int j = base + 32 * u + lane;
+        x[u] = j < s1 ? v[j] : 0.0f;
+      }
+#pragma unroll
+      for (int u = 0; u < C; ++u) {
+        const int j = base + 32 * u + lane;
+        const bool f = j < s1 && (x[u] > hi || (x[u] >= lo && state[j] == 1));
+        m[u] = __ballot_sync(0xffffffffu, f);
+      }
     };
     int c = 0;
-    for (int j = j0; j < j1; ++j) c += flag_of(j);
-    const int incl = block_inclusive_scan<NT>(c, sh.scan_buf, nullptr);
-    int w = incl - c;
-    for (int j = j0; j < j1; ++j)
-      if (flag_of(j)) p.out[w++] = p.cand ? p.cand[j] : j;
+    for (int base = s0; base < s1; base += 32 * C) {
+      uint32_t m[C];
+      flags(base, m);
+#pragma unroll
+      for (int u = 0; u < C; ++u) c += __popc(m[u]);
+    }
+    if (lane == 0) sh.scan_buf[warp] = c;
+    __syncthreads();
+    int w = 0;
+#pragma unroll
+    for (int u = 0; u < W; ++u) w += u < warp ? sh.scan_buf[u] : 0;
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int base = s0; base < s1; base += 32 * C) {
+      uint32_t m[C];
+      flags(base, m);
+#pragma unroll
+      for (int u = 0; u < C; ++u) {
+        const int j = base + 32 * u + lane;
+        if ((m[u] >> lane) & 1u) p.out[w + __popc(m[u] & lt)] = p.cand ? p.cand[j] : j;
+        w += __popc(m[u]);
+      }
+    }
     return;
   }
   int written = 0, ties_taken = 0;
