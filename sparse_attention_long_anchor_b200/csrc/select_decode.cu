@@ -634,11 +634,10 @@ __global__ void __launch_bounds__(kCNT, 1) anchor_select_kernel(const SelArgs a,
       raise_error(a.err, kErrTimeout);
     const int k0 = r * kRoundKeys, nk = min(kRoundKeys, cnt - k0);
     const uint32_t slot = ring + (uint32_t)((r % kSlots) * L::RB);
-    if (16 * warp < nk) {
-      // S^T for 16 keys: A = K rows g and g + 8 of the group (d-permuted
-      // 16-byte loads), B = q^T; k-step 2s+t takes dims 32s + 8c + 4t + {0..3}
+    const bool have = 16 * warp < nk;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    if (have) {
       const uint32_t row0 = slot + (uint32_t)((16 * warp + g) * D * 2 + 16 * c);
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int s = 0; s < KS; ++s) {
         uint4 ka, kc;
@@ -653,6 +652,13 @@ __global__ void __launch_bounds__(kCNT, 1) anchor_select_kernel(const SelArgs a,
         mma_bf16_16816(acc, a0, qb[s].x, qb[s].y);
         mma_bf16_16816(acc, a1, qb[s].z, qb[s].w);
       }
+    }
+    __syncthreads();
+    if (tid == 0 && r + kSlots < nr) {
+      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+      issue(r + kSlots);
+    }
+    if (have) {
       const int i0 = k0 + 16 * warp + g, i1 = i0 + 8;   // local key indices
       if (i0 < cnt) {
         const float s0 = acc[0] * scale2, s1 = acc[1] * scale2;
@@ -669,12 +675,8 @@ __global__ void __launch_bounds__(kCNT, 1) anchor_select_kernel(const SelArgs a,
         mx1 = fmaxf(mx1, s1);
       }
     }
-    __syncthreads();   // every warp is done with this slot
-    if (tid == 0 && r + kSlots < nr) {
-      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-      issue(r + kSlots);
-    }
   }
+  __syncthreads();
 
   // ---- softmax statistics of every head over the cluster: each CTA
   // publishes its own (max, sum of exp2(s - max)); one exchange, partial sums
