@@ -28,6 +28,19 @@ inline int choose_cluster_size(long long problems, const int* sizes, const int* 
   return best;
 }
 
+// Short-list sparse decode: a launch is latency-bound and, with programmatic
+// dependent launch, the next launch's clusters start early and gather their
+// rows while this one runs, but only if both launches' clusters are resident
+// at once.  So the largest size at which twice the problems fit the device
+// (active >= 2 problems) is taken; if no size allows that, the
+// fewest-waves rule above.
+inline int choose_overlap_cluster_size(long long problems, const int* sizes, const int* active, const bool* fits,
+                                       int n) {
+  for (int i = 0; i < n; ++i)
+    if (fits[i] && active[i] > 0 && (long long)active[i] >= 2 * problems) return sizes[i];
+  return choose_cluster_size(problems, sizes, active, fits, n);
+}
+
 // Waves that `problems` clusters of the chosen size take (0 if `chosen` is
 // not one of sizes[] or none of it runs).
 inline long long cluster_waves(long long problems, const int* sizes, const int* active, int n, int chosen) {

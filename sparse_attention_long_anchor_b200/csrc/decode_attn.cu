@@ -59,7 +59,7 @@ struct Lay {
   static constexpr size_t qs = slabs + (size_t)kWarps * WARPB;   // [8][D] bf16 query rows
   static constexpr size_t idx = qs + 8 * D * 2;
   static constexpr size_t recv_o = idx + IDXN * 4;         // [G*D] f32, written by the peers
-  static constexpr size_t recv_ml = recv_o + 8 * D * 4;    // [16][8] (m, l)
+  static constexpr size_t recv_ml = recv_o + (8 * D + 4 * kMaxCS) * 4;   // [16][8] (m, l)
   static constexpr size_t bar = recv_ml + kMaxCS * 8 * 8;  // mbarrier of the incoming partials
   static constexpr size_t total = bar + 16;
   // after the gather loop, inside the slabs
@@ -97,7 +97,7 @@ struct BLay {
   static constexpr size_t qs = slabs + (size_t)kWarps * WARPB;
   static constexpr size_t idx = qs + 8 * D * 2;
   static constexpr size_t recv_o = idx + IDXN * 4;
-  static constexpr size_t recv_ml = recv_o + 8 * D * 4;
+  static constexpr size_t recv_ml = recv_o + (8 * D + 4 * kMaxCS) * 4;
   static constexpr size_t bar = recv_ml + kMaxCS * 8 * 8;
   static constexpr size_t sbar = bar + 16;                 // [warps][stages] mbarriers of the stages
   static constexpr size_t total = sbar + (size_t)kWarps * kStagesB * 8;
@@ -170,14 +170,17 @@ __global__ void __launch_bounds__(kThreads, (kMode & 3) == 2 ? 1 : 2) decode_att
   const int g = lane >> 2, c = lane & 3;
   const int G = a.G;
   const int E = G * D;
-  const int en = E / CS;              // output elements owned by each CTA (a multiple of 4)
+  // output elements owned by each CTA: en (a multiple of 4) for the first
+  // ones, what is left for the last owner, none past it
+  const int en = ((E + CS - 1) / CS + 3) & ~3;
+  const int en_mine = max(0, min(en, E - rank * en));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar = sbase + (uint32_t)L::bar;
   if (threadIdx.x == 0) {
     mbar_init(bar, 1);
     mbar_fence_init();
-    // every CTA of the cluster sends en outputs and G (m, l) pairs
-    mbar_arrive_expect_tx(bar, (uint32_t)(E * 4 + CS * G * 8));
+    // every CTA of the cluster sends this CTA's en_mine outputs and G (m, l) pairs
+    mbar_arrive_expect_tx(bar, (uint32_t)(CS * en_mine * 4 + CS * G * 8));
   }
   cluster_arrive_release();   // the matching wait comes before the first push
   [[maybe_unused]] const uint32_t sbar0 =
@@ -610,7 +613,7 @@ __global__ void __launch_bounds__(kThreads, (kMode & 3) == 2 ? 1 : 2) decode_att
   const float2* rml = reinterpret_cast<const float2*>(smem + L::recv_ml);
   if (warp < G) merge_weights(CS, rml + warp, wts + warp, head + warp, lane);
   __syncthreads();
-  if ((int)threadIdx.x < en) {
+  if ((int)threadIdx.x < en_mine) {
     const float* ro = reinterpret_cast<const float*>(smem + L::recv_o);
     const int e = rank * en + threadIdx.x;
     const int gg = e / D, dd = e - gg * D;
@@ -641,42 +644,43 @@ cudaLaunchConfig_t make_cfg(int cs, int bh, cudaStream_t stream, cudaLaunchAttri
   return cfg;
 }
 
-// Cluster sizes of the sparse decode, largest first.  One cluster per
-// (batch, list) problem: at batch 1 the largest cluster spreads the gathers
-// widest (the kernel is latency-bound there); with many problems the fewest
-// waves matter (choose_cluster_size).  The bulk mode (one CTA per SM) also
-// takes pairs, so 64 problems still fit one wave.
-constexpr int kDecSizes[] = {16, 8, 4, 2};
-constexpr int kNumDecSizes = 4;
+// Cluster sizes of the sparse decode, largest first; one cluster per
+// (batch, list) problem.  Short lists (mode 0): the largest size at which a
+// launch and its successor are resident together (choose_overlap_cluster_size;
+// on a 148-SM part 14 clusters of 16 fit at two CTAs per SM, so the
+// Llama-shaped layer's 8 problems take 14 CTAs each), among the sizes that
+// keep every warp at two slices or fewer.  Owners of the output elements
+// get equal shares rounded to 4, so a size need not divide G d.  Long lists
+// (the bulk mode, one CTA per SM): the fewest waves, pairs included, so 64
+// problems still fit one wave.
+constexpr int kDecSizes0[] = {16, 15, 14, 13, 12, 10, 8, 4};
+constexpr int kNumDecSizes0 = 8;
+constexpr int kDecSizesB[] = {16, 8, 4, 2};
+constexpr int kNumDecSizesB = 4;
+constexpr int kMaxDecSizes = 8;
 
+// clusters of sizes[i] the device runs at once (cached per device)
 template <int D, int kMode>
-int decode_cluster_size(long long problems) {
-  static int cached[64][kNumDecSizes] = {{0}};   // max active clusters + 1 (0 = unknown)
+const int* decode_active(const int* sizes, int n) {
+  static int cached[64][kMaxDecSizes + 1] = {{0}};   // [0]: 1 once filled
+  static const int none[kMaxDecSizes] = {0};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 8;
-  const int n_sizes = (kMode & 3) == 2 ? kNumDecSizes : kNumDecSizes - 1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return none;
   if (!cached[dev][0]) {
-    for (int i = 0; i < n_sizes; ++i) {
-      const int cs = kDecSizes[i];
-      int n = 0;
+    for (int i = 0; i < n; ++i) {
+      int m = 0;
       if (ensure_func_attrs(reinterpret_cast<const void*>(decode_attn_kernel<D, kMode>), LayOf<D, kMode>::total,
-                            cs > 8) == cudaSuccess) {
+                            sizes[i] > 8) == cudaSuccess) {
         cudaLaunchAttribute attr[1];
-        cudaLaunchConfig_t cfg = make_cfg<D, kMode>(cs, 1, nullptr, attr);
-        if (cudaOccupancyMaxActiveClusters(&n, decode_attn_kernel<D, kMode>, &cfg) != cudaSuccess) n = 0;
+        cudaLaunchConfig_t cfg = make_cfg<D, kMode>(sizes[i], 1, nullptr, attr);
+        if (cudaOccupancyMaxActiveClusters(&m, decode_attn_kernel<D, kMode>, &cfg) != cudaSuccess) m = 0;
       }
-      cached[dev][i] = 1 + n;
+      cached[dev][1 + i] = m;
     }
     cudaGetLastError();
+    cached[dev][0] = 1;
   }
-  int active[kNumDecSizes];
-  bool fits[kNumDecSizes];
-  for (int i = 0; i < n_sizes; ++i) {
-    active[i] = cached[dev][i] - 1;
-    fits[i] = true;
-  }
-  const int cs = choose_cluster_size(problems, kDecSizes, active, fits, n_sizes);
-  return cs > 0 ? cs : 8;
+  return &cached[dev][1];
 }
 
 template <int D, int kMode>
@@ -699,13 +703,18 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t stream) {
   const long long problems = (long long)a.B * a.Hp;
   const int list_len = a.idx ? topk_count(a.N, a.num, a.den) : a.N;
   // few keys per CTA: every warp's slices issued up front, two CTAs per SM
-  const int cs = decode_cluster_size<D, 0 | kPaged>(problems);
-  const int per = share_of(list_len, cs);
-  if ((a.G * D) % cs != 0) return cudaErrorInvalidValue;
-  if (per <= 2 * 16 * kWarps) return launch_cs<D, 0 | kPaged>(a, cs, per, stream);
+  {
+    const int* act = decode_active<D, 0 | kPaged>(kDecSizes0, kNumDecSizes0);
+    bool fits[kNumDecSizes0];
+    for (int i = 0; i < kNumDecSizes0; ++i) fits[i] = share_of(list_len, kDecSizes0[i]) <= 2 * 16 * kWarps;
+    const int cs = choose_overlap_cluster_size(problems, kDecSizes0, act, fits, kNumDecSizes0);
+    if (cs > 0) return launch_cs<D, 0 | kPaged>(a, cs, share_of(list_len, cs), stream);
+  }
   // many keys per CTA: bulk-copied stages, one CTA per SM
-  const int csb = decode_cluster_size<D, 2 | kPaged>(problems);
-  if ((a.G * D) % csb != 0) return cudaErrorInvalidValue;
+  const int* act = decode_active<D, 2 | kPaged>(kDecSizesB, kNumDecSizesB);
+  const bool fits[kNumDecSizesB] = {true, true, true, true};
+  int csb = choose_cluster_size(problems, kDecSizesB, act, fits, kNumDecSizesB);
+  if (csb <= 0) csb = 8;
   return launch_cs<D, 2 | kPaged>(a, csb, share_of(list_len, csb), stream);
 }
 

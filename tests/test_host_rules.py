@@ -99,6 +99,44 @@ def test_fused_select_one_wave_rule(fused_chosen, case):
     assert fused_chosen[case] == expected, (problems, active, fits)
 
 
+# choose_overlap_cluster_size over the short-list decode's sizes: the largest
+# size at which twice the problems are resident, else the fewest waves
+SIZES0 = [16, 15, 14, 13, 12, 10, 8, 4]
+ACT0 = [14, 15, 17, 18, 21, 22, 33, 71]          # a plausible two-CTAs-per-SM device
+FIT_LLAMA = [1, 1, 1, 1, 0, 0, 0, 0]             # 3277 keys: 256 per CTA or fewer needs 13 CTAs or more
+OVERLAP_CASES = [
+    (8, ACT0, FIT_LLAMA, 14),      # 14 and 15 < 16: 14 CTAs (17 clusters resident)
+    (8, [14, 16, 17, 18, 21, 22, 33, 71], FIT_LLAMA, 15),
+    (7, ACT0, FIT_LLAMA, 16),      # 14 >= 2 x 7
+    (2, ACT0, [1] * 8, 16),
+    (16, ACT0, FIT_LLAMA, 14),     # nothing holds 32: fewest waves (one at 14 and 13), then the largest
+    (40, ACT0, [1] * 8, 4),        # 71 < 80: fewest waves, one wave only at 4
+    (8, ACT0, [0] * 8, 0),         # no size keeps the short-list mode: the bulk mode runs
+]
+
+
+def _overlap_program() -> str:
+    lines = ['#include <cstdio>', '#include "cluster_choice.h"', "int main() {",
+             "  const int sizes[8] = {%s};" % ", ".join(map(str, SIZES0))]
+    for p, act, fits, _ in OVERLAP_CASES:
+        lines.append("  { const int a[8] = {%s}; const bool f[8] = {%s};"
+                     % (", ".join(map(str, act)), ", ".join("true" if x else "false" for x in fits)))
+        lines.append('    std::printf("%%d\\n", kascade::choose_overlap_cluster_size(%dLL, sizes, a, f, 8)); }' % p)
+    lines += ["  return 0;", "}"]
+    return "\n".join(lines) + "\n"
+
+
+@pytest.fixture(scope="module")
+def overlap_chosen(tmp_path_factory):
+    return _compile_and_run(tmp_path_factory, _overlap_program())
+
+
+@pytest.mark.parametrize("case", range(len(OVERLAP_CASES)))
+def test_decode_overlap_rule(overlap_chosen, case):
+    problems, active, fits, expected = OVERLAP_CASES[case]
+    assert overlap_chosen[case] == expected, (problems, active, fits)
+
+
 @pytest.fixture(scope="module")
 def chosen(tmp_path_factory):
     cxx = shutil.which("g++") or shutil.which("c++")
