@@ -32,13 +32,16 @@ inline int choose_cluster_size(long long problems, const int* sizes, const int* 
 // dependent launch, the next launch's clusters start early and gather their
 // rows while this one runs, but only if both launches' clusters are resident
 // at once.  So the largest size at which twice the problems fit the device
-// (active >= 2 problems) is taken; if no size allows that, the
-// fewest-waves rule above.
+// (active >= 2 problems) is taken; else the largest at which all problems
+// run in one wave; else 0 (the caller's long-list mode, which moves more
+// keys per CTA, takes over).
 inline int choose_overlap_cluster_size(long long problems, const int* sizes, const int* active, const bool* fits,
                                        int n) {
   for (int i = 0; i < n; ++i)
     if (fits[i] && active[i] > 0 && (long long)active[i] >= 2 * problems) return sizes[i];
-  return choose_cluster_size(problems, sizes, active, fits, n);
+  for (int i = 0; i < n; ++i)
+    if (fits[i] && active[i] > 0 && (long long)active[i] >= problems) return sizes[i];
+  return 0;
 }
 
 // Waves that `problems` clusters of the chosen size take (0 if `chosen` is

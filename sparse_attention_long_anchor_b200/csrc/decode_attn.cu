@@ -646,10 +646,10 @@ cudaLaunchConfig_t make_cfg(int cs, int bh, cudaStream_t stream, cudaLaunchAttri
 
 // Cluster sizes of the sparse decode, largest first; one cluster per
 // (batch, list) problem.  Short lists (mode 0): the largest size at which a
-// launch and its successor are resident together (choose_overlap_cluster_size;
-// on a 148-SM part 14 clusters of 16 fit at two CTAs per SM, so the
-// Llama-shaped layer's 8 problems take 14 CTAs each), among the sizes that
-// keep every warp at two slices or fewer.  Owners of the output elements
+// launch and its successor are resident together, else the largest with one
+// wave (choose_overlap_cluster_size), among the sizes that keep every warp
+// at two slices or fewer; on a 148-SM part 14 clusters of 16 fit at two
+// CTAs per SM, so the Llama-shaped layer's 8 problems take 13 CTAs each.  Owners of the output elements
 // get equal shares rounded to 4, so a size need not divide G d.  Long lists
 // (the bulk mode, one CTA per SM): the fewest waves, pairs included, so 64
 // problems still fit one wave.

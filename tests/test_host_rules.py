@@ -100,7 +100,8 @@ def test_fused_select_one_wave_rule(fused_chosen, case):
 
 
 # choose_overlap_cluster_size over the short-list decode's sizes: the largest
-# size at which twice the problems are resident, else the fewest waves
+# size at which twice the problems are resident, else the largest with one
+# wave, else 0 (the bulk mode)
 SIZES0 = [16, 15, 14, 13, 12, 10, 8, 4]
 ACT0 = [14, 15, 17, 18, 21, 22, 33, 71]          # a plausible two-CTAs-per-SM device
 FIT_LLAMA = [1, 1, 1, 1, 0, 0, 0, 0]             # 3277 keys: 256 per CTA or fewer needs 13 CTAs or more
@@ -109,8 +110,9 @@ OVERLAP_CASES = [
     (8, [14, 16, 17, 18, 21, 22, 33, 71], FIT_LLAMA, 15),
     (7, ACT0, FIT_LLAMA, 16),      # 14 >= 2 x 7
     (2, ACT0, [1] * 8, 16),
-    (16, ACT0, FIT_LLAMA, 14),     # nothing holds 32: fewest waves (one at 14 and 13), then the largest
-    (40, ACT0, [1] * 8, 4),        # 71 < 80: fewest waves, one wave only at 4
+    (16, ACT0, FIT_LLAMA, 14),     # nothing holds 32: the largest size with one wave
+    (40, ACT0, [1] * 8, 4),        # 71 < 80: one wave only at 4
+    (64, ACT0, FIT_LLAMA, 0),      # batch 8 of the Llama layer: no one-wave size, the bulk mode runs
     (8, ACT0, [0] * 8, 0),         # no size keeps the short-list mode: the bulk mode runs
 ]
 
