@@ -566,7 +566,42 @@ def dense_denominators(kc, torch, dec, pre, reps):
         flops = 4 * pcfg.hq * pcfg.d * sum(min(32 * (i + 1), pcfg.n_ctx) for i in range(-(-pcfg.n_ctx // 32))) * 32
         out[PREFILL_CFG] = {"dense_causal_ms_per_layer": mean(t), "flops_per_layer": flops,
                             "tflops": flops / (mean(t) * 1e-3) / 1e12}
+    torch_sdpa_context(torch, dec, pre, reps, out)
     return out
+
+
+def torch_sdpa_context(torch, dec, pre, reps, out):
+    """For context beside the library's own dense path: PyTorch's
+    scaled_dot_product_attention (whatever backend it picks on this device)
+    on the same decode layers (grouped query heads) and on one prefill layer
+    (causal; K and V expanded to the query heads outside the timed region).
+    A library kernel, not this library's path; None where it fails."""
+    import torch.nn.functional as F
+    dcfg = dec["cfg"]
+    try:
+        layers = dec["layers"]
+        g = capture(torch, lambda: [F.scaled_dot_product_attention(*layers[l], enable_gqa=True)
+                                    for l in range(dcfg.n_layers)])
+        t = time_graph(torch, g, reps)
+        del g
+        out[DECODE_CFG]["torch_sdpa_us_per_layer"] = mean(t) * 1e3 / dcfg.n_layers
+    except Exception as e:   # noqa: BLE001 - context only
+        out[DECODE_CFG]["torch_sdpa_us_per_layer"] = None
+        out[DECODE_CFG]["torch_sdpa_error"] = str(e).splitlines()[0][:200]
+    if pre is None:
+        return
+    try:
+        q, k, v = pre["layers"][1]
+        rep = q.shape[1] // k.shape[1]
+        ke, ve = k.repeat_interleave(rep, dim=1), v.repeat_interleave(rep, dim=1)
+        g = capture(torch, lambda: F.scaled_dot_product_attention(q, ke, ve, is_causal=True))
+        t = time_graph(torch, g, 3)
+        del g, ke, ve
+        out[PREFILL_CFG]["torch_sdpa_causal_ms_per_layer"] = mean(t)
+    except Exception as e:   # noqa: BLE001 - context only
+        out[PREFILL_CFG]["torch_sdpa_causal_ms_per_layer"] = None
+        out[PREFILL_CFG]["torch_sdpa_error"] = str(e).splitlines()[0][:200]
+    torch.cuda.empty_cache()
 
 
 def run_kascade(args, rank, world, local):
@@ -649,9 +684,15 @@ def run_kascade(args, rank, world, local):
     dense = dense_denominators(kc, torch, dec, pre, reps)
     dense[DECODE_CFG]["sparse_us_per_layer_step"] = headline["us_per_layer_step"]
     dense[DECODE_CFG]["speedup"] = dense[DECODE_CFG]["dense_us_per_layer"] / headline["us_per_layer_step"]
+    sd = dense[DECODE_CFG].get("torch_sdpa_us_per_layer")
+    if sd:
+        dense[DECODE_CFG]["speedup_vs_torch_sdpa"] = sd / headline["us_per_layer_step"]
     if pre is not None:
         dense[PREFILL_CFG]["sparse_ms_per_layer"] = prefill_obj["value"]
         dense[PREFILL_CFG]["speedup"] = dense[PREFILL_CFG]["dense_causal_ms_per_layer"] / prefill_obj["value"]
+        sp = dense[PREFILL_CFG].get("torch_sdpa_causal_ms_per_layer")
+        if sp:
+            dense[PREFILL_CFG]["speedup_vs_torch_sdpa"] = sp / prefill_obj["value"]
 
     # ---- end to end through the public API: the step's queries (every
     # layer's q, one pinned host buffer) copied in, the layers run, the step's
