@@ -34,6 +34,7 @@
 #include "cluster_choice.h"
 #include "common.cuh"
 #include "kernels.h"
+#include "tc.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -119,6 +120,12 @@ struct BLay {
 // they are consumed (one CTA per SM).  Bit 2 (kPagedBit): rows addressed
 // through a page table.
 constexpr int kPagedBit = 4;
+// kMode bit 4 (bulk mode, contiguous cache, no index list: the dense form):
+// a slice's 16 consecutive rows arrive as one 128-byte-swizzled TMA tile per
+// 64 columns of K and of V, instead of one request per row
+constexpr int kDenseBit = 16;
+template <int D>
+constexpr int kDenseStage = 2 * 16 * D * 2;   // K (16 rows) then V, each as 2 KB tiles of 64 columns
 template <int D, int kMode>
 using LayOf = typename std::conditional<(kMode & 3) == 2, BLay<D>, Lay<D>>::type;
 
@@ -147,10 +154,16 @@ __device__ __forceinline__ void merge_weights(int n, const float2* ml, float* w,
 // refilled as they are consumed (one CTA per SM, for many keys per CTA).
 // kMode & kPagedBit: K and V rows through the page table.
 template <int D, int kMode>
-__global__ void __launch_bounds__(kThreads, (kMode & 3) == 2 ? 1 : 2) decode_attn_kernel(const AttnArgs a, int per) {
+__global__ void __launch_bounds__(kThreads, (kMode & 3) == 2 ? 1 : 2)
+    decode_attn_kernel(const AttnArgs a, int per, const __grid_constant__ CUtensorMap mk,
+                       const __grid_constant__ CUtensorMap mv) {
   using L = LayOf<D, kMode>;
   constexpr bool kBulk = (kMode & 3) == 2;
   constexpr bool kPaged = (kMode & kPagedBit) != 0;
+  constexpr bool kDense = (kMode & kDenseBit) != 0;
+  static_assert(!kDense || (kBulk && !kPaged), "the tile form serves the contiguous bulk mode");
+  static_assert(!kDense || 1023 + kWarps * kStagesB * kDenseStage<D> <= kWarps * BLay<D>::WARPB,
+                "aligned tile stages fit the stage region");
   constexpr int KS = D / 32;          // 16-byte K loads per key row per lane
   constexpr int CH = D / 8;           // 16-byte chunks per row
   extern __shared__ __align__(128) char smem[];
@@ -276,11 +289,29 @@ __global__ void __launch_bounds__(kThreads, (kMode & 3) == 2 ? 1 : 2) decode_att
   // copy each (lanes 0-15, completing on the stage's mbarrier), V rows by
   // 16-byte cp.async (every lane, one commit group per stage).
   const int n_my = warp < n_slices ? (n_slices - warp + kWarps - 1) / kWarps : 0;
+  // the tile form: stages 1024-byte aligned (the swizzle repeats every 8
+  // rows of 128 bytes), inside the stage region the index staging leaves free
+  [[maybe_unused]] const uint32_t dbase =
+      ((sbase + 1023u) & ~1023u) + (uint32_t)(warp * kStagesB * kDenseStage<D>);
+  [[maybe_unused]] const int dslab = (int)slab;
   [[maybe_unused]] auto issue_bulk = [&](int it) {
     using B = BLay<D>;
     const int sl = warp + kWarps * it;
     const int st = it % kStagesB;
     const uint32_t sb = sbar0 + 8 * st;
+    if constexpr (kDense) {
+      if (lane == 0) {
+        const uint32_t kd = dbase + (uint32_t)(st * kDenseStage<D>), vd = kd + kDenseStage<D> / 2;
+        const int row = c0 + sl * 16;   // rows past the list are masked, past the slab read zeros
+        mbar_arrive_expect_tx(sb, (uint32_t)(2 * 16 * D * 2));
+#pragma unroll
+        for (int bx = 0; bx < D / 64; ++bx) {
+          tc::tma_load_3d(kd + (uint32_t)(bx * 2048), &mk, bx * 64, row, dslab, sb);
+          tc::tma_load_3d(vd + (uint32_t)(bx * 2048), &mv, bx * 64, row, dslab, sb);
+        }
+      }
+      return;
+    }
     const uint32_t kdst = wbase + (uint32_t)(st * B::STAGE);
     if (lane == 0) mbar_arrive_expect_tx(sb, (uint32_t)(16 * B::ROWB));
     __syncwarp();
@@ -466,8 +497,16 @@ __global__ void __launch_bounds__(kThreads, (kMode & 3) == 2 ? 1 : 2) decode_att
   // order above; the query rows read with the same chunk order)
   [[maybe_unused]] auto step_bulk = [&](int sl, int st) {
     using B = BLay<D>;
-    const uint32_t kst = wbase + (uint32_t)(st * B::STAGE);
-    const uint32_t vst = kst + (uint32_t)B::TB;
+    const uint32_t kst = kDense ? dbase + (uint32_t)(st * kDenseStage<D>) : wbase + (uint32_t)(st * B::STAGE);
+    const uint32_t vst = kDense ? kst + kDenseStage<D> / 2 : kst + (uint32_t)B::TB;
+    // 16-byte chunk ch of row r: pitch-padded rows, or the tile form's
+    // swizzled 64-column tiles
+    auto chunk_at = [&](uint32_t base, int r, int ch) -> uint32_t {
+      if constexpr (kDense)
+        return base + (uint32_t)((ch >> 3) * 2048 + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
+      else
+        return base + (uint32_t)(r * B::PITCH + ch * 16);
+    };
     const char* qg = smem + L::qs + (size_t)(g * D) * 2;
     float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -475,8 +514,8 @@ __global__ void __launch_bounds__(kThreads, (kMode & 3) == 2 ? 1 : 2) decode_att
       const int ch = 8 * (q >> 1) + 2 * c + (q & 1);
       const uint2 qlo = *reinterpret_cast<const uint2*>(qg + ch * 16);
       const uint2 qhi = *reinterpret_cast<const uint2*>(qg + ch * 16 + 8);
-      const uint4 k0 = lds_v4(kst + g * B::PITCH + ch * 16);
-      const uint4 k1 = lds_v4(kst + (8 + g) * B::PITCH + ch * 16);
+      const uint4 k0 = lds_v4(chunk_at(kst, g, ch));
+      const uint4 k1 = lds_v4(chunk_at(kst, 8 + g, ch));
       const uint32_t a0[4] = {k0.x, k1.x, k0.y, k1.y};
       const uint32_t a1[4] = {k0.z, k1.z, k0.w, k1.w};
       mma_bf16_16816(q & 1 ? sb : sa, a0, qlo.x, qlo.y);
@@ -510,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, (kMode & 3) == 2 ? 1 : 2) decode_att
 #pragma unroll
     for (int i = 0; i < D / 16; ++i) {
       uint32_t r4[4];
-      ldmatrix_x4_trans(r4, vst + vrow * B::PITCH + (2 * i + vch) * 16);
+      ldmatrix_x4_trans(r4, chunk_at(vst, vrow, 2 * i + vch));
       float t[4] = {oacc[i][0] * al0, oacc[i][1] * al1, oacc[i][2] * al0, oacc[i][3] * al1};
       mma_bf16_16816(t, r4, b0, b1);
       oacc[i][0] = t[0];
@@ -688,8 +727,16 @@ cudaError_t launch_cs(const AttnArgs& a, int cs, int per, cudaStream_t stream) {
   const size_t smem = LayOf<D, kMode>::total;
   const cudaError_t e = ensure_func_attrs(reinterpret_cast<const void*>(decode_attn_kernel<D, kMode>), smem, cs > 8);
   if (e != cudaSuccess) return e;
+  // K and V as [B Hkv][N][D] in tiles of 16 rows x 64 columns (the tile
+  // form reads them; the other forms get the maps unused)
+  CUtensorMap mk{}, mv{};
+  if constexpr ((kMode & kDenseBit) != 0) {
+    if (!tc::make_map_3d(&mk, a.k, (uint64_t)D, (uint64_t)a.N, (uint64_t)a.B * a.Hkv, 16) ||
+        !tc::make_map_3d(&mv, a.v, (uint64_t)D, (uint64_t)a.N, (uint64_t)a.B * a.Hkv, 16))
+      return cudaErrorInvalidValue;
+  }
   return launch_ex(decode_attn_kernel<D, kMode>, dim3(cs, a.B * a.Hp), dim3(kThreads), smem, stream,
-                   (a.flags & 1) != 0, cs, a, per);
+                   (a.flags & 1) != 0, cs, a, per, mk, mv);
 }
 
 int share_of(int list_len, int cs) {
@@ -710,11 +757,15 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t stream) {
     const int cs = choose_overlap_cluster_size(problems, kDecSizes0, act, fits, kNumDecSizes0);
     if (cs > 0) return launch_cs<D, 0 | kPaged>(a, cs, share_of(list_len, cs), stream);
   }
-  // many keys per CTA: bulk-copied stages, one CTA per SM
+  // many keys per CTA: bulk-copied stages, one CTA per SM; the dense form
+  // of a contiguous cache as whole tiles
   const int* act = decode_active<D, 2 | kPaged>(kDecSizesB, kNumDecSizesB);
   const bool fits[kNumDecSizesB] = {true, true, true, true};
   int csb = choose_cluster_size(problems, kDecSizesB, act, fits, kNumDecSizesB);
   if (csb <= 0) csb = 8;
+  if constexpr (kPaged == 0) {
+    if (!a.idx) return launch_cs<D, 2 | kDenseBit>(a, csb, share_of(list_len, csb), stream);
+  }
   return launch_cs<D, 2 | kPaged>(a, csb, share_of(list_len, csb), stream);
 }
 

@@ -89,10 +89,15 @@ def test_decode_zero_query_ties_go_to_lowest_index():
     assert np.array_equal(idx_g[0, 0], np.arange(kk)) and np.array_equal(idx_g[0, 1], np.arange(kk))
 
 
-def test_dense_decode():
+@pytest.mark.parametrize("B,Hq,Hkv,d,N", [
+    (2, 16, 4, 128, 5000),     # long lists: contiguous rows as whole 16-row tiles, ragged tail
+    (1, 8, 2, 64, 9001),       # d = 64: one tile per row block
+    (1, 32, 8, 128, 32768),    # the Llama-shaped layer, the dense denominator of the benchmark
+    (1, 8, 2, 128, 700),       # short lists: the up-front form
+])
+def test_dense_decode(B, Hq, Hkv, d, N):
     kc = _kc()
-    B, Hq, Hkv, d, N = 2, 16, 4, 128, 5000
-    q, k, v = gen_inputs(dict(B=B, Hq=Hq, Hkv=Hkv, d=d, N=N), seed=5)
+    q, k, v = gen_inputs(dict(B=B, Hq=Hq, Hkv=Hkv, d=d, N=N), seed=5 + N)
     s = kc.Shape.make(B, Hq, Hkv, d, 1, N)
     lse = torch.empty(B, Hq, device="cuda")
     o = kc.dense_ref(s, q, k, v, lse=lse, ws=kc.Workspace(s, (kc.OP_DENSE,)))
