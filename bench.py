@@ -651,6 +651,11 @@ def run_kascade(args, rank, world, local):
     pre_steps = [e1.elapsed_time(e2) for _, e1, e2 in ev] if g_pre is not None else []
     dec_ms = dist_max(mean(dec_steps), world)
     pre_ms = dist_max(mean(pre_steps), world) if pre_steps else 0.0
+    # the decode step's spread over 100 further replays (10 untimed first),
+    # apart from the timed steps above
+    for _ in range(10):
+        g_dec.replay()
+    replays_100 = spread(time_graph(torch, g_dec, 100))
     del g_dec, g_pre
 
     # ---- per-kernel components of the headline stack (CUDA events over
@@ -666,6 +671,7 @@ def run_kascade(args, rank, world, local):
                 "us_per_launch": comp["sparse_decode_us_per_launch"]}
     sb = step_bytes_decode(dcfg)
     headline = {"us_per_layer_step": dec_ms * 1e3 / n_dec, "ms_per_step": dec_ms, "step_ms_spread": spread(dec_steps),
+                "step_ms_spread_100_replays": replays_100,
                 "layer_step_GBps": sb / (dec_ms * 1e-3) / 1e9,
                 "layer_step_frac_of_hbm": sb / (dec_ms * 1e-3) / 1e9 / pk["hbm_gbs"], **comp}
     # kernels per step, as the library reports them for these shapes on this device
@@ -724,6 +730,38 @@ def run_kascade(args, rank, world, local):
     t1.record()
     torch.cuda.synchronize()
     e2e_ms = dist_max(t0.elapsed_time(t1) / args.steps, world)
+
+    # prefill end to end through the public API: layer 0's queries copied in
+    # from pinned host memory, the 36 layers as eager calls, the last layer's
+    # output copied back
+    if pre is not None:
+        n_pre = pre["cfg"].n_layers
+        pq = pre["layers"][0][0]
+        po = pre["outs"][n_pre - 1]
+        host_pq = pq.cpu().pin_memory()
+        host_po = torch.empty(po.shape, dtype=po.dtype, pin_memory=True)
+
+        def e2e_prefill_step():
+            pq.copy_(host_pq, non_blocking=True)
+            for l in range(n_pre):
+                run_layer(kc, pre, l)
+            host_po.copy_(po, non_blocking=True)
+
+        e2e_prefill_step()
+        torch.cuda.synchronize()
+        p_steps = max(1, min(args.steps, 3))
+        t0.record()
+        for _ in range(p_steps):
+            e2e_prefill_step()
+        t1.record()
+        torch.cuda.synchronize()
+        pe2e_ms = dist_max(t0.elapsed_time(t1) / p_steps, world)
+        prefill_obj["e2e"] = {"value": pe2e_ms / n_pre, "unit": "ms/layer", "steps": p_steps,
+                              "h2d_bytes_per_step": host_pq.numel() * host_pq.element_size(),
+                              "d2h_bytes_per_step": host_po.numel() * host_po.element_size(),
+                              "path": "eager Python API calls per layer; layer 0's q in and the last layer's o out, "
+                                      "one pinned copy each"}
+        del host_pq, host_po
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
