@@ -66,11 +66,40 @@ def peaks():
                 "source": "fallback"}
 
 
+def strip_comments(src: str) -> str:
+    """C/C++/CUDA source without its comments and blank-line or indentation
+    differences: string and character literals are kept as they are, every
+    comment is dropped, and each remaining line is stripped of surrounding
+    whitespace (empty lines dropped)."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        ch = src[i]
+        if ch in "\"'":
+            j = i + 1
+            while j < n and src[j] != ch:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(ch)
+            i += 1
+    lines = (ln.strip() for ln in "".join(out).splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
 def kernel_source_hash(name: str) -> str:
+    """Hash of a kernel source's code (comments and layout ignored), which
+    keys the stored ncu counters to the code they were taken on."""
     import hashlib
     path = os.path.join(ROOT, "sparse_attention_long_anchor_b200", "csrc", name)
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    with open(path, encoding="utf-8") as f:
+        return hashlib.sha256(strip_comments(f.read()).encode()).hexdigest()[:16]
 
 
 def profiled_traffic(kernel: str):

@@ -45,7 +45,7 @@ namespace {
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kMaxCS = 16;
-constexpr int kIdxStage = 512;      // index entries staged in shared memory, modes 0 and 1
+constexpr int kIdxStage = 512;      // index entries staged in shared memory, short-list mode
 constexpr int kIdxStageB = 3584;    // the bulk mode's (a 2-CTA cluster's share of 64K at 10 %)
 constexpr int kErrMergeTimeout = 3; // device error word: a merge wait gave up
 constexpr int kErrGather = 6;       // device error word: a bulk-copied row never arrived
@@ -92,7 +92,7 @@ struct BLay {
   static constexpr int TB = 16 * PITCH;                    // 16 rows of one tensor
   static constexpr int STAGE = 2 * TB;                     // K rows, then V rows
   static constexpr int WARPB = kStagesB * STAGE;
-  static constexpr int SLAB = 16 * ROWB;                   // (the two-slab modes' unit; unused here)
+  static constexpr int SLAB = 16 * ROWB;                   // (the short-list mode's unit; not used here)
   static constexpr int IDXN = kIdxStageB;
   static constexpr size_t slabs = 0;
   static constexpr size_t qs = slabs + (size_t)kWarps * WARPB;
